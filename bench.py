@@ -1,0 +1,383 @@
+"""Throughput of the expert-choice MoE FFN layer on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--intermediate split|bf16]
+
+A step is one pass of the whole layer (router + softmax, per-expert top-C select, token
+lists, gathered GEMM1 + SwiGLU, GEMM2 + combine weight, fixed-order combine) over one
+batch of seeded synthetic tokens. The default workload is a 1024 px CFG pair: two images
+of 64 x 64 = 4096 patch tokens, T = 8192, d = 2048, 64 experts, F = 1024, C = 128,
+tokens scaled by LogNormal(0, 0.5).
+
+Multi-GPU: expert-choice selection over the flat token axis couples every token, so the
+layer does not shard without changing its result; N GPUs run N independent replicas
+(one batch each, seed = rank), and value = all ranks' tokens / the slowest rank's time.
+
+`--impl reference` times the CPU oracle (fp64 numpy) on this host's cores instead, on
+the same workload and metric (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "expert-choice MoE layer tokens/s & TFLOP/s vs B200 bf16 peak; select/combine GB/s"
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="1024px_cfg")
+    ap.add_argument("--intermediate", choices=("split", "bf16"), default="split")
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], tensor=d["bf16_tflops"],
+                    tensor_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, source="fallback")
+
+
+def _workload_config(w, intermediate):
+    return {
+        "workload": f"{w.name}: T={w.T} tokens, d={w.d}, E={w.E} experts, SwiGLU F={w.F}, "
+                    f"capacity_factor={w.capacity_factor:g} (C={w.C})",
+        "T": w.T, "d": w.d, "E": w.E, "F": w.F, "C": w.C,
+        "intermediates": intermediate,
+        "l2": "flushed before every timed step (256 MiB write, outside the step's events)",
+    }
+
+
+# ---- algorithmic bytes / flops of each stage (minimum traffic the method must move) ----
+
+def stage_bytes(w, intermediate="split"):
+    """Bytes each stage must read + write at least, per layer call."""
+    T, d, E, F, C = w.T, w.d, w.E, w.F, w.C
+    Ce = C
+    hb = 4 if intermediate == "split" else 2   # H: bf16 hi+lo pair, or bf16
+    yb = 4 if intermediate == "split" else 2   # Y: fp32, or bf16
+    return {
+        "router": 2 * T * d + 2 * d * E + 2 * 4 * T * E,          # x, W_r in; scores, scores_t out
+        "select": 4 * T * E + 8 * E * Ce,                          # scores_t in; idx, gate out
+        "csr": 4 * E * Ce + 4 * (T + 1) + 4 * E * Ce,              # idx in; tok_ptr, tok_ent out
+        "gemm1_swiglu": 2 * 2 * E * d * F + 2 * E * Ce * d + hb * E * Ce * F,
+        "gemm2_scale": 2 * E * F * d + hb * E * Ce * F + 4 * E * Ce + yb * E * Ce * d,
+        "combine": yb * E * Ce * d + 4 * (T + 1) + 4 * E * Ce + 2 * T * d,
+    }
+
+
+def stage_flops(w, intermediate="split"):
+    T, d, E, F, C = w.T, w.d, w.E, w.F, w.C
+    return {"router": 2 * T * d * E, "gemm1_swiglu": 4 * E * C * d * F,
+            "gemm2_scale": 2 * E * C * F * d * (2 if intermediate == "split" else 1)}
+
+
+def _traffic(kernel_stage, workload):
+    """dram read+write bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when there is none or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_stage}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    if not m or not h:
+        return None
+    src = os.path.join(ROOT, "diffusion_transformer_moe_b200", "csrc", "experts_sm100.cu")
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
+        return None
+    return float(m.group(1))
+
+
+# ---- clocks during the timed region ----------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [s.strip() for s in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- the CPU oracle (reference arm and cpu_baseline) --------------------------------------
+
+def _oracle_inputs(w, seed):
+    from diffusion_transformer_moe_b200 import inputs as I
+    a = I.make_inputs(w, seed=seed)
+    return (I.to_numpy_f64(a["x"]), I.to_numpy_f64(a["W_r"]), a["W1"].float().numpy(),
+            a["W3"].float().numpy(), a["W2"].float().numpy())
+
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()
+             if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _time_oracle(w, args, seed, reps):
+    """Seconds per full oracle layer over `reps` repetitions of the whole workload."""
+    from oracle import nmoe_oracle as O
+    x, W_r, W1, W3, W2 = args
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        O.layer(x, W_r, W1, W3, W2, w.C)
+    return (time.perf_counter() - t0) / reps
+
+
+def cpu_baseline(w, seed=0, budget_s=12.0):
+    args = _oracle_inputs(w, seed)
+    one = _time_oracle(w, args, seed, 1)
+    reps = max(1, int(budget_s / max(one, 1e-3)))
+    per = _time_oracle(w, args, seed, reps)
+    return {"value": w.T / per, "unit": "tokens/s", "cores": _oracle_threads(),
+            "kind": "oracle",
+            "sample": f"the whole {w.name} layer (all {w.T} tokens, all {w.E} experts), "
+                      f"fp64 numpy oracle, {reps} repetitions after one untimed"}
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    data = _oracle_inputs(w, 0)
+    for _ in range(args.warmup):
+        _time_oracle(w, data, 0, 1)
+    per = [_time_oracle(w, data, 0, 1) for _ in range(args.steps)]
+    tot = sum(per)
+    value = w.T * args.steps / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _workload_config(w, "fp64 oracle"),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _oracle_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step is the whole {w.name} layer on the host cores"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---- our CUDA path ---------------------------------------------------------------------
+
+def run_ours(args, w, rank, world, local_rank, dist):
+    import torch
+    import diffusion_transformer_moe_b200 as nm
+    from diffusion_transformer_moe_b200 import inputs as I
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    a = I.make_inputs(w, seed=rank)
+    x = a["x"].to(dev)
+    W_r, W1, W3, W2 = (a[k].to(dev) for k in ("W_r", "W1", "W3", "W2"))
+    inter = args.intermediate
+    ws = torch.empty(nm.workspace_size(w.T, w.d, w.E, w.F, w.C, intermediate=inter,
+                                       host_io=True), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(x)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    K = args.steps
+    trace = nm.Trace(K)
+
+    def step(tr=None):
+        nm.forward(x, W_r, W1, W3, W2, w.C, out=out, workspace=ws, intermediate=inter,
+                   trace=tr)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if nm.get_last_error() != 0:
+        raise RuntimeError("device-side check failed during warm-up")
+
+    clocks = ClockSampler(local_rank)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(trace)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = sum(s.elapsed_time(e) for s, e in ev)
+    stage_ms, ncalls = trace.read()
+    if nm.get_last_error() != 0:
+        raise RuntimeError("device-side check failed during the timed steps")
+
+    # end to end through the C ABI with host buffers: H2D of x and D2H of out per step
+    x_host = a["x"].pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    for _ in range(max(1, args.warmup // 2)):
+        nm.forward(x_host, W_r, W1, W3, W2, w.C, out=out_host, workspace=ws,
+                   intermediate=inter, host_io=True)
+    torch.cuda.synchronize()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        nm.forward(x_host, W_r, W1, W3, W2, w.C, out=out_host, workspace=ws,
+                   intermediate=inter, host_io=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in e2e_ev)
+
+    if dist is not None:
+        t = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = t.tolist()
+    if rank != 0:
+        return
+
+    peaks = _peaks()
+    per_step_s = ms / 1e3 / K
+    tokens = w.T * world * K
+    value = tokens / (ms / 1e3)
+    sb = stage_bytes(w, inter)
+    sf = stage_flops(w, inter)
+    stages = {}
+    for name, tot in stage_ms.items():
+        avg_s = tot / 1e3 / max(ncalls, 1)
+        st = {"us": avg_s * 1e6, "GB/s": sb[name] / avg_s / 1e9,
+              "hbm_frac": sb[name] / avg_s / 1e9 / peaks["hbm"]}
+        if name in sf:
+            st["TFLOP/s"] = sf[name] / avg_s / 1e12
+        stages[name] = st
+    dom = max(stage_ms, key=lambda k: stage_ms[k])
+    dom_s = stage_ms[dom] / 1e3 / max(ncalls, 1)
+    achieved = sb[dom] / dom_s / 1e9
+    roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm"],
+            "unit": "GB/s", "frac": achieved / peaks["hbm"],
+            "traffic": _traffic(dom, w.name),
+            "algorithmic_bytes_per_launch": sb[dom],
+            "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)"
+            if peaks["source"] == "measured" else "fallback 6650 GB/s"}
+    flops = w.expert_flops() + w.router_flops()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(_workload_config(w, inter), parallelism=f"replicas x{world}"),
+        "tflops": flops / per_step_s / 1e12,
+        "tensor_frac_of_layer": flops / per_step_s / 1e12 / peaks["tensor_sustained"],
+        "roofline": roof,
+        "stages": stages,
+        "gpu_launches": 6 * K,
+        "e2e": {"value": w.T * world * K / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+        "clocks": clk,
+    }
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = _args()
+    from diffusion_transformer_moe_b200 import inputs as I
+    w = I.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+        dist = tdist
+    try:
+        run_ours(args, w, rank, world, local_rank, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

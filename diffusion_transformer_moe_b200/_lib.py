@@ -1,0 +1,255 @@
+"""ctypes binding of libnmoe (include/nmoe.h). Argument marshalling only.
+
+Every function here hands device pointers, sizes and the current CUDA stream to the
+C ABI; all of the layer's arithmetic runs in the library's CUDA kernels. There is no
+fallback: if the shared library is missing, or a call fails, an error is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnmoe.so")
+
+NMOE_BF16, NMOE_F32 = 0, 1
+SCORE = {"softmax": 0, "sigmoid": 1}
+COMBINE = {"raw": 0, "normalized": 1}
+INTERMEDIATE = {"split": 0, "bf16": 1}
+N_STAGES = 6
+STATUS = {
+    0: "NMOE_OK", 1: "NMOE_ERR_INVALID_ARG", 2: "NMOE_ERR_UNSUPPORTED",
+    3: "NMOE_ERR_WORKSPACE", 4: "NMOE_ERR_CUDA", 5: "NMOE_ERR_TIMEOUT",
+    6: "NMOE_ERR_DEVICE_CHECK", 7: "NMOE_ERR_NO_DEVICE",
+}
+
+# Every symbol include/nmoe.h declares.
+EXPORTS = (
+    "nmoe_options_init", "nmoe_router", "nmoe_select", "nmoe_forward", "nmoe_forward_ex",
+    "nmoe_workspace_size", "nmoe_get_last_error", "nmoe_status_str", "nmoe_trace_create",
+    "nmoe_trace_read", "nmoe_trace_reset", "nmoe_trace_destroy", "nmoe_stage_name",
+    "nmoe_build_info",
+)
+
+
+class NmoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class Options(C.Structure):
+    _fields_ = [
+        ("dtype", C.c_int), ("score_fn", C.c_int), ("combine", C.c_int),
+        ("route_scale", C.c_float), ("n_segments", C.c_int64), ("router_bias", C.c_void_p),
+        ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t),
+        ("scores_out", C.c_void_p), ("idx_out", C.c_void_p), ("host_io", C.c_int),
+        ("trace", C.c_void_p), ("intermediate", C.c_int), ("out_f32", C.c_int),
+    ]
+
+
+_lib = None
+_lock = threading.Lock()
+_i64 = C.c_int64
+_vp = C.c_void_p
+
+
+def lib() -> C.CDLL:
+    """The loaded shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m diffusion_transformer_moe_b200.build`")
+            L = C.CDLL(LIB_PATH)
+            L.nmoe_options_init.argtypes = [C.POINTER(Options)]
+            L.nmoe_options_init.restype = None
+            L.nmoe_router.argtypes = [_vp, _vp, _i64, _i64, _i64, C.c_int, C.c_int, _vp, _i64,
+                                      _vp, _vp, _vp]
+            L.nmoe_router.restype = C.c_int
+            L.nmoe_select.argtypes = [_vp, _i64, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
+            L.nmoe_select.restype = C.c_int
+            L.nmoe_forward.argtypes = [_vp] * 5 + [_i64] * 5 + [_vp, _vp]
+            L.nmoe_forward.restype = C.c_int
+            L.nmoe_forward_ex.argtypes = [_vp] * 5 + [_i64] * 5 + [_vp, _vp,
+                                                                  C.POINTER(Options)]
+            L.nmoe_forward_ex.restype = C.c_int
+            L.nmoe_workspace_size.argtypes = [_i64] * 5 + [C.POINTER(Options)]
+            L.nmoe_workspace_size.restype = C.c_size_t
+            L.nmoe_get_last_error.argtypes = [_vp]
+            L.nmoe_get_last_error.restype = C.c_int
+            L.nmoe_status_str.argtypes = [C.c_int]
+            L.nmoe_status_str.restype = C.c_char_p
+            L.nmoe_trace_create.argtypes = [C.c_int, C.POINTER(_vp)]
+            L.nmoe_trace_create.restype = C.c_int
+            L.nmoe_trace_read.argtypes = [_vp, C.POINTER(C.c_double), C.POINTER(C.c_int)]
+            L.nmoe_trace_read.restype = C.c_int
+            L.nmoe_trace_reset.argtypes = [_vp]
+            L.nmoe_trace_reset.restype = C.c_int
+            L.nmoe_trace_destroy.argtypes = [_vp]
+            L.nmoe_trace_destroy.restype = None
+            L.nmoe_stage_name.argtypes = [C.c_int]
+            L.nmoe_stage_name.restype = C.c_char_p
+            L.nmoe_build_info.argtypes = []
+            L.nmoe_build_info.restype = C.c_char_p
+            _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise NmoeError(status, what)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return NMOE_BF16
+    if t.dtype == torch.float32:
+        return NMOE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
+            n_segments=1, router_bias=None, workspace=None, scores_out=None, idx_out=None,
+            host_io=False, trace=None, intermediate="split", out_f32=False) -> Options:
+    o = Options()
+    lib().nmoe_options_init(C.byref(o))
+    o.dtype = dtype
+    o.score_fn = SCORE[score_fn]
+    o.combine = COMBINE[combine]
+    o.route_scale = float(route_scale)
+    o.n_segments = int(n_segments)
+    o.router_bias = _ptr(router_bias)
+    if workspace is not None:
+        o.workspace = workspace.data_ptr()
+        o.workspace_bytes = workspace.numel() * workspace.element_size()
+    o.scores_out = _ptr(scores_out)
+    o.idx_out = _ptr(idx_out)
+    o.host_io = 1 if host_io else 0
+    o.trace = None if trace is None else trace.handle
+    o.intermediate = INTERMEDIATE[intermediate]
+    o.out_f32 = 1 if out_f32 else 0
+    return o
+
+
+def router(x, W_r, score_fn="softmax", router_bias=None, n_segments=1, stream=None):
+    """scores [T,E], scores_t [E,T] (fp32) for x [T,d], W_r [d,E]."""
+    _dev(x, "x"); _dev(W_r, "W_r")
+    T, d = x.shape
+    E = W_r.shape[1]
+    scores = torch.empty(T, E, device=x.device, dtype=torch.float32)
+    scores_t = torch.empty(E, T, device=x.device, dtype=torch.float32)
+    _check(lib().nmoe_router(x.data_ptr(), W_r.data_ptr(), T, d, E, _dt(x), SCORE[score_fn],
+                             _ptr(router_bias), n_segments, scores.data_ptr(),
+                             scores_t.data_ptr(), _stream(stream)), "nmoe_router")
+    return scores, scores_t
+
+
+def select(scores_t, C_: int, n_segments=1, csr=True, stream=None):
+    """idx [E, n_segments*C] int32, gate fp32, and (if csr) tok_ptr [T+1], tok_ent."""
+    _dev(scores_t, "scores_t")
+    E, T = scores_t.shape
+    Ce = n_segments * C_
+    dev = scores_t.device
+    idx = torch.empty(E, Ce, device=dev, dtype=torch.int32)
+    gate = torch.empty(E, Ce, device=dev, dtype=torch.float32)
+    tok_ptr = torch.empty(T + 1, device=dev, dtype=torch.int32) if csr else None
+    tok_ent = torch.empty(E * Ce, device=dev, dtype=torch.int32) if csr else None
+    _check(lib().nmoe_select(scores_t.data_ptr(), T, E, C_, n_segments, idx.data_ptr(),
+                             gate.data_ptr(), _ptr(tok_ptr), _ptr(tok_ent), _stream(stream)),
+           "nmoe_select")
+    return idx, gate, tok_ptr, tok_ent
+
+
+def forward(x, W_r, W1, W3, W2, C_: int, out=None, stream=None, **opts):
+    """The whole layer. ``opts`` are the nmoe_options fields (score_fn, combine,
+    route_scale, n_segments, router_bias, workspace, scores_out, idx_out, trace,
+    intermediate, out_f32). With ``host_io=True`` x and out are pinned CPU tensors."""
+    host_io = bool(opts.get("host_io", False))
+    for n, t in (("W_r", W_r), ("W1", W1), ("W3", W3), ("W2", W2)):
+        _dev(t, n)
+    if not host_io:
+        _dev(x, "x")
+    T, d = x.shape
+    E, _, F = W1.shape
+    if out is None:
+        odt = torch.float32 if opts.get("out_f32", False) else x.dtype
+        out = torch.empty(T, d, dtype=odt, device="cpu" if host_io else x.device,
+                          pin_memory=host_io)
+    o = options(dtype=_dt(x), **opts)
+    if opts or x.dtype != torch.bfloat16:
+        st = lib().nmoe_forward_ex(x.data_ptr(), W_r.data_ptr(), W1.data_ptr(), W3.data_ptr(),
+                                   W2.data_ptr(), T, d, E, F, C_, out.data_ptr(),
+                                   _stream(stream), C.byref(o))
+    else:
+        st = lib().nmoe_forward(x.data_ptr(), W_r.data_ptr(), W1.data_ptr(), W3.data_ptr(),
+                                W2.data_ptr(), T, d, E, F, C_, out.data_ptr(), _stream(stream))
+    _check(st, "nmoe_forward")
+    return out
+
+
+def workspace_size(T, d, E, F, C_, **opts) -> int:
+    o = options(**opts)
+    return int(lib().nmoe_workspace_size(T, d, E, F, C_, C.byref(o)))
+
+
+def get_last_error(stream=None) -> int:
+    return int(lib().nmoe_get_last_error(_stream(stream)))
+
+
+def build_info() -> str:
+    return lib().nmoe_build_info().decode()
+
+
+class Trace:
+    """Per-stage CUDA-event timer of nmoe_forward_ex calls (include/nmoe.h nmoe_trace)."""
+
+    def __init__(self, max_calls: int):
+        h = _vp()
+        _check(lib().nmoe_trace_create(max_calls, C.byref(h)), "nmoe_trace_create")
+        self.handle = h.value
+
+    def read(self):
+        ms = (C.c_double * N_STAGES)()
+        n = C.c_int()
+        _check(lib().nmoe_trace_read(self.handle, ms, C.byref(n)), "nmoe_trace_read")
+        names = [lib().nmoe_stage_name(i).decode() for i in range(N_STAGES)]
+        return dict(zip(names, list(ms))), n.value
+
+    def reset(self):
+        _check(lib().nmoe_trace_reset(self.handle), "nmoe_trace_reset")
+
+    def close(self):
+        if self.handle:
+            lib().nmoe_trace_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,461 @@
+// C ABI of libnmoe: argument checks, workspace layout, stage launches.
+//
+// Every entry point validates its arguments on the host before it touches CUDA, so a
+// rejected call enqueues nothing. The layer's steps run in this library's kernels in
+// launch order router -> select -> csr -> gemm1 -> gemm2 -> combine, all on the
+// caller's stream, with no host synchronisation (every shape is fixed by (T, E, C):
+// expert choice gives each expert exactly C tokens per segment).
+#include <math.h>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "nmoe_internal.cuh"
+#include "experts_sm100.cuh"
+#include "router_sm100.cuh"
+
+// Per-device error word: kernels OR kErr* bits into it; nmoe_get_last_error reads and
+// clears it. Host code reaches it through cudaGetSymbolAddress.
+__device__ unsigned nmoe_g_err_word;
+
+namespace {
+
+using nmoe::Shape;
+
+struct DevState {
+  bool ready = false;
+  bool ok = false;
+  int sm_count = 0;
+  unsigned* err = nullptr;
+};
+
+std::mutex g_mu;
+constexpr int kMaxDevices = 64;
+DevState g_dev[kMaxDevices];
+
+nmoe_status dev_state(DevState** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return NMOE_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevState& s = g_dev[dev];
+  if (!s.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return NMOE_ERR_CUDA;
+    }
+    s.ok = (major == 10 && minor == 0);
+    s.sm_count = sms;
+    if (s.ok) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, nmoe_g_err_word) != cudaSuccess) {
+        cudaGetLastError();
+        return NMOE_ERR_CUDA;
+      }
+      s.err = static_cast<unsigned*>(p);
+    }
+    s.ready = true;
+  }
+  if (!s.ok) return NMOE_ERR_NO_DEVICE;
+  *out = &s;
+  return NMOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+size_t esize(nmoe_dtype dt) { return dt == NMOE_F32 ? 4 : 2; }
+
+nmoe_options default_options() {
+  nmoe_options o;
+  nmoe_options_init(&o);
+  return o;
+}
+
+// Sizes and enums shared by every entry point.
+nmoe_status check_shape(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C, int64_t n_seg,
+                        nmoe_dtype dt, bool need_dF) {
+  if (dt != NMOE_BF16 && dt != NMOE_F32) return NMOE_ERR_INVALID_ARG;
+  if (T < 1 || T >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
+  if (E < 1 || E > 256) return NMOE_ERR_INVALID_ARG;
+  if (n_seg < 1 || n_seg > 65535 || T % n_seg != 0) return NMOE_ERR_INVALID_ARG;
+  if (C < 1 || C > T / n_seg) return NMOE_ERR_INVALID_ARG;
+  if (E * n_seg * C >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
+  if (need_dF) {
+    if (d < 1 || F < 1) return NMOE_ERR_INVALID_ARG;
+    if (d % 8 != 0 || F % 8 != 0) return NMOE_ERR_UNSUPPORTED;
+    if (d >= (int64_t(1) << 31) || F >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
+  }
+  return NMOE_OK;
+}
+
+Shape make_shape(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C, int64_t n_seg) {
+  Shape s;
+  s.T = (int)T; s.d = (int)d; s.E = (int)E; s.F = (int)F; s.C = (int)C;
+  s.n_seg = (int)n_seg; s.S = (int)(T / n_seg); s.Ce = (int)(n_seg * C);
+  return s;
+}
+
+// Bytes per element of the H and Y intermediates: fp32 layers and SPLIT bf16 layers
+// use 4 (fp32, or a bf16 hi/lo pair), BF16 intermediates use 2.
+size_t inter_size(nmoe_dtype dt, const nmoe_options& o) {
+  return (dt == NMOE_F32 || o.intermediate == NMOE_INTERMEDIATE_SPLIT) ? 4 : 2;
+}
+size_t out_size(nmoe_dtype dt, const nmoe_options& o) {
+  return (dt == NMOE_F32 || o.out_f32) ? 4 : 2;
+}
+
+struct Layout {
+  size_t scores, scores_t, idx, gate, tok_ptr, tok_ent, H, Y, xin, xout, total;
+};
+
+Layout make_layout(const Shape& s, nmoe_dtype dt, const nmoe_options& o) {
+  Layout L;
+  size_t off = 0;
+  const size_t is = inter_size(dt, o);
+  const size_t none = ~size_t(0);
+  auto take = [&](size_t bytes) { size_t at = off; off = align256(off + bytes); return at; };
+  L.scores = o.scores_out ? none : take(sizeof(float) * (size_t)s.T * s.E);
+  L.scores_t = take(sizeof(float) * (size_t)s.T * s.E);
+  L.idx = o.idx_out ? none : take(sizeof(int32_t) * (size_t)s.E * s.Ce);
+  L.gate = take(sizeof(float) * (size_t)s.E * s.Ce);
+  L.tok_ptr = take(sizeof(int32_t) * ((size_t)s.T + 1));
+  L.tok_ent = take(sizeof(int32_t) * (size_t)s.E * s.Ce);
+  L.H = take(is * (size_t)s.E * s.Ce * s.F);
+  L.Y = take(is * (size_t)s.E * s.Ce * s.d);
+  L.xin = o.host_io ? take(esize(dt) * (size_t)s.T * s.d) : none;
+  L.xout = o.host_io ? take(out_size(dt, o) * (size_t)s.T * s.d) : none;
+  L.total = off;
+  return L;
+}
+
+nmoe_status options_ok(const nmoe_options& o) {
+  if (o.score_fn != NMOE_SCORE_SOFTMAX && o.score_fn != NMOE_SCORE_SIGMOID)
+    return NMOE_ERR_INVALID_ARG;
+  if (o.combine != NMOE_COMBINE_RAW && o.combine != NMOE_COMBINE_NORMALIZED)
+    return NMOE_ERR_INVALID_ARG;
+  if (!isfinite(o.route_scale)) return NMOE_ERR_INVALID_ARG;
+  if (o.router_bias && (reinterpret_cast<uintptr_t>(o.router_bias) & 3u))
+    return NMOE_ERR_INVALID_ARG;
+  if (o.scores_out && !aligned16(o.scores_out)) return NMOE_ERR_INVALID_ARG;
+  if (o.idx_out && !aligned16(o.idx_out)) return NMOE_ERR_INVALID_ARG;
+  if (o.workspace && (reinterpret_cast<uintptr_t>(o.workspace) & 255u))
+    return NMOE_ERR_INVALID_ARG;
+  if (o.intermediate != NMOE_INTERMEDIATE_SPLIT && o.intermediate != NMOE_INTERMEDIATE_BF16)
+    return NMOE_ERR_INVALID_ARG;
+  return NMOE_OK;
+}
+
+}  // namespace
+
+struct nmoe_trace {
+  int max_calls = 0;
+  int n = 0;
+  std::vector<cudaEvent_t> ev;  // (NMOE_N_STAGES + 1) per call
+};
+
+namespace {
+
+cudaEvent_t* trace_slot(nmoe_trace* tr) {
+  if (!tr || tr->n >= tr->max_calls) return nullptr;
+  return &tr->ev[(size_t)tr->n++ * (NMOE_N_STAGES + 1)];
+}
+
+nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const void* W3,
+                         const void* W2, int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
+                         void* out, cudaStream_t st, const nmoe_options& o) {
+  nmoe_status v = check_shape(T, d, E, F, C, o.n_segments, o.dtype, true);
+  if (v != NMOE_OK) return v;
+  if ((v = options_ok(o)) != NMOE_OK) return v;
+  if (!x || !W_r || !W1 || !W3 || !W2 || !out) return NMOE_ERR_INVALID_ARG;
+  if (!aligned16(W_r) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2))
+    return NMOE_ERR_INVALID_ARG;
+  if (!o.host_io && (!aligned16(x) || !aligned16(out))) return NMOE_ERR_INVALID_ARG;
+  if (x == out) return NMOE_ERR_INVALID_ARG;
+
+  DevState* ds = nullptr;
+  if ((v = dev_state(&ds)) != NMOE_OK) return v;
+  const Shape s = make_shape(T, d, E, F, C, o.n_segments);
+  if (s.Ce > 65535 * 64) return NMOE_ERR_UNSUPPORTED;
+  const Layout L = make_layout(s, o.dtype, o);
+
+  char* ws = static_cast<char*>(o.workspace);
+  bool own = false;
+  if (!ws) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), L.total, st) != cudaSuccess) {
+      cudaGetLastError();
+      return NMOE_ERR_WORKSPACE;
+    }
+    own = true;
+  } else if (o.workspace_bytes < L.total) {
+    return NMOE_ERR_WORKSPACE;
+  }
+
+  float* scores = o.scores_out ? o.scores_out : reinterpret_cast<float*>(ws + L.scores);
+  float* scores_t = reinterpret_cast<float*>(ws + L.scores_t);
+  int32_t* idx = o.idx_out ? o.idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* gate = reinterpret_cast<float*>(ws + L.gate);
+  int32_t* tok_ptr = reinterpret_cast<int32_t*>(ws + L.tok_ptr);
+  int32_t* tok_ent = reinterpret_cast<int32_t*>(ws + L.tok_ent);
+  void* H = ws + L.H;
+  void* Y = ws + L.Y;
+  const size_t xbytes = esize(o.dtype) * (size_t)s.T * s.d;
+  const size_t obytes = out_size(o.dtype, o) * (size_t)s.T * s.d;
+  const bool f32 = o.dtype == NMOE_F32;
+  const bool split = !f32 && o.intermediate == NMOE_INTERMEDIATE_SPLIT;
+  const bool y_f32 = f32 || split;
+  const bool out_f32 = f32 || o.out_f32;
+
+  const void* xd = x;
+  void* outd = out;
+  cudaError_t e = cudaSuccess;
+  if (o.host_io) {
+    xd = ws + L.xin;
+    outd = ws + L.xout;
+    e = cudaMemcpyAsync(ws + L.xin, x, xbytes, cudaMemcpyHostToDevice, st);
+  }
+  cudaEvent_t* ev = trace_slot(o.trace);
+  auto mark = [&](int i) {
+    if (ev && e == cudaSuccess) e = cudaEventRecord(ev[i], st);
+  };
+  mark(0);
+  if (e == cudaSuccess) {
+    if (o.dtype == NMOE_BF16 && nmoe::router_sm100_supported(s))
+      e = nmoe::launch_router_sm100(xd, W_r, s, o.score_fn, o.router_bias, scores, scores_t,
+                                    ds->err, st);
+    else
+      e = nmoe::launch_router_simt(xd, W_r, s, o.dtype, o.score_fn, o.router_bias, scores,
+                                   scores_t, st);
+  }
+  mark(1);
+  if (e == cudaSuccess) e = nmoe::launch_select(scores_t, s, idx, gate, ds->err, st);
+  mark(2);
+  if (e == cudaSuccess)
+    e = nmoe::launch_csr(idx, s, tok_ptr, tok_ent, gate, o.combine, o.route_scale, ds->err, st);
+  mark(3);
+  const bool tc = !f32 && nmoe::experts_sm100_supported(s);
+  // SPLIT on the tensor cores: H_hi then H_lo, each [E*Ce, F] bf16; on the CUDA cores
+  // (shapes the tcgen05 kernels do not take) H is one fp32 array of the same size.
+  void* H_lo = static_cast<char*>(H) + sizeof(uint16_t) * (size_t)s.E * s.Ce * s.F;
+  if (e == cudaSuccess)
+    e = tc ? nmoe::launch_gemm1_sm100(xd, idx, W1, W3, s, split, H, H_lo, ds->err,
+                                      ds->sm_count, st)
+           : nmoe::launch_gemm1_simt(xd, idx, W1, W3, s, o.dtype, split, H, st);
+  mark(4);
+  if (e == cudaSuccess)
+    e = tc ? nmoe::launch_gemm2_sm100(H, H_lo, gate, W2, s, split, Y, ds->err, ds->sm_count, st)
+           : nmoe::launch_gemm2_simt(H, gate, W2, s, o.dtype, split, y_f32, Y, st);
+  mark(5);
+  if (e == cudaSuccess)
+    e = nmoe::launch_combine(Y, tok_ptr, tok_ent, s, y_f32, out_f32, outd, ds->sm_count, st);
+  mark(6);
+  if (o.host_io && e == cudaSuccess)
+    e = cudaMemcpyAsync(out, outd, obytes, cudaMemcpyDeviceToHost, st);
+  if (own) {
+    cudaError_t f = cudaFreeAsync(ws, st);
+    if (e == cudaSuccess) e = f;
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return NMOE_ERR_CUDA;
+  }
+  return NMOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void nmoe_options_init(nmoe_options* o) {
+  if (!o) return;
+  o->dtype = NMOE_BF16;
+  o->score_fn = NMOE_SCORE_SOFTMAX;
+  o->combine = NMOE_COMBINE_RAW;
+  o->route_scale = 1.0f;
+  o->n_segments = 1;
+  o->router_bias = nullptr;
+  o->workspace = nullptr;
+  o->workspace_bytes = 0;
+  o->scores_out = nullptr;
+  o->idx_out = nullptr;
+  o->host_io = 0;
+  o->trace = nullptr;
+  o->intermediate = NMOE_INTERMEDIATE_SPLIT;
+  o->out_f32 = 0;
+}
+
+nmoe_status nmoe_router(const void* x, const void* W_r, int64_t T, int64_t d, int64_t E,
+                        nmoe_dtype dtype, nmoe_score_fn score_fn, const float* router_bias,
+                        int64_t n_segments, float* scores, float* scores_t,
+                        nmoe_stream_t stream) {
+  nmoe_status v = check_shape(T, d, E, 1, 1, n_segments, dtype, false);
+  if (v != NMOE_OK) return v;
+  if (d < 1 || d >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
+  if (d % 8 != 0) return NMOE_ERR_UNSUPPORTED;
+  if (score_fn != NMOE_SCORE_SOFTMAX && score_fn != NMOE_SCORE_SIGMOID)
+    return NMOE_ERR_INVALID_ARG;
+  if (!x || !W_r || (!scores && !scores_t)) return NMOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W_r)) return NMOE_ERR_INVALID_ARG;
+  if ((scores && !aligned16(scores)) || (scores_t && !aligned16(scores_t)))
+    return NMOE_ERR_INVALID_ARG;
+  if (router_bias && (reinterpret_cast<uintptr_t>(router_bias) & 3u)) return NMOE_ERR_INVALID_ARG;
+  DevState* ds = nullptr;
+  if ((v = dev_state(&ds)) != NMOE_OK) return v;
+  const Shape s = make_shape(T, d, E, 8, 1, n_segments);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dtype == NMOE_BF16 && nmoe::router_sm100_supported(s) && scores && scores_t)
+    e = nmoe::launch_router_sm100(x, W_r, s, score_fn, router_bias, scores, scores_t, ds->err,
+                                  st);
+  else
+    e = nmoe::launch_router_simt(x, W_r, s, dtype, score_fn, router_bias, scores, scores_t, st);
+  if (e != cudaSuccess) { cudaGetLastError(); return NMOE_ERR_CUDA; }
+  return NMOE_OK;
+}
+
+nmoe_status nmoe_select(const float* scores_t, int64_t T, int64_t E, int64_t C,
+                        int64_t n_segments, int32_t* idx, float* gate, int32_t* tok_ptr,
+                        int32_t* tok_ent, nmoe_stream_t stream) {
+  nmoe_status v = check_shape(T, 8, E, 8, C, n_segments, NMOE_F32, false);
+  if (v != NMOE_OK) return v;
+  if (!scores_t || !idx || !gate) return NMOE_ERR_INVALID_ARG;
+  if ((tok_ptr == nullptr) != (tok_ent == nullptr)) return NMOE_ERR_INVALID_ARG;
+  if (!aligned16(scores_t) || !aligned16(idx) || !aligned16(gate)) return NMOE_ERR_INVALID_ARG;
+  if (tok_ptr && (!aligned16(tok_ptr) || !aligned16(tok_ent))) return NMOE_ERR_INVALID_ARG;
+  DevState* ds = nullptr;
+  if ((v = dev_state(&ds)) != NMOE_OK) return v;
+  const Shape s = make_shape(T, 8, E, 8, C, n_segments);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = nmoe::launch_select(scores_t, s, idx, gate, ds->err, st);
+  if (e == cudaSuccess && tok_ptr)
+    e = nmoe::launch_csr(idx, s, tok_ptr, tok_ent, gate, NMOE_COMBINE_RAW, 1.f, ds->err, st);
+  if (e != cudaSuccess) { cudaGetLastError(); return NMOE_ERR_CUDA; }
+  return NMOE_OK;
+}
+
+nmoe_status nmoe_forward(const void* x, const void* W_r, const void* W1, const void* W3,
+                         const void* W2, int64_t T, int64_t d, int64_t E, int64_t F,
+                         int64_t C, void* out, nmoe_stream_t stream) {
+  return forward_impl(x, W_r, W1, W3, W2, T, d, E, F, C, out,
+                      static_cast<cudaStream_t>(stream), default_options());
+}
+
+nmoe_status nmoe_forward_ex(const void* x, const void* W_r, const void* W1, const void* W3,
+                            const void* W2, int64_t T, int64_t d, int64_t E, int64_t F,
+                            int64_t C, void* out, nmoe_stream_t stream,
+                            const nmoe_options* opts) {
+  return forward_impl(x, W_r, W1, W3, W2, T, d, E, F, C, out,
+                      static_cast<cudaStream_t>(stream), opts ? *opts : default_options());
+}
+
+size_t nmoe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
+                           const nmoe_options* opts) {
+  const nmoe_options o = opts ? *opts : default_options();
+  if (check_shape(T, d, E, F, C, o.n_segments, o.dtype, true) != NMOE_OK) return 0;
+  return make_layout(make_shape(T, d, E, F, C, o.n_segments), o.dtype, o).total;
+}
+
+nmoe_status nmoe_get_last_error(nmoe_stream_t stream) {
+  DevState* ds = nullptr;
+  nmoe_status v = dev_state(&ds);
+  if (v != NMOE_OK) return v;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return NMOE_ERR_CUDA;
+  }
+  unsigned word = 0;
+  if (cudaMemcpy(&word, ds->err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return NMOE_ERR_CUDA;
+  }
+  if (word != 0 && cudaMemset(ds->err, 0, sizeof(unsigned)) != cudaSuccess) {
+    cudaGetLastError();
+    return NMOE_ERR_CUDA;
+  }
+  if (word & nmoe::kErrTimeout) return NMOE_ERR_TIMEOUT;
+  if (word & nmoe::kErrDeviceCheck) return NMOE_ERR_DEVICE_CHECK;
+  return NMOE_OK;
+}
+
+const char* nmoe_status_str(nmoe_status s) {
+  switch (s) {
+    case NMOE_OK: return "ok";
+    case NMOE_ERR_INVALID_ARG: return "invalid argument";
+    case NMOE_ERR_UNSUPPORTED: return "unsupported size or option";
+    case NMOE_ERR_WORKSPACE: return "workspace too small or allocation failed";
+    case NMOE_ERR_CUDA: return "CUDA error";
+    case NMOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case NMOE_ERR_DEVICE_CHECK: return "device-side check failed";
+    case NMOE_ERR_NO_DEVICE: return "no sm_100 device is current";
+  }
+  return "unknown status";
+}
+
+nmoe_status nmoe_trace_create(int max_calls, nmoe_trace** out) {
+  if (!out || max_calls < 1) return NMOE_ERR_INVALID_ARG;
+  nmoe_trace* tr = new (std::nothrow) nmoe_trace();
+  if (!tr) return NMOE_ERR_WORKSPACE;
+  tr->max_calls = max_calls;
+  tr->ev.assign((size_t)max_calls * (NMOE_N_STAGES + 1), nullptr);
+  for (auto& e : tr->ev) {
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaGetLastError();
+      nmoe_trace_destroy(tr);
+      return NMOE_ERR_CUDA;
+    }
+  }
+  *out = tr;
+  return NMOE_OK;
+}
+
+nmoe_status nmoe_trace_read(nmoe_trace* tr, double* stage_ms, int* n_calls) {
+  if (!tr || !stage_ms) return NMOE_ERR_INVALID_ARG;
+  for (int i = 0; i < NMOE_N_STAGES; ++i) stage_ms[i] = 0.0;
+  for (int c = 0; c < tr->n; ++c) {
+    cudaEvent_t* ev = &tr->ev[(size_t)c * (NMOE_N_STAGES + 1)];
+    if (cudaEventSynchronize(ev[NMOE_N_STAGES]) != cudaSuccess) {
+      cudaGetLastError();
+      return NMOE_ERR_CUDA;
+    }
+    for (int i = 0; i < NMOE_N_STAGES; ++i) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, ev[i], ev[i + 1]) != cudaSuccess) {
+        cudaGetLastError();
+        return NMOE_ERR_CUDA;
+      }
+      stage_ms[i] += ms;
+    }
+  }
+  if (n_calls) *n_calls = tr->n;
+  return NMOE_OK;
+}
+
+nmoe_status nmoe_trace_reset(nmoe_trace* tr) {
+  if (!tr) return NMOE_ERR_INVALID_ARG;
+  tr->n = 0;
+  return NMOE_OK;
+}
+
+void nmoe_trace_destroy(nmoe_trace* tr) {
+  if (!tr) return;
+  for (auto& e : tr->ev)
+    if (e) cudaEventDestroy(e);
+  delete tr;
+}
+
+const char* nmoe_stage_name(int stage) {
+  static const char* names[NMOE_N_STAGES] = {"router", "select", "csr", "gemm1_swiglu",
+                                             "gemm2_scale", "combine"};
+  return (stage >= 0 && stage < NMOE_N_STAGES) ? names[stage] : "unknown";
+}
+
+const char* nmoe_build_info(void) {
+  return "nmoe sm_100a: router tcgen05(bf16)/simt(fp32); select radix; csr lower-bound; "
+         "experts tcgen05+TMA gather4(bf16)/simt(fp32); combine fixed-order";
+}
+
+}  // extern "C"

@@ -1,0 +1,429 @@
+// Grouped SwiGLU expert GEMMs on the 5th-generation tensor cores.
+//
+// The packed SwiGLU experts of the NucleusMoE-Image walkthrough (section 6: fused
+// gate/up projection of shape (experts, hidden, 2 * moe_intermediate_dim), then the down
+// projection; "only two grouped matmuls at runtime"; the grouped path wants each
+// expert's tokens as one contiguous block). Expert choice makes every block exactly
+// Ce = n_segments * C rows, so both GEMMs have static shapes:
+//
+//   gemm1: H[e, s, :] = silu(x[idx[e,s]] W1_e) * (x[idx[e,s]] W3_e)
+//   gemm2: Y[e*Ce + s, :] = gate[e, s] * (H[e, s, :] W2_e)
+//
+// Instead of permuting tokens into per-expert blocks, gemm1 gathers the 128 rows of an
+// A tile straight from x with TMA tile::gather4 (32 copies of 4 rows per k-block).
+//
+// Intermediate precision. With SPLIT (the default), H is stored as a pair of bf16
+// arrays hi = bf16(h), lo = bf16(h - hi) (about 16 significant bits), gemm2 runs both
+// halves against the same W2 tile into one fp32 accumulator, and Y is stored in fp32.
+// Without SPLIT, H and Y are single bf16 arrays (the usual bf16 MoE numerics), which
+// moves ~10% fewer bytes but lets large-magnitude tokens drift by ~0.1-0.2 absolute.
+//
+// One persistent CTA per SM walks tiles (expert, 128-row block, N block) in a static
+// round-robin. Warp roles: warp 0 issues TMA copies into a shared-memory ring, warp 1
+// (one thread) issues tcgen05.mma into a double-buffered TMEM accumulator (2 x 256 fp32
+// columns), warps 2-5 run the epilogue (tcgen05.ld, SwiGLU or gate scale, stores) while
+// the next tile's MMAs run. Tile: M = 128 rows, K = 64 per stage, N = 256 accumulator
+// columns (gemm1: 128 gate + 128 up columns of F; gemm2: 256 columns of d). A is
+// K-major, B (the weights, [E, K, N] with N contiguous) is MN-major; both use the
+// 128-byte swizzle. Every wait is bounded; a wait that runs out sets the device error
+// word and the kernel drains its copies and MMAs, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include "experts_sm100.cuh"
+#include "sm100_ptx.cuh"
+
+namespace nmoe {
+namespace {
+
+using namespace ptx;
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kABytes = kBM * kBK * 2;          // 16 KB per A tile
+constexpr int kBBoxBytes = 64 * kBK * 2;        // 8 KB: 64 N x 64 K
+constexpr int kBBytes = 4 * kBBoxBytes;         // 32 KB: N = 256
+constexpr int kAccCols = 256;
+constexpr int kTmemCols = 2 * kAccCols;
+constexpr int kThreads = 192;
+constexpr uint64_t kWaitNs = 2000000000ull;     // 2 s per wait
+constexpr uint64_t kDrainNs = 20000000ull;      // 20 ms per drain wait
+
+enum { kGemm1 = 0, kGemm2 = 1 };
+
+template <int MODE, bool SPLIT>
+struct Cfg {
+  static constexpr int kATiles = (MODE == kGemm2 && SPLIT) ? 2 : 1;
+  static constexpr int kStageBytes = kATiles * kABytes + kBBytes;
+  static constexpr int kStages = (MODE == kGemm2 && SPLIT) ? 3 : 4;
+  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
+};
+
+struct Params {
+  int Ce;          // rows per expert
+  int K;           // reduction length (d for gemm1, F for gemm2)
+  int N;           // output row length (F for gemm1, d for gemm2)
+  int tiles_m, tiles_n, num_tiles;
+  const int32_t* idx;    // gemm1: chosen tokens [E, Ce]
+  const float* gate;     // gemm2: combine weights [E, Ce]
+  void* out;             // gemm1: H (hi) [E*Ce, F] bf16; gemm2: Y [E*Ce, d] (fp32 if SPLIT)
+  void* out_lo;          // gemm1 with SPLIT: H lo [E*Ce, F] bf16
+  unsigned* err;
+};
+
+__device__ __forceinline__ float silu_f32(float g) { return g / (1.f + expf(-g)); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// lo half of the (hi, lo) split: bf16(v - bf16(v)), for two values
+__device__ __forceinline__ uint32_t pack_lo_bf16x2(float a, float b, uint32_t hi) {
+  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&hi);
+  float2 f = __bfloat1622float2(h);
+  return pack_bf16x2(a - f.x, b - f.y);
+}
+
+template <int MODE, bool SPLIT>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                    const __grid_constant__ CUtensorMap map_a2,
+                    const __grid_constant__ CUtensorMap map_b0,
+                    const __grid_constant__ CUtensorMap map_b1, const Params p) {
+  using C = Cfg<MODE, SPLIT>;
+  constexpr int kStages = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = (p.K + kBK - 1) / kBK;
+  constexpr int n_per_tile = MODE == kGemm1 ? 128 : 256;
+  // stage s: A tile(s) at s * kStageBytes, B boxes after them
+  auto a_tile = [&](int s, int which) { return smem + s * C::kStageBytes + which * kABytes; };
+  auto b_tile = [&](int s) { return smem + s * C::kStageBytes + C::kATiles * kABytes; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) { mbar_init(&full_bar[i], 1); mbar_init(&empty_bar[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tfull_bar[i], 1); mbar_init(&tempty_bar[i], 4); }
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&map_a);
+    if (C::kATiles == 2) prefetch_tensormap(&map_a2);
+    prefetch_tensormap(&map_b0);
+    if (MODE == kGemm1) prefetch_tensormap(&map_b1);
+  }
+  if (warp == 2) tmem_alloc(&tmem_base_sh, kTmemCols);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+  volatile int* abort_v = &abort_flag;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, issued_par = 0;  // per stage: ever issued / parity of last issue
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int e = tile / (p.tiles_m * p.tiles_n);
+      const int rem = tile % (p.tiles_m * p.tiles_n);
+      const int m0 = (rem / p.tiles_n) * kBM;
+      const int n0 = (rem % p.tiles_n) * n_per_tile;
+      int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+      if (MODE == kGemm1) {
+        const int32_t* ir = p.idx + (int64_t)e * p.Ce;
+        const int s = m0 + 4 * lane;
+        r0 = s + 0 < p.Ce ? ir[s + 0] : 0;
+        r1 = s + 1 < p.Ce ? ir[s + 1] : 0;
+        r2 = s + 2 < p.Ce ? ir[s + 2] : 0;
+        r3 = s + 3 < p.Ce ? ir[s + 3] : 0;
+      }
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, kWaitNs);
+        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
+        __syncwarp();
+        const int k0 = kb * kBK;
+        uint8_t* b_dst = b_tile(stage);
+        if (MODE == kGemm1) {
+          tma_gather4(a_tile(stage, 0) + lane * 512, &map_a, &full_bar[stage], k0, r0, r1, r2,
+                      r3);
+          if (lane < 4) {
+            const CUtensorMap* mb = lane < 2 ? &map_b0 : &map_b1;
+            tma_load_3d(b_dst + lane * kBBoxBytes, mb, &full_bar[stage], n0 + 64 * (lane & 1),
+                        k0, e);
+          }
+        } else {
+          if (lane == 0)
+            tma_load_2d(a_tile(stage, 0), &map_a, &full_bar[stage], k0, e * p.Ce + m0);
+          if (C::kATiles == 2 && lane == 1)
+            tma_load_2d(a_tile(stage, 1), &map_a2, &full_bar[stage], k0, e * p.Ce + m0);
+          if (lane < 4)
+            tma_load_3d(b_dst + lane * kBBoxBytes, &map_b0, &full_bar[stage], n0 + 64 * lane,
+                        k0, e);
+        }
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    if (*abort_v && lane == 0) {
+      // let every copy this CTA issued land before the CTA can exit
+      int dummy = 0;
+      for (int s = 0; s < kStages; ++s)
+        if (issued_mask & (1u << s))
+          mbar_wait(&full_bar[s], (issued_par >> s) & 1u, &dummy, kDrainNs);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one thread) ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kBM, 256, 1);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        if (!(ok = mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_v, kWaitNs))) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!(ok = mbar_wait(&full_bar[stage], phase, abort_v, kWaitNs))) break;
+          tc_fence_after();
+          const uint32_t b_addr = smem_u32(b_tile(stage));
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, kBBoxBytes, 1024);
+#pragma unroll
+            for (int h = 0; h < C::kATiles; ++h) {
+              const uint64_t ad = sdesc_sw128(smem_u32(a_tile(stage, h)) + kk * 32, 16, 1024);
+              mma_bf16(d_tmem, ad, bd, idesc, (kb | kk | h) != 0);
+            }
+          }
+          mma_commit(&empty_bar[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull_bar[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      // every MMA issued above has completed once drain_bar flips
+      mma_commit(&drain_bar);
+      int dummy = 0;
+      mbar_wait(&drain_bar, 0, &dummy, kDrainNs);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;       // accumulator row = tile row
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int e = tile / (p.tiles_m * p.tiles_n);
+      const int rem = tile % (p.tiles_m * p.tiles_n);
+      const int m0 = (rem / p.tiles_n) * kBM;
+      const int n0 = (rem % p.tiles_n) * n_per_tile;
+      int w = 1;
+      if (lane == 0) w = mbar_wait(&tfull_bar[acc], acc_phase, abort_v, kWaitNs);
+      if (__shfl_sync(0xffffffffu, w, 0) == 0) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * kAccCols;
+      const int s = m0 + row;
+      const bool valid = s < p.Ce;
+      const int64_t orow = ((int64_t)e * p.Ce + (valid ? s : 0)) * p.N;
+      if (MODE == kGemm1) {
+        __nv_bfloat16* hi = static_cast<__nv_bfloat16*>(p.out) + orow;
+        __nv_bfloat16* lo = static_cast<__nv_bfloat16*>(p.out_lo) + orow;
+#pragma unroll 1
+        for (int j0 = 0; j0 < 128; j0 += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(taddr + j0, g);
+          tmem_ld32(taddr + 128 + j0, u);
+          tmem_ld_wait();
+          float h[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            h[i] = silu_f32(__uint_as_float(g[i])) * __uint_as_float(u[i]);
+          uint32_t ph[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ph[i] = pack_bf16x2(h[2 * i], h[2 * i + 1]);
+          if (valid) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int f = n0 + j0 + 8 * v;
+              if (f < p.N) {
+                *reinterpret_cast<uint4*>(hi + f) =
+                    make_uint4(ph[4 * v], ph[4 * v + 1], ph[4 * v + 2], ph[4 * v + 3]);
+                if (SPLIT) {
+                  uint4 l;
+                  l.x = pack_lo_bf16x2(h[8 * v + 0], h[8 * v + 1], ph[4 * v + 0]);
+                  l.y = pack_lo_bf16x2(h[8 * v + 2], h[8 * v + 3], ph[4 * v + 1]);
+                  l.z = pack_lo_bf16x2(h[8 * v + 4], h[8 * v + 5], ph[4 * v + 2]);
+                  l.w = pack_lo_bf16x2(h[8 * v + 6], h[8 * v + 7], ph[4 * v + 3]);
+                  *reinterpret_cast<uint4*>(lo + f) = l;
+                }
+              }
+            }
+          }
+        }
+      } else {
+        const float gw = valid ? p.gate[(int64_t)e * p.Ce + s] : 0.f;
+#pragma unroll 1
+        for (int j0 = 0; j0 < 256; j0 += 32) {
+          uint32_t y[32];
+          tmem_ld32(taddr + j0, y);
+          tmem_ld_wait();
+          if (SPLIT) {
+            float* yr = static_cast<float*>(p.out) + orow;
+            if (valid) {
+#pragma unroll
+              for (int v = 0; v < 8; ++v) {
+                const int c = n0 + j0 + 4 * v;
+                if (c < p.N)
+                  *reinterpret_cast<float4*>(yr + c) = make_float4(
+                      gw * __uint_as_float(y[4 * v]), gw * __uint_as_float(y[4 * v + 1]),
+                      gw * __uint_as_float(y[4 * v + 2]), gw * __uint_as_float(y[4 * v + 3]));
+              }
+            }
+          } else {
+            __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.out) + orow;
+            uint32_t h[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              h[i] = pack_bf16x2(gw * __uint_as_float(y[2 * i]),
+                                 gw * __uint_as_float(y[2 * i + 1]));
+            if (valid) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const int c = n0 + j0 + 8 * v;
+                if (c < p.N)
+                  *reinterpret_cast<uint4*>(yr + c) =
+                      make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_flag) atomicOr(p.err, kErrTimeout);
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---- host side ----------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle. dims/box are innermost first; strides are the
+// byte strides of dims 1.. (rank - 1 entries).
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+              const uint64_t* strides, const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  uint32_t elem[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Weights [E, K, N] bf16, N contiguous: boxes of 64 N x 64 K of one expert.
+bool weight_map(CUtensorMap* m, const void* W, int E, int K, int N) {
+  uint64_t dims[3] = {(uint64_t)N, (uint64_t)K, (uint64_t)E};
+  uint64_t strides[2] = {(uint64_t)N * 2, (uint64_t)K * N * 2};
+  uint32_t box[3] = {64, 64, 1};
+  return make_map(m, W, 3, dims, strides, box);
+}
+
+// Rows of a [rows, cols] bf16 matrix, boxes of box_rows x 64 columns.
+bool rows_map(CUtensorMap* m, const void* base, int64_t rows, int cols, uint32_t box_rows) {
+  uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+  uint64_t strides[1] = {(uint64_t)cols * 2};
+  uint32_t box[2] = {64, box_rows};
+  return make_map(m, base, 2, dims, strides, box);
+}
+
+template <int MODE, bool SPLIT>
+cudaError_t launch(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b0,
+                   const CUtensorMap& b1, const Params& p, int sm_count, cudaStream_t st) {
+  auto k = grouped_gemm_kernel<MODE, SPLIT>;
+  const size_t smem = Cfg<MODE, SPLIT>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
+  k<<<grid, kThreads, smem, st>>>(a, a2, b0, b1, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool experts_sm100_supported(const Shape& s) {
+  return s.d >= 64 && s.F >= 64 && (int64_t)s.E * s.Ce >= kBM && s.d % 8 == 0 &&
+         s.F % 8 == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1,
+                               const void* W3, const Shape& s, bool split, void* H_hi,
+                               void* H_lo, unsigned* err, int sm_count, cudaStream_t st) {
+  CUtensorMap ma, mb0, mb1;
+  if (!rows_map(&ma, x, s.T, s.d, 1) || !weight_map(&mb0, W1, s.E, s.d, s.F) ||
+      !weight_map(&mb1, W3, s.E, s.d, s.F))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.Ce = s.Ce; p.K = s.d; p.N = s.F;
+  p.tiles_m = (int)ceil_div(s.Ce, kBM);
+  p.tiles_n = (int)ceil_div(s.F, 128);
+  p.num_tiles = s.E * p.tiles_m * p.tiles_n;
+  p.idx = idx; p.gate = nullptr; p.out = H_hi; p.out_lo = H_lo; p.err = err;
+  return split ? launch<kGemm1, true>(ma, ma, mb0, mb1, p, sm_count, st)
+               : launch<kGemm1, false>(ma, ma, mb0, mb1, p, sm_count, st);
+}
+
+cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
+                               const void* W2, const Shape& s, bool split, void* Y, unsigned* err,
+                               int sm_count, cudaStream_t st) {
+  CUtensorMap ma, ma2, mb;
+  const int64_t rows = (int64_t)s.E * s.Ce;
+  if (!rows_map(&ma, H_hi, rows, s.F, kBM) || !weight_map(&mb, W2, s.E, s.F, s.d))
+    return cudaErrorInvalidValue;
+  if (split && !rows_map(&ma2, H_lo, rows, s.F, kBM)) return cudaErrorInvalidValue;
+  if (!split) ma2 = ma;
+  Params p;
+  p.Ce = s.Ce; p.K = s.F; p.N = s.d;
+  p.tiles_m = (int)ceil_div(s.Ce, kBM);
+  p.tiles_n = (int)ceil_div(s.d, 256);
+  p.num_tiles = s.E * p.tiles_m * p.tiles_n;
+  p.idx = nullptr; p.gate = gate; p.out = Y; p.out_lo = nullptr; p.err = err;
+  return split ? launch<kGemm2, true>(ma, ma2, mb, mb, p, sm_count, st)
+               : launch<kGemm2, false>(ma, ma2, mb, mb, p, sm_count, st);
+}
+
+}  // namespace nmoe

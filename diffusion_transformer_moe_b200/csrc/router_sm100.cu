@@ -1,0 +1,292 @@
+// Router GEMM + score function on the tensor cores, for bf16 inputs.
+//
+// NucleusMoE-Image walkthrough, section 6.2: gate = Linear(hidden, experts, no bias),
+// scored by softmax (or sigmoid), then viewed per expert. logits[t, e] = x[t, :] W_r[:, e].
+//
+// Precision: the scores must match an fp64 reference to 1e-5 relative, and with
+// LogNormal-scaled tokens the logits reach |l| ~ 30, where a single fp32 accumulator
+// over d = 2048 drifts by more than that (tensor-core accumulation also truncates). So
+// the MMAs accumulate only 32-long k-chunks in TMEM (two chunk slices per 64-wide
+// k-block), and the epilogue warps read every chunk back with tcgen05.ld and add it to
+// fp64 running sums in registers. Max, exp and the normalisation run in fp64; each
+// score is rounded once to fp32.
+//
+// One CTA per 128 tokens. Warp 0 streams x tiles and W_r tiles with TMA into a 6-stage
+// ring; warp 1 (one thread) issues tcgen05.mma (M = 128, N = E rounded up to 64, K = 16)
+// into a ring of TMEM chunk buffers; 4*G epilogue warps (G = ceil(E/32)) each own 32
+// tokens x 32 experts. Every wait is bounded.
+#include <cudaTypedefs.h>
+
+#include "router_sm100.cuh"
+#include "sm100_ptx.cuh"
+
+namespace nmoe {
+namespace {
+
+using namespace ptx;
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kStages = 6;
+constexpr int kABytes = kBM * kBK * 2;     // 16 KB
+constexpr int kBBoxBytes = 64 * kBK * 2;   // 8 KB: 64 experts x 64 k
+constexpr int kMaxE = 128;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint64_t kDrainNs = 20000000ull;
+
+struct Params {
+  int T, d, E, S;
+  int epad;         // N of the MMA: E rounded up to 64
+  int nbox;         // epad / 64
+  int nbuf;         // TMEM chunk buffers of 2 * epad columns
+  int score_fn;
+  const float* bias;
+  float* scores;
+  float* scores_t;
+  unsigned* err;
+};
+
+template <int G>
+__global__ void __launch_bounds__(64 + 128 * G, 1)
+router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
+                    const __grid_constant__ CUtensorMap map_w, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int b_bytes = p.nbox * kBBoxBytes;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kABytes;
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t tfull_bar[8], tempty_bar[8], drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = (p.d + kBK - 1) / kBK;
+  const int t0 = blockIdx.x * kBM;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) { mbar_init(&full_bar[i], 1); mbar_init(&empty_bar[i], 1); }
+    for (int i = 0; i < p.nbuf; ++i) { mbar_init(&tfull_bar[i], 1); mbar_init(&tempty_bar[i], 4 * G); }
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&map_x);
+    prefetch_tensormap(&map_w);
+  }
+  if (warp == 2) tmem_alloc(&tmem_base_sh, 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+  volatile int* abort_v = &abort_flag;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, issued_par = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, kWaitNs)) break;
+        mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
+        tma_load_2d(sA + stage * kABytes, &map_x, &full_bar[stage], kb * kBK, t0);
+        for (int j = 0; j < p.nbox; ++j)
+          tma_load_2d(sB + stage * b_bytes + j * kBBoxBytes, &map_w, &full_bar[stage], 64 * j,
+                      kb * kBK);
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      if (*abort_v) {
+        int dummy = 0;
+        for (int s = 0; s < kStages; ++s)
+          if (issued_mask & (1u << s))
+            mbar_wait(&full_bar[s], (issued_par >> s) & 1u, &dummy, kDrainNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(kBM, p.epad, 1);
+      int stage = 0, buf = 0;
+      uint32_t phase = 0, buf_phase = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(&tempty_bar[buf], buf_phase ^ 1, abort_v, kWaitNs)) break;
+        if (!mbar_wait(&full_bar[stage], phase, abort_v, kWaitNs)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(sA + stage * kABytes);
+        const uint32_t b_addr = smem_u32(sB + stage * b_bytes);
+        const uint32_t d0 = tmem_base + buf * 2 * p.epad;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, kBBoxBytes, 1024);
+          // chunk slice kk / 2, restarted at the first MMA of each slice
+          mma_bf16(d0 + (kk >> 1) * p.epad, ad, bd, idesc, kk & 1);
+        }
+        mma_commit(&empty_bar[stage]);
+        mma_commit(&tfull_bar[buf]);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        if (++buf == p.nbuf) { buf = 0; buf_phase ^= 1; }
+      }
+      mma_commit(&drain_bar);
+      int dummy = 0;
+      mbar_wait(&drain_bar, 0, &dummy, kDrainNs);
+    }
+  } else {
+    // ---------------- epilogue: 32 tokens x 32 experts per warp ----------------
+    const int q = warp & 3;
+    const int g = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    double acc[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc[j] = 0.0;
+    int buf = 0;
+    uint32_t buf_phase = 0;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      int w = 1;
+      if (lane == 0) w = mbar_wait(&tfull_bar[buf], buf_phase, abort_v, kWaitNs);
+      if (__shfl_sync(0xffffffffu, w, 0) == 0) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t taddr =
+          tmem_base + ((uint32_t)(q * 32) << 16) + buf * 2 * p.epad + g * 32;
+      // two chunk slices x two halves of this warp's 32 experts, 16 columns at a time
+#pragma unroll
+      for (int part = 0; part < 4; ++part) {
+        uint32_t c[16];
+        tmem_ld16(taddr + (part >> 1) * p.epad + (part & 1) * 16, c);
+        tmem_ld_wait();
+        if (part == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[(part & 1) * 16 + j] += (double)__uint_as_float(c[j]);
+      }
+      if (++buf == p.nbuf) { buf = 0; buf_phase ^= 1; }
+    }
+    // Every MMA has completed once the last chunk was read, so the stage ring is idle:
+    // keep the fp64 logits there, [128][E + 1], and finish row by row.
+    double* lg = reinterpret_cast<double*>(smem);
+    const int ld = p.E + 1;
+    const int e0 = g * 32;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (e0 + j < p.E) lg[row * ld + e0 + j] = acc[j];
+    const int nthreads = 128 * G;
+    const int ew = warp - 2;  // epilogue warp 0 .. 4G-1
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+    for (int r = ew; r < kBM; r += 4 * G) {
+      double* lr = lg + r * ld;
+      const int t = t0 + r;
+      if (p.bias != nullptr && t < p.T) {
+        const float* b = p.bias + (int64_t)(t / p.S) * p.E;
+        for (int e = lane; e < p.E; e += 32) lr[e] += (double)b[e];
+      }
+      if (p.score_fn == NMOE_SCORE_SOFTMAX) {
+        double m = -INFINITY;
+        for (int e = lane; e < p.E; e += 32) m = fmax(m, lr[e]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+        double z = 0.0;
+        for (int e = lane; e < p.E; e += 32) {
+          double v = exp(lr[e] - m);
+          lr[e] = v;
+          z += v;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        for (int e = lane; e < p.E; e += 32) lr[e] = lr[e] / z;
+      } else {
+        for (int e = lane; e < p.E; e += 32) lr[e] = 1.0 / (1.0 + exp(-lr[e]));
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+    if (ok) {
+      const int tid = threadIdx.x - 64;
+      const int rows = min(kBM, p.T - t0);
+      for (int i = tid; i < rows * p.E; i += nthreads) {
+        const int r = i / p.E, e = i - r * p.E;
+        p.scores[(int64_t)(t0 + r) * p.E + e] = (float)lg[r * ld + e];
+      }
+      for (int i = tid; i < kBM * p.E; i += nthreads) {
+        const int e = i / kBM, r = i - e * kBM;
+        if (r < rows) p.scores_t[(int64_t)e * p.T + t0 + r] = (float)lg[r * ld + e];
+      }
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_flag) atomicOr(p.err, kErrTimeout);
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+bool map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_in,
+            uint32_t box_out) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  uint64_t dims[2] = {inner, outer};
+  uint64_t strides[1] = {inner * 2};
+  uint32_t box[2] = {box_in, box_out};
+  uint32_t elem[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool router_sm100_supported(const Shape& s) {
+  return s.E >= 1 && s.E <= kMaxE && s.T >= kBM && s.d >= kBK && s.d % 8 == 0 &&
+         encode_fn() != nullptr;
+}
+
+cudaError_t launch_router_sm100(const void* x, const void* W_r, const Shape& s,
+                                nmoe_score_fn fn, const float* bias, float* scores,
+                                float* scores_t, unsigned* err, cudaStream_t st) {
+  Params p;
+  p.T = s.T; p.d = s.d; p.E = s.E; p.S = s.S;
+  p.epad = (int)ceil_div(s.E, 64) * 64;
+  p.nbox = p.epad / 64;
+  p.nbuf = 512 / (2 * p.epad);
+  if (p.nbuf > 8) p.nbuf = 8;
+  p.score_fn = (int)fn;
+  p.bias = bias; p.scores = scores; p.scores_t = scores_t; p.err = err;
+  CUtensorMap mx, mw;
+  if (!map_2d(&mx, x, (uint64_t)s.d, (uint64_t)s.T, 64, kBM) ||
+      !map_2d(&mw, W_r, (uint64_t)s.E, (uint64_t)s.d, 64, 64))
+    // a shape the tensor maps cannot describe: the CUDA-core router computes the same
+    return launch_router_simt(x, W_r, s, NMOE_BF16, fn, bias, scores, scores_t, st);
+  size_t smem = (size_t)kStages * (kABytes + p.nbox * kBBoxBytes);
+  const size_t logits = sizeof(double) * kBM * (size_t)(s.E + 1);
+  smem = (smem > logits ? smem : logits) + 1024;
+  const int G = (int)ceil_div(s.E, 32);
+  auto k = G == 1 ? router_sm100_kernel<1>
+         : G == 2 ? router_sm100_kernel<2>
+         : G == 3 ? router_sm100_kernel<3>
+                  : router_sm100_kernel<4>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<(unsigned)ceil_div(s.T, kBM), 64 + 128 * G, smem, st>>>(mx, mw, p);
+  return cudaGetLastError();
+}
+
+}  // namespace nmoe

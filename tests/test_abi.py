@@ -1,0 +1,103 @@
+"""The C ABI library loads, exports what include/nmoe.h declares, and rejects bad
+arguments on the host before touching CUDA (CPU only: no compute call is made)."""
+
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import diffusion_transformer_moe_b200 as nm
+from diffusion_transformer_moe_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"NMOE_API\s+[\w\s\*]*?\b(nmoe_\w+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = nm.lib()
+    declared = _declared()
+    assert declared, "no declarations found"
+    assert declared == set(L.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_options_struct_matches_defaults():
+    o = L.Options()
+    nm.lib().nmoe_options_init(C.byref(o))
+    assert (o.dtype, o.score_fn, o.combine, o.n_segments, o.host_io) == (0, 0, 0, 1, 0)
+    assert o.route_scale == 1.0 and not o.workspace and not o.trace
+
+
+def test_status_strings_and_build_info():
+    lib = nm.lib()
+    for s in range(8):
+        assert lib.nmoe_status_str(s)
+    assert b"sm_100a" in lib.nmoe_build_info()
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced (checks fail first)
+
+
+@pytest.mark.parametrize("args,expect", [
+    (dict(T=0), 1), (dict(E=0), 1), (dict(E=257), 1), (dict(C=0), 1), (dict(C=65), 1),
+    (dict(d=12), 2), (dict(F=20), 2), (dict(x=0), 1), (dict(x=FAKE + 8), 1),
+    (dict(out=FAKE), 1),
+])
+def test_forward_rejects_bad_arguments_on_host(args, expect):
+    a = dict(x=FAKE, W_r=FAKE + 4096, W1=FAKE + 8192, W3=FAKE + 12288, W2=FAKE + 16384,
+             T=64, d=16, E=4, F=16, C=8, out=FAKE + 32768)
+    a.update(args)
+    st = nm.lib().nmoe_forward(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], a["T"], a["d"],
+                               a["E"], a["F"], a["C"], a["out"], None)
+    assert st == expect
+
+
+def test_select_and_router_reject_bad_arguments_on_host():
+    lib = nm.lib()
+    # C larger than a segment
+    assert lib.nmoe_select(FAKE, 64, 4, 33, 2, FAKE, FAKE, None, None, None) == 1
+    # T not divisible by the segments
+    assert lib.nmoe_select(FAKE, 63, 4, 3, 2, FAKE, FAKE, None, None, None) == 1
+    # only one of tok_ptr / tok_ent
+    assert lib.nmoe_select(FAKE, 64, 4, 3, 1, FAKE, FAKE, FAKE, None, None) == 1
+    # misaligned idx
+    assert lib.nmoe_select(FAKE, 64, 4, 3, 1, FAKE + 4, FAKE, None, None, None) == 1
+    # no output at all
+    assert lib.nmoe_router(FAKE, FAKE, 64, 16, 4, 0, 0, None, 1, None, None, None) == 1
+    # bad score function
+    assert lib.nmoe_router(FAKE, FAKE, 64, 16, 4, 0, 7, None, 1, FAKE, None, None) == 1
+
+
+def test_workspace_size_accounts_for_every_buffer():
+    T, d, E, F, C_ = 8192, 2048, 64, 1024, 128
+    n = nm.workspace_size(T, d, E, F, C_)
+    Ce = E * C_
+    # default (split) intermediates: H as a bf16 hi/lo pair, Y in fp32 -> 4 bytes each
+    minimum = 4 * T * E * 2 + 4 * Ce * 3 + 4 * (T + 1) + 4 * Ce * F + 4 * Ce * d
+    assert minimum <= n <= minimum + 16 * 256
+    small = nm.workspace_size(T, d, E, F, C_, intermediate="bf16")
+    assert small == n - 2 * Ce * F - 2 * Ce * d
+    assert nm.workspace_size(T, d, E, F, T + 1) == 0  # invalid sizes give 0
+    host = nm.workspace_size(T, d, E, F, C_, host_io=True)
+    assert host >= n + 2 * 2 * T * d
+    host32 = nm.workspace_size(T, d, E, F, C_, host_io=True, out_f32=True)
+    assert host32 >= n + 2 * T * d + 4 * T * d
+
+
+def test_missing_gpu_is_reported_not_crashed():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    # valid arguments on a machine without a device: NMOE_ERR_NO_DEVICE
+    st = nm.lib().nmoe_forward(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 16, 4, 16, 8, FAKE + 64, None)
+    assert st == 7
