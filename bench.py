@@ -25,7 +25,6 @@ import json
 import os
 import re
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -40,8 +39,8 @@ L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 def _args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="1024px_cfg")
     ap.add_argument("--intermediate", choices=("split", "bf16"), default="split")
@@ -112,54 +111,66 @@ def _traffic(kernel_stage, workload):
 # ---- clocks during the timed region ----------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clocks and clock-event reasons every 10 ms through NVML (read only)."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.mx = None
+        self.reasons = set()
+        self.err = None
+        self._stop = threading.Event()
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except (OSError, ValueError):
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = self.gpu
+            if vis:
+                first = vis.split(",")[self.gpu].strip()
+                idx = int(first) if first.isdigit() else self.gpu
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.mx = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = f"nvml unavailable: {type(e).__name__}"
+            return
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for name, bit in self.REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception as e:
+                self.err = f"nvml sample failed: {type(e).__name__}"
+                return
+            self._stop.wait(0.01)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, mx, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
-            f = [s.strip() for s in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.err and not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err]}
+        self._stop.set()
+        self.t.join(timeout=2)
+        if not self.samples:
+            self._sample()
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.mx,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 # ---- the CPU oracle (reference arm and cpu_baseline) --------------------------------------
@@ -181,35 +192,70 @@ def _oracle_threads():
         return os.cpu_count() or 1
 
 
-def _time_oracle(w, args, seed, reps):
-    """Seconds per full oracle layer over `reps` repetitions of the whole workload."""
+def _oracle_step(w, data, experts=None):
+    """One oracle pass: router, scores and selection over all tokens, then the SwiGLU
+    experts and combine for `experts` (all experts if None). Returns (seconds spent,
+    seconds the whole layer would take: the expert part scaled to all E experts)."""
     from oracle import nmoe_oracle as O
-    x, W_r, W1, W3, W2 = args
+    import numpy as np
+    x, W_r, W1, W3, W2 = data
     t0 = time.perf_counter()
-    for _ in range(reps):
-        O.layer(x, W_r, W1, W3, W2, w.C)
-    return (time.perf_counter() - t0) / reps
+    p = O.scores_from_logits(O.router_logits(x, W_r))
+    idx = O.select(O.round_f32(p), w.C)
+    wts = O.combine_weights(p, idx)
+    t1 = time.perf_counter()
+    ex = range(w.E) if experts is None else experts
+    out = np.zeros_like(x)
+    for e in ex:
+        out[idx[e]] += wts[e][:, None] * O.swiglu_ffn(x[idx[e]], W1[e], W3[e], W2[e])
+    t2 = time.perf_counter()
+    scale = w.E / max(1, len(ex))
+    return t2 - t0, (t1 - t0) + scale * (t2 - t1)
+
+
+def _sample_plan(w, data, budget_s):
+    """Experts per step so that one step stays within budget_s (whole layer if it fits)."""
+    _, full = _oracle_step(w, data)
+    if full <= budget_s:
+        return None, f"the whole {w.name} layer (all {w.T} tokens, all {w.E} experts)"
+    k = max(1, int(w.E * budget_s / full))
+    return k, (f"router, scores and selection over all {w.T} tokens of {w.name}, plus the "
+               f"SwiGLU experts and combine of {k} of the {w.E} experts (rotating), the "
+               f"expert time scaled to all {w.E} experts")
 
 
 def cpu_baseline(w, seed=0, budget_s=12.0):
-    args = _oracle_inputs(w, seed)
-    one = _time_oracle(w, args, seed, 1)
-    reps = max(1, int(budget_s / max(one, 1e-3)))
-    per = _time_oracle(w, args, seed, reps)
-    return {"value": w.T / per, "unit": "tokens/s", "cores": _oracle_threads(),
-            "kind": "oracle",
-            "sample": f"the whole {w.name} layer (all {w.T} tokens, all {w.E} experts), "
-                      f"fp64 numpy oracle, {reps} repetitions after one untimed"}
+    data = _oracle_inputs(w, seed)
+    k, what = _sample_plan(w, data, budget_s)
+    spent, est, n = 0.0, 0.0, 0
+    while spent < budget_s:
+        ex = None if k is None else [(n * k + j) % w.E for j in range(k)]
+        s_, e_ = _oracle_step(w, data, ex)
+        spent += s_
+        est += e_
+        n += 1
+    return {"value": w.T * n / est, "unit": "tokens/s", "cores": _oracle_threads(),
+            "kind": "oracle", "sample": f"{what}; fp64 numpy oracle, {n} steps after one "
+                                        f"untimed, {spent:.1f} s of CPU time"}
 
 
 def run_reference(args, w, rank):
     if rank != 0:
         return
     data = _oracle_inputs(w, 0)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    k, what = _sample_plan(w, data, budget)
+    step = 0
+
+    def one():
+        nonlocal step
+        ex = None if k is None else [(step * k + j) % w.E for j in range(k)]
+        step += 1
+        return _oracle_step(w, data, ex)[1]
+
     for _ in range(args.warmup):
-        _time_oracle(w, data, 0, 1)
-    per = [_time_oracle(w, data, 0, 1) for _ in range(args.steps)]
-    tot = sum(per)
+        one()
+    tot = sum(one() for _ in range(args.steps))
     value = w.T * args.steps / tot
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
@@ -218,8 +264,7 @@ def run_reference(args, w, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _workload_config(w, "fp64 oracle"),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _oracle_threads(),
-                         "kind": "oracle",
-                         "sample": f"each step is the whole {w.name} layer on the host cores"},
+                         "kind": "oracle", "sample": f"each step: {what}"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
