@@ -32,7 +32,7 @@ EXPORTS = (
     "nmoe_options_init", "nmoe_router", "nmoe_select", "nmoe_forward", "nmoe_forward_ex",
     "nmoe_workspace_size", "nmoe_get_last_error", "nmoe_status_str", "nmoe_trace_create",
     "nmoe_trace_read", "nmoe_trace_reset", "nmoe_trace_destroy", "nmoe_stage_name",
-    "nmoe_build_info",
+    "nmoe_build_info", "nmoe_forward_noalloc",
 )
 
 
@@ -100,6 +100,8 @@ def lib() -> C.CDLL:
             L.nmoe_stage_name.restype = C.c_char_p
             L.nmoe_build_info.argtypes = []
             L.nmoe_build_info.restype = C.c_char_p
+            L.nmoe_forward_noalloc.argtypes = [_vp] * 5 + [_i64] * 5 + [_vp, _vp]
+            L.nmoe_forward_noalloc.restype = C.c_int
             _lib = L
     return _lib
 

@@ -182,6 +182,29 @@ NMOE_API nmoe_status nmoe_trace_reset(nmoe_trace* tr);
 NMOE_API void nmoe_trace_destroy(nmoe_trace* tr);
 NMOE_API const char* nmoe_stage_name(int stage);
 
+/* The whole layer, like nmoe_forward (bf16, default options), for callers that cannot
+ * allocate device memory while they run it: code under a memory manager that owns all
+ * of the device's memory (a caching allocator, a pre-partitioned arena), real-time
+ * paths that must not enter the CUDA allocator, or hosts that forbid allocation after
+ * start-up. The pages describe no such entry point; it exists for those callers.
+ *   - Scratch lives in one fixed array of NMOE_NOALLOC_SCRATCH_BYTES (128 MiB) in device
+ *     memory, reserved on every device that loads this library and held until the
+ *     process exits. The call makes no cudaMalloc, cudaFree or other allocation.
+ *   - Sizes whose scratch (nmoe_workspace_size with default options) exceeds that
+ *     capacity are rejected with NMOE_ERR_WORKSPACE before anything is enqueued
+ *     (T = 8192, d = 2048, E = 64, F = 1024, C = 128 needs ~100 MiB and fits).
+ *   - The first call on a device looks the array's address up on that device; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (nothing in it needs to start at zero). Calls whose work overlaps on the
+ *     GPU (other streams, or concurrent host threads) race on it: order them.
+ * Arguments, layouts, ownership and the other errors are those of nmoe_forward. */
+#define NMOE_NOALLOC_SCRATCH_BYTES ((size_t)128 << 20)
+NMOE_API nmoe_status nmoe_forward_noalloc(const void* x, const void* W_r, const void* W1,
+                                          const void* W3, const void* W2, int64_t T,
+                                          int64_t d, int64_t E, int64_t F, int64_t C,
+                                          void* out, nmoe_stream_t stream);
+
 /* Build identification: a static string (architecture, kernel variants). */
 NMOE_API const char* nmoe_build_info(void);
 
