@@ -44,6 +44,8 @@ def _args():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="1024px_cfg")
     ap.add_argument("--intermediate", choices=("split", "bf16"), default="split")
+    ap.add_argument("--tma-gather", action="store_true",
+                    help="gather the gate/up GEMM's token rows with TMA tile::gather4")
     return ap.parse_args()
 
 
@@ -294,7 +296,7 @@ def run_ours(args, w, rank, world, local_rank, dist):
 
     def step(tr=None):
         nm.forward(x, W_r, W1, W3, W2, w.C, out=out, workspace=ws, intermediate=inter,
-                   trace=tr)
+                   trace=tr, tma_gather=args.tma_gather)
 
     def barrier():
         if dist is not None:
@@ -331,7 +333,7 @@ def run_ours(args, w, rank, world, local_rank, dist):
     out_host = torch.empty_like(x_host).pin_memory()
     for _ in range(max(1, args.warmup // 2)):
         nm.forward(x_host, W_r, W1, W3, W2, w.C, out=out_host, workspace=ws,
-                   intermediate=inter, host_io=True)
+                   intermediate=inter, host_io=True, tma_gather=args.tma_gather)
     torch.cuda.synchronize()
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
@@ -341,7 +343,7 @@ def run_ours(args, w, rank, world, local_rank, dist):
         flush.zero_()
         e2e_ev[i][0].record(stream)
         nm.forward(x_host, W_r, W1, W3, W2, w.C, out=out_host, workspace=ws,
-                   intermediate=inter, host_io=True)
+                   intermediate=inter, host_io=True, tma_gather=args.tma_gather)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -382,7 +384,8 @@ def run_ours(args, w, rank, world, local_rank, dist):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(_workload_config(w, inter), parallelism=f"replicas x{world}"),
+        "config": dict(_workload_config(w, inter), parallelism=f"replicas x{world}",
+                       gather="tma gather4" if args.tma_gather else "cp.async"),
         "tflops": flops / per_step_s / 1e12,
         "tensor_frac_of_layer": flops / per_step_s / 1e12 / peaks["tensor_sustained"],
         "roofline": roof,

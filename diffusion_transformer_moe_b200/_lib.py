@@ -49,6 +49,7 @@ class Options(C.Structure):
         ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t),
         ("scores_out", C.c_void_p), ("idx_out", C.c_void_p), ("host_io", C.c_int),
         ("trace", C.c_void_p), ("intermediate", C.c_int), ("out_f32", C.c_int),
+        ("tma_gather", C.c_int),
     ]
 
 
@@ -137,7 +138,8 @@ def _dev(t: torch.Tensor, name: str) -> None:
 
 def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
             n_segments=1, router_bias=None, workspace=None, scores_out=None, idx_out=None,
-            host_io=False, trace=None, intermediate="split", out_f32=False) -> Options:
+            host_io=False, trace=None, intermediate="split", out_f32=False,
+            tma_gather=False) -> Options:
     o = Options()
     lib().nmoe_options_init(C.byref(o))
     o.dtype = dtype
@@ -155,6 +157,7 @@ def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
     o.trace = None if trace is None else trace.handle
     o.intermediate = INTERMEDIATE[intermediate]
     o.out_f32 = 1 if out_f32 else 0
+    o.tma_gather = 1 if tma_gather else 0
     return o
 
 
@@ -190,7 +193,8 @@ def select(scores_t, C_: int, n_segments=1, csr=True, stream=None):
 def forward(x, W_r, W1, W3, W2, C_: int, out=None, stream=None, **opts):
     """The whole layer. ``opts`` are the nmoe_options fields (score_fn, combine,
     route_scale, n_segments, router_bias, workspace, scores_out, idx_out, trace,
-    intermediate, out_f32). With ``host_io=True`` x and out are pinned CPU tensors."""
+    intermediate, out_f32, tma_gather). With ``host_io=True`` x and out are pinned CPU
+    tensors."""
     host_io = bool(opts.get("host_io", False))
     for n, t in (("W_r", W_r), ("W1", W1), ("W3", W3), ("W2", W2)):
         _dev(t, n)

@@ -242,8 +242,8 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   // (shapes the tcgen05 kernels do not take) H is one fp32 array of the same size.
   void* H_lo = static_cast<char*>(H) + sizeof(uint16_t) * (size_t)s.E * s.Ce * s.F;
   if (e == cudaSuccess)
-    e = tc ? nmoe::launch_gemm1_sm100(xd, idx, W1, W3, s, split, H, H_lo, ds->err,
-                                      ds->sm_count, st)
+    e = tc ? nmoe::launch_gemm1_sm100(xd, idx, W1, W3, s, split, o.tma_gather != 0, H, H_lo,
+                                      ds->err, ds->sm_count, st)
            : nmoe::launch_gemm1_simt(xd, idx, W1, W3, s, o.dtype, split, H, st);
   mark(4);
   if (e == cudaSuccess)
@@ -286,6 +286,7 @@ void nmoe_options_init(nmoe_options* o) {
   o->trace = nullptr;
   o->intermediate = NMOE_INTERMEDIATE_SPLIT;
   o->out_f32 = 0;
+  o->tma_gather = 0;
 }
 
 nmoe_status nmoe_router(const void* x, const void* W_r, int64_t T, int64_t d, int64_t E,

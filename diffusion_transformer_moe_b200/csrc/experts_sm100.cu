@@ -9,8 +9,12 @@
 //   gemm1: H[e, s, :] = silu(x[idx[e,s]] W1_e) * (x[idx[e,s]] W3_e)
 //   gemm2: Y[e*Ce + s, :] = gate[e, s] * (H[e, s, :] W2_e)
 //
-// Instead of permuting tokens into per-expert blocks, gemm1 gathers the 128 rows of an
-// A tile straight from x with TMA tile::gather4 (32 copies of 4 rows per k-block).
+// Instead of permuting tokens into per-expert blocks, gemm1 gathers the 128 rows of its
+// A tile straight from x. Two ways are built: four producer warps issuing 16-byte
+// cp.async copies into the 128-byte-swizzled tile (default), or TMA tile::gather4 (32
+// copies of 4 rows per k-block). On B200 the gather4 form caps gemm1 at about half the
+// HBM rate (measured: 201 us against 109 us for the same bytes as plain tiles at
+// T = 8192, d = 2048, E = 64, F = 1024), so cp.async is the default.
 //
 // Intermediate precision. With SPLIT (the default), H is stored as a pair of bf16
 // arrays hi = bf16(h), lo = bf16(h - hi) (about 16 significant bits), gemm2 runs both
@@ -19,14 +23,16 @@
 // moves ~10% fewer bytes but lets large-magnitude tokens drift by ~0.1-0.2 absolute.
 //
 // One persistent CTA per SM walks tiles (expert, 128-row block, N block) in a static
-// round-robin. Warp roles: warp 0 issues TMA copies into a shared-memory ring, warp 1
-// (one thread) issues tcgen05.mma into a double-buffered TMEM accumulator (2 x 256 fp32
-// columns), warps 2-5 run the epilogue (tcgen05.ld, SwiGLU or gate scale, stores) while
-// the next tile's MMAs run. Tile: M = 128 rows, K = 64 per stage, N = 256 accumulator
-// columns (gemm1: 128 gate + 128 up columns of F; gemm2: 256 columns of d). A is
-// K-major, B (the weights, [E, K, N] with N contiguous) is MN-major; both use the
-// 128-byte swizzle. Every wait is bounded; a wait that runs out sets the device error
-// word and the kernel drains its copies and MMAs, frees TMEM and returns.
+// round-robin. Warp roles: warp 0 issues the TMA copies (weights, and A unless cp.async
+// gathers it), warp 1 allocates TMEM and one of its threads issues tcgen05.mma into a
+// double-buffered accumulator (2 x 256 fp32 columns), the cp.async warps (gemm1) fill
+// the A tiles, and eight epilogue warps (two per TMEM lane quarter) drain a finished
+// accumulator with tcgen05.ld while the next tile's MMAs run. Tile: M = 128 rows,
+// K = 64 per stage, N = 256 accumulator columns (gemm1: 128 gate + 128 up columns of F;
+// gemm2: 256 columns of d). A is K-major, B (the weights, [E, K, N] with N contiguous)
+// is MN-major; both use the 128-byte swizzle. Every wait is bounded; a wait that runs
+// out sets the device error word and the kernel drains its copies and MMAs, frees TMEM
+// and returns.
 #include <cudaTypedefs.h>
 
 #include "experts_sm100.cuh"
@@ -44,17 +50,23 @@ constexpr int kBBoxBytes = 64 * kBK * 2;        // 8 KB: 64 N x 64 K
 constexpr int kBBytes = 4 * kBBoxBytes;         // 32 KB: N = 256
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 2 * kAccCols;
-constexpr int kThreads = 192;
 constexpr uint64_t kWaitNs = 2000000000ull;     // 2 s per wait
 constexpr uint64_t kDrainNs = 20000000ull;      // 20 ms per drain wait
 
 enum { kGemm1 = 0, kGemm2 = 1 };
+enum { kGatherLsu = 0, kGatherTma4 = 1 };       // how gemm1 fetches its token rows
 
-template <int MODE, bool SPLIT>
+template <int MODE, bool SPLIT, int GATHER>
 struct Cfg {
+  static constexpr bool kLsuA = MODE == kGemm1 && GATHER == kGatherLsu;
   static constexpr int kATiles = (MODE == kGemm2 && SPLIT) ? 2 : 1;
   static constexpr int kStageBytes = kATiles * kABytes + kBBytes;
   static constexpr int kStages = (MODE == kGemm2 && SPLIT) ? 3 : 4;
+  static constexpr int kAWarps = kLsuA ? 4 : 0;          // cp.async gather warps
+  static constexpr int kEpiWarps = 8;                    // two per TMEM lane quarter
+  static constexpr int kEpiWarp0 = 2 + kAWarps;
+  static constexpr int kThreads = 32 * (2 + kAWarps + kEpiWarps);
+  static constexpr int kFullCount = 1 + 32 * kAWarps;    // TMA arrive + one per gather thread
   static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
 };
 
@@ -70,7 +82,11 @@ struct Params {
   unsigned* err;
 };
 
-__device__ __forceinline__ float silu_f32(float g) { return g / (1.f + expf(-g)); }
+// silu(g) = g * sigmoid(g); the reciprocal is correctly rounded and exp's error is a
+// few ulp, far below the hi/lo split's 16 bits. g -> -inf gives -0, g -> +inf gives g.
+__device__ __forceinline__ float silu_f32(float g) {
+  return g * __frcp_rn(1.f + __expf(-g));
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -84,13 +100,14 @@ __device__ __forceinline__ uint32_t pack_lo_bf16x2(float a, float b, uint32_t hi
   return pack_bf16x2(a - f.x, b - f.y);
 }
 
-template <int MODE, bool SPLIT>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int MODE, bool SPLIT, int GATHER>
+__global__ void __launch_bounds__(Cfg<MODE, SPLIT, GATHER>::kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                     const __grid_constant__ CUtensorMap map_a2,
                     const __grid_constant__ CUtensorMap map_b0,
-                    const __grid_constant__ CUtensorMap map_b1, const Params p) {
-  using C = Cfg<MODE, SPLIT>;
+                    const __grid_constant__ CUtensorMap map_b1, const __nv_bfloat16* x,
+                    const Params p) {
+  using C = Cfg<MODE, SPLIT, GATHER>;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -108,17 +125,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
   auto b_tile = [&](int s) { return smem + s * C::kStageBytes + C::kATiles * kABytes; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) { mbar_init(&full_bar[i], 1); mbar_init(&empty_bar[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&tfull_bar[i], 1); mbar_init(&tempty_bar[i], 4); }
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full_bar[i], C::kFullCount);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull_bar[i], 1);
+      mbar_init(&tempty_bar[i], C::kEpiWarps);
+    }
     mbar_init(&drain_bar, 1);
     abort_flag = 0;
     fence_mbar_init();
-    prefetch_tensormap(&map_a);
+    if (!C::kLsuA) prefetch_tensormap(&map_a);
     if (C::kATiles == 2) prefetch_tensormap(&map_a2);
     prefetch_tensormap(&map_b0);
     if (MODE == kGemm1) prefetch_tensormap(&map_b1);
   }
-  if (warp == 2) tmem_alloc(&tmem_base_sh, kTmemCols);
+  if (warp == 1) tmem_alloc(&tmem_base_sh, kTmemCols);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
@@ -135,7 +158,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       const int m0 = (rem / p.tiles_n) * kBM;
       const int n0 = (rem % p.tiles_n) * n_per_tile;
       int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
-      if (MODE == kGemm1) {
+      if (MODE == kGemm1 && !C::kLsuA) {
         const int32_t* ir = p.idx + (int64_t)e * p.Ce;
         const int s = m0 + 4 * lane;
         r0 = s + 0 < p.Ce ? ir[s + 0] : 0;
@@ -149,13 +172,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, kWaitNs);
         ok = __shfl_sync(0xffffffffu, w, 0) != 0;
         if (!ok) break;
-        if (lane == 0) mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
+        if (lane == 0)
+          mbar_arrive_expect_tx(&full_bar[stage],
+                                C::kLsuA ? (uint32_t)kBBytes : (uint32_t)C::kStageBytes);
         __syncwarp();
         const int k0 = kb * kBK;
         uint8_t* b_dst = b_tile(stage);
         if (MODE == kGemm1) {
-          tma_gather4(a_tile(stage, 0) + lane * 512, &map_a, &full_bar[stage], k0, r0, r1, r2,
-                      r3);
+          if (!C::kLsuA)
+            tma_gather4(a_tile(stage, 0) + lane * 512, &map_a, &full_bar[stage], k0, r0, r1,
+                        r2, r3);
           if (lane < 4) {
             const CUtensorMap* mb = lane < 2 ? &map_b0 : &map_b1;
             tma_load_3d(b_dst + lane * kBBoxBytes, mb, &full_bar[stage], n0 + 64 * (lane & 1),
@@ -183,6 +209,53 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         if (issued_mask & (1u << s))
           mbar_wait(&full_bar[s], (issued_par >> s) & 1u, &dummy, kDrainNs);
     }
+  } else if (C::kLsuA && warp >= 2 && warp < 2 + C::kAWarps) {
+    // ---------------- cp.async gather of the token rows (gemm1) ----------------
+    // Warp pw owns tile rows [32 pw, 32 pw + 32); per instruction each group of eight
+    // lanes copies one row's 128-byte k-slice (eight 16-byte pieces), and the piece c of
+    // row r lands at r * 128 + ((c ^ (r % 8)) * 16): the 128-byte swizzle TMA would apply.
+    // Each thread's copies arrive on the stage's full barrier by themselves when they
+    // land (cp.async.mbarrier.arrive.noinc), so the warp never waits for its own data.
+    const int pw = warp - 2;
+    const int sub = lane >> 3, c = lane & 7;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      const int e = tile / (p.tiles_m * p.tiles_n);
+      const int rem = tile % (p.tiles_m * p.tiles_n);
+      const int m0 = (rem / p.tiles_n) * kBM;
+      const __nv_bfloat16* src[8];
+      uint32_t dst_off[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = pw * 32 + i * 4 + sub;
+        const int s = m0 + r;
+        const int t = s < p.Ce ? p.idx[(int64_t)e * p.Ce + s] : 0;
+        src[i] = x + (int64_t)t * p.K + c * 8;
+        dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
+      }
+      for (int kb = 0; kb < nk; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, kWaitNs);
+        if (__shfl_sync(0xffffffffu, w, 0) == 0) { ok = false; break; }
+        uint8_t* dst = a_tile(stage, 0);
+        const int k0 = kb * kBK;
+        if (k0 + c * 8 < p.K) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) cp_async16(dst + dst_off[i], src[i] + k0);
+          cp_async_arrive_noinc(&full_bar[stage]);
+        } else {  // beyond d: zeros, as the TMA path's out-of-bounds fill
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<uint4*>(dst + dst_off[i]) = make_uint4(0, 0, 0, 0);
+          fence_proxy_async_smem();
+          mbar_arrive(&full_bar[stage]);
+        }
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    cp_async_wait<0>();  // no copy may still be writing when the CTA exits
   } else if (warp == 1) {
     // ---------------- MMA issuer (one thread) ----------------
     if (lane == 0) {
@@ -197,6 +270,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         for (int kb = 0; kb < nk; ++kb) {
           if (!(ok = mbar_wait(&full_bar[stage], phase, abort_v, kWaitNs))) break;
           tc_fence_after();
+          if (C::kLsuA) fence_proxy_async_smem();  // cp.async writes -> tensor-core reads
           const uint32_t b_addr = smem_u32(b_tile(stage));
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
@@ -219,10 +293,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       int dummy = 0;
       mbar_wait(&drain_bar, 0, &dummy, kDrainNs);
     }
-  } else {
-    // ---------------- epilogue (warps 2..5) ----------------
-    const int q = warp & 3;              // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;       // accumulator row = tile row
+  } else if (warp >= C::kEpiWarp0) {
+    // ---------------- epilogue: eight warps, two per TMEM lane quarter ----------------
+    const int q = warp & 3;                         // TMEM lane quarter this warp may access
+    const int half = (warp - C::kEpiWarp0) >> 2;    // which half of the columns
+    const int row = q * 32 + lane;                  // accumulator row = tile row
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
@@ -242,7 +317,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         __nv_bfloat16* hi = static_cast<__nv_bfloat16*>(p.out) + orow;
         __nv_bfloat16* lo = static_cast<__nv_bfloat16*>(p.out_lo) + orow;
 #pragma unroll 1
-        for (int j0 = 0; j0 < 128; j0 += 32) {
+        for (int j0 = 64 * half; j0 < 64 * half + 64; j0 += 32) {
           uint32_t g[32], u[32];
           tmem_ld32(taddr + j0, g);
           tmem_ld32(taddr + 128 + j0, u);
@@ -276,7 +351,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       } else {
         const float gw = valid ? p.gate[(int64_t)e * p.Ce + s] : 0.f;
 #pragma unroll 1
-        for (int j0 = 0; j0 < 256; j0 += 32) {
+        for (int j0 = 128 * half; j0 < 128 * half + 128; j0 += 32) {
           uint32_t y[32];
           tmem_ld32(taddr + j0, y);
           tmem_ld_wait();
@@ -320,7 +395,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
 
   __syncthreads();
   if (threadIdx.x == 0 && abort_flag) atomicOr(p.err, kErrTimeout);
-  if (warp == 2) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
@@ -371,15 +446,17 @@ bool rows_map(CUtensorMap* m, const void* base, int64_t rows, int cols, uint32_t
   return make_map(m, base, 2, dims, strides, box);
 }
 
-template <int MODE, bool SPLIT>
+template <int MODE, bool SPLIT, int GATHER>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b0,
-                   const CUtensorMap& b1, const Params& p, int sm_count, cudaStream_t st) {
-  auto k = grouped_gemm_kernel<MODE, SPLIT>;
-  const size_t smem = Cfg<MODE, SPLIT>::kSmem;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                   const CUtensorMap& b1, const __nv_bfloat16* x, const Params& p,
+                   int sm_count, cudaStream_t st) {
+  using C = Cfg<MODE, SPLIT, GATHER>;
+  auto k = grouped_gemm_kernel<MODE, SPLIT, GATHER>;
+  cudaError_t e =
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
-  k<<<grid, kThreads, smem, st>>>(a, a2, b0, b1, p);
+  k<<<grid, C::kThreads, C::kSmem, st>>>(a, a2, b0, b1, x, p);
   return cudaGetLastError();
 }
 
@@ -391,8 +468,9 @@ bool experts_sm100_supported(const Shape& s) {
 }
 
 cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1,
-                               const void* W3, const Shape& s, bool split, void* H_hi,
-                               void* H_lo, unsigned* err, int sm_count, cudaStream_t st) {
+                               const void* W3, const Shape& s, bool split, bool tma_gather,
+                               void* H_hi, void* H_lo, unsigned* err, int sm_count,
+                               cudaStream_t st) {
   CUtensorMap ma, mb0, mb1;
   if (!rows_map(&ma, x, s.T, s.d, 1) || !weight_map(&mb0, W1, s.E, s.d, s.F) ||
       !weight_map(&mb1, W3, s.E, s.d, s.F))
@@ -403,8 +481,12 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
   p.tiles_n = (int)ceil_div(s.F, 128);
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
   p.idx = idx; p.gate = nullptr; p.out = H_hi; p.out_lo = H_lo; p.err = err;
-  return split ? launch<kGemm1, true>(ma, ma, mb0, mb1, p, sm_count, st)
-               : launch<kGemm1, false>(ma, ma, mb0, mb1, p, sm_count, st);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (tma_gather)
+    return split ? launch<kGemm1, true, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st)
+                 : launch<kGemm1, false, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st);
+  return split ? launch<kGemm1, true, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st)
+               : launch<kGemm1, false, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st);
 }
 
 cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
@@ -422,8 +504,8 @@ cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* 
   p.tiles_n = (int)ceil_div(s.d, 256);
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
   p.idx = nullptr; p.gate = gate; p.out = Y; p.out_lo = nullptr; p.err = err;
-  return split ? launch<kGemm2, true>(ma, ma2, mb, mb, p, sm_count, st)
-               : launch<kGemm2, false>(ma, ma2, mb, mb, p, sm_count, st);
+  return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st)
+               : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st);
 }
 
 }  // namespace nmoe

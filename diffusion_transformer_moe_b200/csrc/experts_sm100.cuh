@@ -7,12 +7,14 @@ namespace nmoe {
 // True when the tcgen05 kernels cover this shape (bf16 only).
 bool experts_sm100_supported(const Shape& s);
 
-// H[e, s, :] = silu(x[idx[e,s]] W1_e) * (x[idx[e,s]] W3_e), rows gathered by TMA.
+// H[e, s, :] = silu(x[idx[e,s]] W1_e) * (x[idx[e,s]] W3_e), the rows gathered from x by
+// cp.async (default) or by TMA tile::gather4 (tma_gather).
 // split: H is written as bf16 hi = bf16(h) to H_hi and lo = bf16(h - hi) to H_lo;
 // otherwise only H_hi (bf16(h)) is written.
 cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1,
-                               const void* W3, const Shape& s, bool split, void* H_hi,
-                               void* H_lo, unsigned* err, int sm_count, cudaStream_t st);
+                               const void* W3, const Shape& s, bool split, bool tma_gather,
+                               void* H_hi, void* H_lo, unsigned* err, int sm_count,
+                               cudaStream_t st);
 
 // Y[e*Ce + s, :] = gate[e, s] * (H[e, s, :] W2_e). split: H = H_hi + H_lo and Y is fp32;
 // otherwise H = H_hi and Y is bf16.

@@ -114,6 +114,9 @@ typedef struct nmoe_options {
   nmoe_trace* trace;         /* NULL, or a timer to record per-stage events into */
   nmoe_intermediate intermediate;  /* bf16 layers: storage of H and Y (default SPLIT) */
   int out_f32;               /* nonzero: out is fp32 even when dtype is bf16 */
+  int tma_gather;            /* nonzero: the gate/up GEMM fetches its token rows with TMA
+                                tile::gather4 instead of cp.async (about 2x slower on
+                                B200; kept for comparison) */
 } nmoe_options;
 
 /* Fills `o` with the defaults: bf16, softmax, raw combine, route_scale 1, one segment,

@@ -123,7 +123,9 @@ def test_small_shapes_match_oracle(dtype, T, d, E, F, C_):
 
 
 @pytest.mark.parametrize("opts", [dict(out_f32=True), dict(intermediate="bf16"),
-                                  dict(intermediate="bf16", out_f32=True)])
+                                  dict(intermediate="bf16", out_f32=True),
+                                  dict(tma_gather=True),
+                                  dict(tma_gather=True, intermediate="bf16")])
 def test_output_and_intermediate_options_match_oracle(opts):
     a = I.make_small(300, 136, 5, 200, "bf16", seed=77)
     _full_parity(a, 37, "bf16f32" if opts.get("out_f32") else "bf16", opts)
