@@ -11,14 +11,23 @@
 // fp64 running sums in registers. Max, exp and the normalisation run in fp64; each
 // score is rounded once to fp32.
 //
-// One CTA per 128 tokens. Warp 0 streams x tiles and W_r tiles with TMA into a 6-stage
-// ring; warp 1 (one thread) issues tcgen05.mma (M = 128, N = E rounded up to 64, K = 16)
-// into a ring of TMEM chunk buffers; 4*G epilogue warps (G = ceil(E/32)) each own 32
-// tokens x 32 experts. Every wait is bounded.
+// Each 128-token tile is split along d between the two CTAs of a cluster (so T = 8192
+// fills 128 SMs, not 64). In each CTA, warp 0 streams x and W_r tiles with TMA into a
+// 6-stage ring; warp 1 (one thread) issues tcgen05.mma (M = 128, N = E rounded up to
+// 64, K = 16) into a ring of TMEM chunk buffers; 4*G epilogue warps (G = ceil(E/32))
+// each own 32 tokens x 32 experts and keep fp64 sums. The second CTA then adds its sums
+// into the first CTA's shared memory (distributed shared memory, no global traffic),
+// and the first CTA applies the score function and writes both score layouts. exp runs
+// in fp32 on the high part of the fp64 argument, corrected to first order by the low
+// part (relative error ~3e-7); every wait is bounded.
 #include <cudaTypedefs.h>
+
+#include <cooperative_groups.h>
 
 #include "router_sm100.cuh"
 #include "sm100_ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace nmoe {
 namespace {
@@ -31,6 +40,7 @@ constexpr int kStages = 6;
 constexpr int kABytes = kBM * kBK * 2;     // 16 KB
 constexpr int kBBoxBytes = 64 * kBK * 2;   // 8 KB: 64 experts x 64 k
 constexpr int kMaxE = 128;
+constexpr int kSplit = 2;   // CTAs per token tile (one cluster), each owning half of d
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint64_t kDrainNs = 20000000ull;
 
@@ -46,7 +56,18 @@ struct Params {
   unsigned* err;
 };
 
-template <int G>
+// exp(a) for an fp64 argument: fp32 exp of the high part times (1 + low part). The low
+// part is below 2^-24 |a|, so dropping its square leaves ~1e-11; expf adds ~2 ulp.
+// Arguments beyond the fp32 exp range use the fp64 exp.
+__device__ __forceinline__ double exp_f64_arg(double a) {
+  if (a < -80.0 || a > 80.0) return exp(a);
+  const float hi = (float)a;
+  return (double)expf(hi) * (1.0 + (a - (double)hi));
+}
+
+// CW: experts per epilogue thread (16 or 32); G = ceil(E / CW) column groups, so the
+// epilogue has 4 G warps (one per TMEM lane quarter and group).
+template <int G, int CW>
 __global__ void __launch_bounds__(64 + 128 * G, 1)
 router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
                     const __grid_constant__ CUtensorMap map_w, const Params p) {
@@ -62,8 +83,12 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nk = (p.d + kBK - 1) / kBK;
-  const int t0 = blockIdx.x * kBM;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int nk_all = (p.d + kBK - 1) / kBK;
+  const int kb0 = rank == 0 ? 0 : (nk_all + 1) / 2;
+  const int nk = rank == 0 ? (nk_all + 1) / 2 : nk_all - (nk_all + 1) / 2;
+  const int t0 = (blockIdx.x / kSplit) * kBM;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) { mbar_init(&full_bar[i], 1); mbar_init(&empty_bar[i], 1); }
@@ -88,10 +113,11 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       for (int kb = 0; kb < nk; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, kWaitNs)) break;
         mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
-        tma_load_2d(sA + stage * kABytes, &map_x, &full_bar[stage], kb * kBK, t0);
+        const int k0 = (kb0 + kb) * kBK;
+        tma_load_2d(sA + stage * kABytes, &map_x, &full_bar[stage], k0, t0);
         for (int j = 0; j < p.nbox; ++j)
           tma_load_2d(sB + stage * b_bytes + j * kBBoxBytes, &map_w, &full_bar[stage], 64 * j,
-                      kb * kBK);
+                      k0);
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == kStages) { stage = 0; phase ^= 1; }
@@ -133,13 +159,14 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       mbar_wait(&drain_bar, 0, &dummy, kDrainNs);
     }
   } else {
-    // ---------------- epilogue: 32 tokens x 32 experts per warp ----------------
+    // ---------------- epilogue: 32 tokens x CW experts per warp ----------------
     const int q = warp & 3;
     const int g = (warp - 2) >> 2;
     const int row = q * 32 + lane;
-    double acc[32];
+    const int e0 = g * CW;
+    double acc[CW];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) acc[j] = 0.0;
+    for (int j = 0; j < CW; ++j) acc[j] = 0.0;
     int buf = 0;
     uint32_t buf_phase = 0;
     bool ok = true;
@@ -149,72 +176,102 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       if (__shfl_sync(0xffffffffu, w, 0) == 0) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr =
-          tmem_base + ((uint32_t)(q * 32) << 16) + buf * 2 * p.epad + g * 32;
-      // two chunk slices x two halves of this warp's 32 experts, 16 columns at a time
+          tmem_base + ((uint32_t)(q * 32) << 16) + buf * 2 * p.epad + e0;
+      // both 32-long chunk slices of this thread's experts, 16 columns at a time; the
+      // two chunk sums are added in fp32 (one rounding), then into fp64
 #pragma unroll
-      for (int part = 0; part < 4; ++part) {
-        uint32_t c[16];
-        tmem_ld16(taddr + (part >> 1) * p.epad + (part & 1) * 16, c);
+      for (int h = 0; h < CW / 16; ++h) {
+        uint32_t c0[16], c1[16];
+        tmem_ld16(taddr + h * 16, c0);
+        tmem_ld16(taddr + p.epad + h * 16, c1);
         tmem_ld_wait();
-        if (part == 3) {
+        if (h == CW / 16 - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty_bar[buf]);
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[(part & 1) * 16 + j] += (double)__uint_as_float(c[j]);
+        for (int j = 0; j < 16; ++j)
+          acc[h * 16 + j] += (double)(__uint_as_float(c0[j]) + __uint_as_float(c1[j]));
       }
       if (++buf == p.nbuf) { buf = 0; buf_phase ^= 1; }
     }
-    // Every MMA has completed once the last chunk was read, so the stage ring is idle:
-    // keep the fp64 logits there, [128][E + 1], and finish row by row.
-    double* lg = reinterpret_cast<double*>(smem);
-    const int ld = p.E + 1;
-    const int e0 = g * 32;
+    // After the cluster barrier both CTAs' stage rings are idle. The second CTA adds its
+    // half-d sums into the first CTA's ring laid out [E][128] (a warp writes 32
+    // consecutive doubles per expert), then the first CTA finishes in registers.
+    double* part = reinterpret_cast<double*>(smem);
+    double* red = part + (size_t)kMaxE * kBM;   // [2][G][128]: row max, then row sum
+    cluster.sync();                       // (1) every ring is idle
+    if (rank != 0) {
+      double* remote = cluster.map_shared_rank(part, 0);
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (e0 + j < p.E) lg[row * ld + e0 + j] = acc[j];
-    const int nthreads = 128 * G;
-    const int ew = warp - 2;  // epilogue warp 0 .. 4G-1
-    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-    for (int r = ew; r < kBM; r += 4 * G) {
-      double* lr = lg + r * ld;
-      const int t = t0 + r;
-      if (p.bias != nullptr && t < p.T) {
-        const float* b = p.bias + (int64_t)(t / p.S) * p.E;
-        for (int e = lane; e < p.E; e += 32) lr[e] += (double)b[e];
+      for (int j = 0; j < CW; ++j)
+        if (e0 + j < p.E) remote[(e0 + j) * kBM + row] = acc[j];
+    }
+    cluster.sync();                       // (2) the second half's sums have landed
+    if (rank == 0) {
+      const int nthreads = 128 * G;
+      const int t = t0 + row;
+      const bool live = t < p.T;
+      const float* b = (p.bias != nullptr && live) ? p.bias + (int64_t)(t / p.S) * p.E : nullptr;
+#pragma unroll
+      for (int j = 0; j < CW; ++j) {
+        if (e0 + j < p.E) {
+          acc[j] += part[(e0 + j) * kBM + row];
+          if (b) acc[j] += (double)b[e0 + j];
+        }
       }
       if (p.score_fn == NMOE_SCORE_SOFTMAX) {
         double m = -INFINITY;
-        for (int e = lane; e < p.E; e += 32) m = fmax(m, lr[e]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+        for (int j = 0; j < CW; ++j)
+          if (e0 + j < p.E) m = fmax(m, acc[j]);
+        red[g * kBM + row] = m;
+        asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+        m = red[row];
+#pragma unroll
+        for (int h = 1; h < G; ++h) m = fmax(m, red[h * kBM + row]);
         double z = 0.0;
-        for (int e = lane; e < p.E; e += 32) {
-          double v = exp(lr[e] - m);
-          lr[e] = v;
-          z += v;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) {
+          acc[j] = (e0 + j < p.E) ? exp_f64_arg(acc[j] - m) : 0.0;
+          z += acc[j];
+        }
+        red[(G + g) * kBM + row] = z;
+        asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+        z = 0.0;
+#pragma unroll
+        for (int h = 0; h < G; ++h) z += red[(G + h) * kBM + row];
+        const double rz = 1.0 / z;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) acc[j] *= rz;
+      } else {
+#pragma unroll
+        for (int j = 0; j < CW; ++j) acc[j] = 1.0 / (1.0 + exp_f64_arg(-acc[j]));
+      }
+      if (ok && live) {
+        float* srow = p.scores + (int64_t)t * p.E + e0;
+        if ((p.E & 3) == 0 && e0 + CW <= p.E) {
+#pragma unroll
+          for (int j = 0; j < CW; j += 4)
+            *reinterpret_cast<float4*>(srow + j) = make_float4(
+                (float)acc[j], (float)acc[j + 1], (float)acc[j + 2], (float)acc[j + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < CW; ++j)
+            if (e0 + j < p.E) srow[j] = (float)acc[j];
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-        for (int e = lane; e < p.E; e += 32) lr[e] = lr[e] / z;
-      } else {
-        for (int e = lane; e < p.E; e += 32) lr[e] = 1.0 / (1.0 + exp(-lr[e]));
+        for (int j = 0; j < CW; ++j)
+          if (e0 + j < p.E) p.scores_t[(int64_t)(e0 + j) * p.T + t] = (float)acc[j];
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-    if (ok) {
-      const int tid = threadIdx.x - 64;
-      const int rows = min(kBM, p.T - t0);
-      for (int i = tid; i < rows * p.E; i += nthreads) {
-        const int r = i / p.E, e = i - r * p.E;
-        p.scores[(int64_t)(t0 + r) * p.E + e] = (float)lg[r * ld + e];
-      }
-      for (int i = tid; i < kBM * p.E; i += nthreads) {
-        const int e = i / kBM, r = i - e * kBM;
-        if (r < rows) p.scores_t[(int64_t)e * p.T + t0 + r] = (float)lg[r * ld + e];
-      }
-    }
+  }
+  if (warp < 2) {
+    // the producer and MMA warps take part in the two cluster barriers as well
+    __syncwarp();
+    cluster.sync();
+    cluster.sync();
   }
 
   __syncthreads();
@@ -276,16 +333,32 @@ cudaError_t launch_router_sm100(const void* x, const void* W_r, const Shape& s,
     // a shape the tensor maps cannot describe: the CUDA-core router computes the same
     return launch_router_simt(x, W_r, s, NMOE_BF16, fn, bias, scores, scores_t, st);
   size_t smem = (size_t)kStages * (kABytes + p.nbox * kBBoxBytes);
-  const size_t logits = sizeof(double) * kBM * (size_t)(s.E + 1);
-  smem = (smem > logits ? smem : logits) + 1024;
-  const int G = (int)ceil_div(s.E, 32);
-  auto k = G == 1 ? router_sm100_kernel<1>
-         : G == 2 ? router_sm100_kernel<2>
-         : G == 3 ? router_sm100_kernel<3>
-                  : router_sm100_kernel<4>;
+  const size_t red = sizeof(double) * kBM * (size_t)(kMaxE + 2 * 4);
+  smem = (smem > red ? smem : red) + 1024;
+  // 16 experts per thread up to E = 64 (up to 16 epilogue warps), 32 beyond
+  const int CW = s.E <= 64 ? 16 : 32;
+  const int G = (int)ceil_div(s.E, CW);
+  auto k = CW == 16 ? (G == 1 ? router_sm100_kernel<1, 16>
+                     : G == 2 ? router_sm100_kernel<2, 16>
+                     : G == 3 ? router_sm100_kernel<3, 16>
+                              : router_sm100_kernel<4, 16>)
+                    : (G == 3 ? router_sm100_kernel<3, 32> : router_sm100_kernel<4, 32>);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<(unsigned)ceil_div(s.T, kBM), 64 + 128 * G, smem, st>>>(mx, mw, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(ceil_div(s.T, kBM) * kSplit));
+  cfg.blockDim = dim3(64 + 128 * G);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k, mx, mw, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
