@@ -97,6 +97,7 @@ Shape make_shape(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C, int64_t 
   Shape s;
   s.T = (int)T; s.d = (int)d; s.E = (int)E; s.F = (int)F; s.C = (int)C;
   s.n_seg = (int)n_seg; s.S = (int)(T / n_seg); s.Ce = (int)(n_seg * C);
+  s.pdl = true;
   return s;
 }
 
@@ -110,7 +111,7 @@ size_t out_size(nmoe_dtype dt, const nmoe_options& o) {
 }
 
 struct Layout {
-  size_t scores, scores_t, idx, gate, tok_ptr, tok_ent, H, Y, xin, xout, total;
+  size_t scores, scores_t, idx, gate, tok_ptr, tok_ent, ent_pos, H, Y, xin, xout, total;
 };
 
 Layout make_layout(const Shape& s, nmoe_dtype dt, const nmoe_options& o) {
@@ -125,6 +126,7 @@ Layout make_layout(const Shape& s, nmoe_dtype dt, const nmoe_options& o) {
   L.gate = take(sizeof(float) * (size_t)s.E * s.Ce);
   L.tok_ptr = take(sizeof(int32_t) * ((size_t)s.T + 1));
   L.tok_ent = take(sizeof(int32_t) * (size_t)s.E * s.Ce);
+  L.ent_pos = take(sizeof(int32_t) * (size_t)s.E * s.Ce);
   L.H = take(is * (size_t)s.E * s.Ce * s.F);
   L.Y = take(is * (size_t)s.E * s.Ce * s.d);
   L.xin = o.host_io ? take(esize(dt) * (size_t)s.T * s.d) : none;
@@ -179,8 +181,10 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
 
   DevState* ds = nullptr;
   if ((v = dev_state(&ds)) != NMOE_OK) return v;
-  const Shape s = make_shape(T, d, E, F, C, o.n_segments);
+  Shape s = make_shape(T, d, E, F, C, o.n_segments);
   if (s.Ce > 65535 * 64) return NMOE_ERR_UNSUPPORTED;
+  // per-stage events sit between the launches, so traced calls run without overlap
+  s.pdl = o.trace == nullptr;
   const Layout L = make_layout(s, o.dtype, o);
 
   char* ws = static_cast<char*>(o.workspace);
@@ -201,6 +205,7 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   float* gate = reinterpret_cast<float*>(ws + L.gate);
   int32_t* tok_ptr = reinterpret_cast<int32_t*>(ws + L.tok_ptr);
   int32_t* tok_ent = reinterpret_cast<int32_t*>(ws + L.tok_ent);
+  int32_t* ent_pos = reinterpret_cast<int32_t*>(ws + L.ent_pos);
   void* H = ws + L.H;
   void* Y = ws + L.Y;
   const size_t xbytes = esize(o.dtype) * (size_t)s.T * s.d;
@@ -235,7 +240,8 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   if (e == cudaSuccess) e = nmoe::launch_select(scores_t, s, idx, gate, ds->err, st);
   mark(2);
   if (e == cudaSuccess)
-    e = nmoe::launch_csr(idx, s, tok_ptr, tok_ent, gate, o.combine, o.route_scale, ds->err, st);
+    e = nmoe::launch_csr(idx, s, tok_ptr, tok_ent, ent_pos, gate, o.combine, o.route_scale,
+                         ds->err, st);
   mark(3);
   const bool tc = !f32 && nmoe::experts_sm100_supported(s);
   // SPLIT on the tensor cores: H_hi then H_lo, each [E*Ce, F] bf16; on the CUDA cores
@@ -247,11 +253,12 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
            : nmoe::launch_gemm1_simt(xd, idx, W1, W3, s, o.dtype, split, H, st);
   mark(4);
   if (e == cudaSuccess)
-    e = tc ? nmoe::launch_gemm2_sm100(H, H_lo, gate, W2, s, split, Y, ds->err, ds->sm_count, st)
-           : nmoe::launch_gemm2_simt(H, gate, W2, s, o.dtype, split, y_f32, Y, st);
+    e = tc ? nmoe::launch_gemm2_sm100(H, H_lo, gate, ent_pos, W2, s, split, Y, ds->err,
+                                      ds->sm_count, st)
+           : nmoe::launch_gemm2_simt(H, gate, W2, ent_pos, s, o.dtype, split, y_f32, Y, st);
   mark(5);
   if (e == cudaSuccess)
-    e = nmoe::launch_combine(Y, tok_ptr, tok_ent, s, y_f32, out_f32, outd, ds->sm_count, st);
+    e = nmoe::launch_combine(Y, tok_ptr, s, y_f32, out_f32, outd, ds->err, ds->sm_count, st);
   mark(6);
   if (o.host_io && e == cudaSuccess)
     e = cudaMemcpyAsync(out, outd, obytes, cudaMemcpyDeviceToHost, st);
@@ -333,7 +340,8 @@ nmoe_status nmoe_select(const float* scores_t, int64_t T, int64_t E, int64_t C,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = nmoe::launch_select(scores_t, s, idx, gate, ds->err, st);
   if (e == cudaSuccess && tok_ptr)
-    e = nmoe::launch_csr(idx, s, tok_ptr, tok_ent, gate, NMOE_COMBINE_RAW, 1.f, ds->err, st);
+    e = nmoe::launch_csr(idx, s, tok_ptr, tok_ent, nullptr, gate, NMOE_COMBINE_RAW, 1.f, ds->err,
+                         st);
   if (e != cudaSuccess) { cudaGetLastError(); return NMOE_ERR_CUDA; }
   return NMOE_OK;
 }

@@ -2,120 +2,147 @@
 //
 // NucleusMoE-Image walkthrough, section 6.2: the weighted outputs of the routed experts
 // are added back onto their tokens (the page uses scatter_add, whose order of additions
-// is not fixed). Here every token gathers its own contributions instead:
-//   out[t, :] = sum over j in [tok_ptr[t], tok_ptr[t+1]) of Y[tok_ent[j], :]
-// in ascending expert order (the order tok_ent lists them), accumulated in fp32 and
-// rounded once to the output type. The combine weight was applied to Y by the down-
-// projection epilogue. A token no expert chose gets an exact zero row.
+// is not fixed). Here the down projection has already written every weighted expert
+// output at its token-major position, so the combine is a segmented sum of contiguous
+// rows:
+//   out[t, :] = sum over r in [tok_ptr[t], tok_ptr[t+1]) of Y[r, :]
+// in ascending expert order (the order of the token lists), accumulated in fp32 and
+// rounded once to the output type. A token no expert chose gets an exact zero row.
 //
-// One warp per token; each lane moves 16-byte vectors and keeps several rows in flight.
+// Each CTA owns a contiguous token range, whose rows of Y form one contiguous span.
+// Every thread owns one 16-byte column group and walks the span row by row with eight
+// independent loads in flight, adding into the current token's sum and storing it when
+// the row index crosses the token's end: the memory access pattern of a plain copy, with
+// no synchronisation between warps.
 #include "nmoe_internal.cuh"
 
 namespace nmoe {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kVecPerLane = 4;   // 16-byte vectors a lane accumulates at once
+constexpr int kAhead = 8;                 // rows loaded per round
+constexpr int kMaxTokPerCta = 4096;
 
-__device__ __forceinline__ void unpack_add(float* acc, const uint4& v, __nv_bfloat16*) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+template <typename T> struct Vec;        // 16 bytes of T, unpacked to fp32
+template <> struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void add(float* a, const uint4& v) {
+    a[0] += __uint_as_float(v.x); a[1] += __uint_as_float(v.y);
+    a[2] += __uint_as_float(v.z); a[3] += __uint_as_float(v.w);
+  }
+};
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void add(float* a, const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __bfloat1622float2(h[i]);
-    acc[2 * i] += f.x;
-    acc[2 * i + 1] += f.y;
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      a[2 * i] += f.x;
+      a[2 * i + 1] += f.y;
+    }
+  }
+};
+
+template <int N>
+__device__ __forceinline__ void store_out(float* dst, const float* a) {
+#pragma unroll
+  for (int i = 0; i < N; i += 4)
+    *reinterpret_cast<float4*>(dst + i) = make_float4(a[i], a[i + 1], a[i + 2], a[i + 3]);
+}
+template <int N>
+__device__ __forceinline__ void store_out(__nv_bfloat16* dst, const float* a) {
+#pragma unroll
+  for (int i = 0; i < N; i += 4) {
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(a[i], a[i + 1]);
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(a[i + 2], a[i + 3]);
+    uint2 v;
+    v.x = *reinterpret_cast<uint32_t*>(&h0);
+    v.y = *reinterpret_cast<uint32_t*>(&h1);
+    *reinterpret_cast<uint2*>(dst + i) = v;
   }
 }
-__device__ __forceinline__ void unpack_add(float* acc, const uint4& v, float*) {
-  acc[0] += __uint_as_float(v.x);
-  acc[1] += __uint_as_float(v.y);
-  acc[2] += __uint_as_float(v.z);
-  acc[3] += __uint_as_float(v.w);
-}
-__device__ __forceinline__ uint4 pack(const float* acc, __nv_bfloat16*) {
-  uint4 v;
-  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-  return v;
-}
-__device__ __forceinline__ uint4 pack(const float* acc, float*) {
-  return make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
-                    __float_as_uint(acc[3]));
-}
 
-// Each lane owns 8 consecutive columns per vector slot: one 16-byte load of bf16 Y or
-// two of fp32 Y, and one 16-byte store of bf16 out or two of fp32 out.
 template <typename TY, typename TO>
-__global__ void __launch_bounds__(kThreads)
-combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr,
-               const int32_t* __restrict__ tok_ent, int Tn, int d, TO* __restrict__ out) {
-  constexpr int W = 8;  // columns per lane per vector slot
-  const int lane = threadIdx.x & 31;
-  const int ngrp = d / W;  // d is a multiple of 8 (checked on the host)
-  for (int t = blockIdx.x * kWarps + (threadIdx.x >> 5); t < Tn; t += gridDim.x * kWarps) {
-    const int beg = tok_ptr[t], end = tok_ptr[t + 1];
-    for (int c0 = 0; c0 < ngrp; c0 += 32 * kVecPerLane) {
-      float acc[kVecPerLane][W];
+__global__ void __launch_bounds__(512)
+combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, int Tn, int d,
+               int tok_per_cta, TO* __restrict__ out) {
+  constexpr int N = Vec<TY>::N;          // columns per 16-byte group
+  pdl_launch_dependents();
+  __shared__ int s_ptr[kMaxTokPerCta + 1];
+  const int t0 = min(Tn, (int)blockIdx.x * tok_per_cta), t1 = min(Tn, t0 + tok_per_cta);
+  pdl_wait();
+  for (int i = threadIdx.x; i <= t1 - t0; i += blockDim.x) s_ptr[i] = tok_ptr[t0 + i];
+  __syncthreads();
+  if (t0 >= t1) return;
+  const int r0 = s_ptr[0], r1 = s_ptr[t1 - t0];
+  const int ngroups = d / N;
+  const int64_t stride = d / N;          // 16-byte groups per row
+  for (int grp = threadIdx.x; grp < ngroups; grp += blockDim.x) {
+    const int col = grp * N;
+    const uint4* src = reinterpret_cast<const uint4*>(Y) + grp;
+    float acc[N];
 #pragma unroll
-      for (int v = 0; v < kVecPerLane; ++v)
+    for (int i = 0; i < N; ++i) acc[i] = 0.f;
+    int t = t0;                           // token whose sum is being built
+    int tend = s_ptr[1];                  // its rows end here
+    for (int r = r0; r < r1; r += kAhead) {
+      uint4 v[kAhead];
 #pragma unroll
-        for (int i = 0; i < W; ++i) acc[v][i] = 0.f;
-      for (int j = beg; j < end; ++j) {
-        const TY* src = Y + (int64_t)tok_ent[j] * d;
-        uint4 r[kVecPerLane][sizeof(TY) / 2];
+      for (int k = 0; k < kAhead; ++k)
+        v[k] = r + k < r1 ? __ldg(src + (int64_t)(r + k) * stride) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int v = 0; v < kVecPerLane; ++v) {
-          const int c = c0 + v * 32 + lane;
+      for (int k = 0; k < kAhead; ++k) {
+        if (r + k < r1) {
+          while (r + k >= tend) {         // token t is complete (or had no rows)
+            store_out<N>(out + (int64_t)t * d + col, acc);
 #pragma unroll
-          for (int h = 0; h < (int)sizeof(TY) / 2; ++h)
-            r[v][h] = c < ngrp ? __ldg(reinterpret_cast<const uint4*>(src + (int64_t)c * W) + h)
-                               : make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < N; ++i) acc[i] = 0.f;
+            ++t;
+            tend = s_ptr[t - t0 + 1];
+          }
+          Vec<TY>::add(acc, v[k]);
         }
-#pragma unroll
-        for (int v = 0; v < kVecPerLane; ++v)
-#pragma unroll
-          for (int h = 0; h < (int)sizeof(TY) / 2; ++h)
-            unpack_add(acc[v] + h * (16 / sizeof(TY)), r[v][h], (TY*)nullptr);
       }
+    }
+    for (; t < t1; ++t) {                  // the last token and any empty ones after it
+      store_out<N>(out + (int64_t)t * d + col, acc);
 #pragma unroll
-      for (int v = 0; v < kVecPerLane; ++v) {
-        const int c = c0 + v * 32 + lane;
-        if (c < ngrp) {
-          uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)t * d + (int64_t)c * W);
-#pragma unroll
-          for (int h = 0; h < (int)sizeof(TO) / 2; ++h)
-            dst[h] = pack(acc[v] + h * (16 / sizeof(TO)), (TO*)nullptr);
-        }
-      }
+      for (int i = 0; i < N; ++i) acc[i] = 0.f;
     }
   }
 }
 
+template <typename TY, typename TO>
+cudaError_t launch_typed(const void* Y, const int32_t* tok_ptr, const Shape& s, void* out,
+                         int sm_count, cudaStream_t st) {
+  constexpr int N = Vec<TY>::N;
+  const int ngroups = s.d / N;
+  int threads = ((ngroups + 31) / 32) * 32;
+  if (threads > 512) threads = 512;
+  // two CTAs per SM, each a contiguous token range
+  int grid = 2 * sm_count;
+  if (grid > s.T) grid = s.T;
+  int per = (int)ceil_div(s.T, grid);
+  if (per > kMaxTokPerCta) {
+    per = kMaxTokPerCta;
+    grid = (int)ceil_div(s.T, per);
+  }
+  return launch_kernel(combine_kernel<TY, TO>, dim3(grid), dim3(threads), 0, st, s.pdl, 1,
+                       (const TY*)Y, tok_ptr, s.T, s.d, per, (TO*)out);
+}
+
 }  // namespace
 
-cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const int32_t* tok_ent,
-                           const Shape& s, bool y_f32, bool out_f32, void* out, int sm_count,
+cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const Shape& s, bool y_f32,
+                           bool out_f32, void* out, unsigned* err, int sm_count,
                            cudaStream_t st) {
+  (void)err;
   using bf = __nv_bfloat16;
-  int64_t blocks = ceil_div(s.T, kWarps);
-  int64_t cap = (int64_t)sm_count * 8;
-  dim3 grid((unsigned)(blocks < cap ? blocks : cap));
   if (s.d % 8 != 0) return cudaErrorInvalidValue;
-  if (y_f32 && out_f32)
-    combine_kernel<float, float><<<grid, kThreads, 0, st>>>((const float*)Y, tok_ptr, tok_ent,
-                                                            s.T, s.d, (float*)out);
-  else if (y_f32)
-    combine_kernel<float, bf><<<grid, kThreads, 0, st>>>((const float*)Y, tok_ptr, tok_ent, s.T,
-                                                         s.d, (bf*)out);
-  else if (out_f32)
-    combine_kernel<bf, float><<<grid, kThreads, 0, st>>>((const bf*)Y, tok_ptr, tok_ent, s.T,
-                                                         s.d, (float*)out);
-  else
-    combine_kernel<bf, bf><<<grid, kThreads, 0, st>>>((const bf*)Y, tok_ptr, tok_ent, s.T, s.d,
-                                                      (bf*)out);
-  return cudaGetLastError();
+  if (y_f32 && out_f32) return launch_typed<float, float>(Y, tok_ptr, s, out, sm_count, st);
+  if (y_f32) return launch_typed<float, bf>(Y, tok_ptr, s, out, sm_count, st);
+  if (out_f32) return launch_typed<bf, float>(Y, tok_ptr, s, out, sm_count, st);
+  return launch_typed<bf, bf>(Y, tok_ptr, s, out, sm_count, st);
 }
 
 }  // namespace nmoe

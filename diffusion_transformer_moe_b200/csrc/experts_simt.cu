@@ -3,7 +3,7 @@
 // The exact-fp32 path of the packed SwiGLU experts (NucleusMoE-Image walkthrough,
 // section 6: fused gate/up projection, then the down projection, "two grouped matmuls"):
 //   gemm1: H[e, s, :] = silu(x[idx[e,s]] W1_e) * (x[idx[e,s]] W3_e)
-//   gemm2: Y[e*Ce + s, :] = gate[e, s] * (H[e, s, :] W2_e)
+//   gemm2: Y[ent_pos[e*Ce + s], :] = gate[e, s] * (H[e, s, :] W2_e)
 // The rows of expert e are gathered straight from x through idx; there is no permuted
 // copy of the tokens. Used for fp32 inputs; bf16 inputs take the tcgen05 kernels.
 #include "nmoe_internal.cuh"
@@ -24,6 +24,8 @@ gemm1_simt_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
   __shared__ float Bg[kBK][kBN + 4];
   __shared__ float Bu[kBK][kBN + 4];
   __shared__ int rows[kBM];
+  pdl_launch_dependents();
+  pdl_wait();
   const int e = blockIdx.z, m0 = blockIdx.y * kBM, n0 = blockIdx.x * kBN;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   if (tid < kBM) rows[tid] = (m0 + tid < Ce) ? idx[(int64_t)e * Ce + m0 + tid] : -1;
@@ -79,9 +81,12 @@ gemm1_simt_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
 template <typename T, typename TH, typename TY>
 __global__ void __launch_bounds__(kThreads)
 gemm2_simt_kernel(const TH* __restrict__ H, const float* __restrict__ gate,
-                  const T* __restrict__ W2, int d, int F, int Ce, TY* __restrict__ Y) {
+                  const T* __restrict__ W2, const int32_t* __restrict__ ent_pos, int d, int F,
+                  int Ce, TY* __restrict__ Y) {
   __shared__ float As[kBK][kBM + 4];
   __shared__ float Bs[kBK][kBN + 4];
+  pdl_launch_dependents();
+  pdl_wait();
   const int e = blockIdx.z, m0 = blockIdx.y * kBM, n0 = blockIdx.x * kBN;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const TH* h = H + (int64_t)e * Ce * F;
@@ -120,10 +125,11 @@ gemm2_simt_kernel(const TH* __restrict__ H, const float* __restrict__ gate,
     int s = m0 + ty * 4 + i;
     if (s >= Ce) continue;
     float w = gate[(int64_t)e * Ce + s];
+    const int64_t yrow = ent_pos[(int64_t)e * Ce + s];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       int n = n0 + tx * 4 + j;
-      if (n < d) Y[((int64_t)e * Ce + s) * d + n] = from_f32<TY>(w * acc[i][j]);
+      if (n < d) Y[yrow * d + n] = from_f32<TY>(w * acc[i][j]);
     }
   }
 }
@@ -136,33 +142,31 @@ cudaError_t launch_gemm1_simt(const void* x, const int32_t* idx, const void* W1,
   using bf = __nv_bfloat16;
   dim3 grid((unsigned)ceil_div(s.F, kBN), (unsigned)ceil_div(s.Ce, kBM), (unsigned)s.E);
   if (dt == NMOE_F32)
-    gemm1_simt_kernel<float, float><<<grid, kThreads, 0, st>>>(
+    return launch_kernel(gemm1_simt_kernel<float, float>, grid, dim3(kThreads), 0, st, s.pdl, 1, 
         (const float*)x, idx, (const float*)W1, (const float*)W3, s.d, s.F, s.Ce, (float*)H);
   else if (h_f32)
-    gemm1_simt_kernel<bf, float><<<grid, kThreads, 0, st>>>(
+    return launch_kernel(gemm1_simt_kernel<bf, float>, grid, dim3(kThreads), 0, st, s.pdl, 1, 
         (const bf*)x, idx, (const bf*)W1, (const bf*)W3, s.d, s.F, s.Ce, (float*)H);
   else
-    gemm1_simt_kernel<bf, bf><<<grid, kThreads, 0, st>>>(
+    return launch_kernel(gemm1_simt_kernel<bf, bf>, grid, dim3(kThreads), 0, st, s.pdl, 1, 
         (const bf*)x, idx, (const bf*)W1, (const bf*)W3, s.d, s.F, s.Ce, (bf*)H);
-  return cudaGetLastError();
 }
 
-cudaError_t launch_gemm2_simt(const void* H, const float* gate, const void* W2, const Shape& s,
-                              nmoe_dtype dt, bool h_f32, bool y_f32, void* Y, cudaStream_t st) {
+cudaError_t launch_gemm2_simt(const void* H, const float* gate, const void* W2,
+                              const int32_t* ent_pos, const Shape& s, nmoe_dtype dt, bool h_f32,
+                              bool y_f32, void* Y, cudaStream_t st) {
   using bf = __nv_bfloat16;
   dim3 grid((unsigned)ceil_div(s.d, kBN), (unsigned)ceil_div(s.Ce, kBM), (unsigned)s.E);
   if (dt == NMOE_F32)
-    gemm2_simt_kernel<float, float, float><<<grid, kThreads, 0, st>>>(
-        (const float*)H, gate, (const float*)W2, s.d, s.F, s.Ce, (float*)Y);
+    return launch_kernel(gemm2_simt_kernel<float, float, float>, grid, dim3(kThreads), 0, st, s.pdl, 1, 
+        (const float*)H, gate, (const float*)W2, ent_pos, s.d, s.F, s.Ce, (float*)Y);
   else if (h_f32 && y_f32)
-    gemm2_simt_kernel<bf, float, float><<<grid, kThreads, 0, st>>>(
-        (const float*)H, gate, (const bf*)W2, s.d, s.F, s.Ce, (float*)Y);
+    return launch_kernel(gemm2_simt_kernel<bf, float, float>, grid, dim3(kThreads), 0, st, s.pdl, 1, 
+        (const float*)H, gate, (const bf*)W2, ent_pos, s.d, s.F, s.Ce, (float*)Y);
   else if (!h_f32 && !y_f32)
-    gemm2_simt_kernel<bf, bf, bf><<<grid, kThreads, 0, st>>>(
-        (const bf*)H, gate, (const bf*)W2, s.d, s.F, s.Ce, (bf*)Y);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+    return launch_kernel(gemm2_simt_kernel<bf, bf, bf>, grid, dim3(kThreads), 0, st, s.pdl, 1, 
+        (const bf*)H, gate, (const bf*)W2, ent_pos, s.d, s.F, s.Ce, (bf*)Y);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace nmoe

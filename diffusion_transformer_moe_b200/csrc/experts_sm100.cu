@@ -7,7 +7,10 @@
 // Ce = n_segments * C rows, so both GEMMs have static shapes:
 //
 //   gemm1: H[e, s, :] = silu(x[idx[e,s]] W1_e) * (x[idx[e,s]] W3_e)
-//   gemm2: Y[e*Ce + s, :] = gate[e, s] * (H[e, s, :] W2_e)
+//   gemm2: Y[ent_pos[e*Ce + s], :] = gate[e, s] * (H[e, s, :] W2_e)
+//
+// (Y rows land in token-major order, so the combine reads each token's rows
+// contiguously.)
 //
 // Instead of permuting tokens into per-expert blocks, gemm1 gathers the 128 rows of its
 // A tile straight from x. Two ways are built: four producer warps issuing 16-byte
@@ -77,6 +80,7 @@ struct Params {
   int tiles_m, tiles_n, num_tiles;
   const int32_t* idx;    // gemm1: chosen tokens [E, Ce]
   const float* gate;     // gemm2: combine weights [E, Ce]
+  const int32_t* ent_pos;  // gemm2: Y row of entry e*Ce + s (token-major order)
   void* out;             // gemm1: H (hi) [E*Ce, F] bf16; gemm2: Y [E*Ce, d] (fp32 if SPLIT)
   void* out_lo;          // gemm1 with SPLIT: H lo [E*Ce, F] bf16
   unsigned* err;
@@ -109,6 +113,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                     const Params p) {
   using C = Cfg<MODE, SPLIT, GATHER>;
   constexpr int kStages = C::kStages;
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -146,6 +151,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
   volatile int* abort_v = &abort_flag;
+  pdl_wait();  // the previous kernel's outputs (idx, x or H, gate) are complete
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -209,6 +215,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         if (issued_mask & (1u << s))
           mbar_wait(&full_bar[s], (issued_par >> s) & 1u, &dummy, kDrainNs);
     }
+    __syncwarp();
   } else if (C::kLsuA && warp >= 2 && warp < 2 + C::kAWarps) {
     // ---------------- cp.async gather of the token rows (gemm1) ----------------
     // Warp pw owns tile rows [32 pw, 32 pw + 32); per instruction each group of eight
@@ -293,6 +300,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       int dummy = 0;
       mbar_wait(&drain_bar, 0, &dummy, kDrainNs);
     }
+    __syncwarp();  // the warp reconverges before the block barrier and the TMEM release
   } else if (warp >= C::kEpiWarp0) {
     // ---------------- epilogue: eight warps, two per TMEM lane quarter ----------------
     const int q = warp & 3;                         // TMEM lane quarter this warp may access
@@ -312,7 +320,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * kAccCols;
       const int s = m0 + row;
       const bool valid = s < p.Ce;
-      const int64_t orow = ((int64_t)e * p.Ce + (valid ? s : 0)) * p.N;
+      const int64_t ent = (int64_t)e * p.Ce + (valid ? s : 0);
+      const int64_t orow = (MODE == kGemm2 ? (int64_t)p.ent_pos[ent] : ent) * p.N;
       if (MODE == kGemm1) {
         __nv_bfloat16* hi = static_cast<__nv_bfloat16*>(p.out) + orow;
         __nv_bfloat16* lo = static_cast<__nv_bfloat16*>(p.out_lo) + orow;
@@ -449,15 +458,11 @@ bool rows_map(CUtensorMap* m, const void* base, int64_t rows, int cols, uint32_t
 template <int MODE, bool SPLIT, int GATHER>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b0,
                    const CUtensorMap& b1, const __nv_bfloat16* x, const Params& p,
-                   int sm_count, cudaStream_t st) {
+                   int sm_count, cudaStream_t st, bool pdl) {
   using C = Cfg<MODE, SPLIT, GATHER>;
-  auto k = grouped_gemm_kernel<MODE, SPLIT, GATHER>;
-  cudaError_t e =
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
-  if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
-  k<<<grid, C::kThreads, C::kSmem, st>>>(a, a2, b0, b1, x, p);
-  return cudaGetLastError();
+  return launch_kernel(grouped_gemm_kernel<MODE, SPLIT, GATHER>, dim3(grid), dim3(C::kThreads),
+                       C::kSmem, st, pdl, 1, a, a2, b0, b1, x, p);
 }
 
 }  // namespace
@@ -480,18 +485,19 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
   p.tiles_m = (int)ceil_div(s.Ce, kBM);
   p.tiles_n = (int)ceil_div(s.F, 128);
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
-  p.idx = idx; p.gate = nullptr; p.out = H_hi; p.out_lo = H_lo; p.err = err;
+  p.idx = idx; p.gate = nullptr; p.ent_pos = nullptr; p.out = H_hi; p.out_lo = H_lo;
+  p.err = err;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (tma_gather)
-    return split ? launch<kGemm1, true, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st)
-                 : launch<kGemm1, false, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st);
-  return split ? launch<kGemm1, true, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st)
-               : launch<kGemm1, false, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st);
+    return split ? launch<kGemm1, true, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl)
+                 : launch<kGemm1, false, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl);
+  return split ? launch<kGemm1, true, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl)
+               : launch<kGemm1, false, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl);
 }
 
 cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
-                               const void* W2, const Shape& s, bool split, void* Y, unsigned* err,
-                               int sm_count, cudaStream_t st) {
+                               const int32_t* ent_pos, const void* W2, const Shape& s, bool split,
+                               void* Y, unsigned* err, int sm_count, cudaStream_t st) {
   CUtensorMap ma, ma2, mb;
   const int64_t rows = (int64_t)s.E * s.Ce;
   if (!rows_map(&ma, H_hi, rows, s.F, kBM) || !weight_map(&mb, W2, s.E, s.F, s.d))
@@ -503,9 +509,10 @@ cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* 
   p.tiles_m = (int)ceil_div(s.Ce, kBM);
   p.tiles_n = (int)ceil_div(s.d, 256);
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
-  p.idx = nullptr; p.gate = gate; p.out = Y; p.out_lo = nullptr; p.err = err;
-  return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st)
-               : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st);
+  p.idx = nullptr; p.gate = gate; p.ent_pos = ent_pos; p.out = Y; p.out_lo = nullptr;
+  p.err = err;
+  return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl)
+               : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl);
 }
 
 }  // namespace nmoe

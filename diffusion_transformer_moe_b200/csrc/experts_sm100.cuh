@@ -16,10 +16,11 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
                                void* H_hi, void* H_lo, unsigned* err, int sm_count,
                                cudaStream_t st);
 
-// Y[e*Ce + s, :] = gate[e, s] * (H[e, s, :] W2_e). split: H = H_hi + H_lo and Y is fp32;
-// otherwise H = H_hi and Y is bf16.
+// Y[ent_pos[e*Ce + s], :] = gate[e, s] * (H[e, s, :] W2_e). split: H = H_hi + H_lo and
+// Y is fp32; otherwise H = H_hi and Y is bf16.
 cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
-                               const void* W2, const Shape& s, bool split, void* Y,
-                               unsigned* err, int sm_count, cudaStream_t st);
+                               const int32_t* ent_pos, const void* W2, const Shape& s,
+                               bool split, void* Y, unsigned* err, int sm_count,
+                               cudaStream_t st);
 
 }  // namespace nmoe

@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "nmoe.h"
 
 namespace nmoe {
@@ -23,6 +25,52 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
   return __float2bfloat16_rn(v);
 }
 
+// Programmatic dependent launch. Every kernel of the layer lets the next kernel on the
+// stream start its prologue early (launch_dependents, issued by every thread at entry)
+// and waits for the previous grid's memory (wait) before its first global access.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Raises a kernel's dynamic shared-memory limit on the current device, once per
+// (kernel, device).
+cudaError_t set_smem_limit(const void* kernel, size_t bytes);
+
+// Launch with programmatic stream serialization (pdl) and an optional 1-D cluster.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, bool pdl, unsigned cluster_x, Args&&... args) {
+  if (smem > 48 * 1024) {
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(kernel), smem);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 // Shapes of one layer call, already validated on the host.
 struct Shape {
   int T;         // tokens
@@ -33,6 +81,7 @@ struct Shape {
   int n_seg;     // segments
   int S;         // tokens per segment = T / n_seg
   int Ce;        // entries per expert = n_seg * C
+  bool pdl;      // launch with programmatic dependent launch
 };
 
 // Launchers. Each returns the launch status (cudaGetLastError after the launch).
@@ -44,10 +93,11 @@ cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, f
                           unsigned* err, cudaStream_t st);
 
 // combine == NMOE_COMBINE_NORMALIZED rewrites gate[] in place to
-// route_scale * gate / (sum of the token's gates).
+// route_scale * gate / (sum of the token's gates). ent_pos (may be NULL) receives, for
+// each entry e*Ce + slot, its index in the token-major order of tok_ent.
 cudaError_t launch_csr(const int32_t* idx, const Shape& s, int32_t* tok_ptr, int32_t* tok_ent,
-                       float* gate, nmoe_combine combine, float route_scale, unsigned* err,
-                       cudaStream_t st);
+                       int32_t* ent_pos, float* gate, nmoe_combine combine, float route_scale,
+                       unsigned* err, cudaStream_t st);
 
 // CUDA-core expert GEMMs. dt is the type of x and the weights; h_f32 / y_f32 select
 // fp32 (else dt) for the H and Y intermediates.
@@ -55,12 +105,15 @@ cudaError_t launch_gemm1_simt(const void* x, const int32_t* idx, const void* W1,
                               const Shape& s, nmoe_dtype dt, bool h_f32, void* H,
                               cudaStream_t st);
 
-cudaError_t launch_gemm2_simt(const void* H, const float* gate, const void* W2, const Shape& s,
-                              nmoe_dtype dt, bool h_f32, bool y_f32, void* Y, cudaStream_t st);
+// Row e*Ce + s of the product goes to Y row ent_pos[e*Ce + s] (token-major order).
+cudaError_t launch_gemm2_simt(const void* H, const float* gate, const void* W2,
+                              const int32_t* ent_pos, const Shape& s, nmoe_dtype dt, bool h_f32,
+                              bool y_f32, void* Y, cudaStream_t st);
 
-// out[t] = sum of Y rows listed for t; Y is fp32 if y_f32 (else bf16), out fp32 if out_f32.
-cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const int32_t* tok_ent,
-                           const Shape& s, bool y_f32, bool out_f32, void* out, int sm_count,
+// out[t] = sum of Y rows tok_ptr[t] .. tok_ptr[t+1]-1 (token-major Y, ascending expert);
+// Y is fp32 if y_f32 (else bf16), out fp32 if out_f32.
+cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const Shape& s, bool y_f32,
+                           bool out_f32, void* out, unsigned* err, int sm_count,
                            cudaStream_t st);
 
 }  // namespace nmoe

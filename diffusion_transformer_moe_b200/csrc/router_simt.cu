@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(kThreads)
 router_simt_kernel(const T* __restrict__ x, const T* __restrict__ W_r, int Tn, int d, int E,
                    int S, int score_fn, const float* __restrict__ bias,
                    float* __restrict__ scores, float* __restrict__ scores_t) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ double smem_d[];
   double* lg = smem_d;                                // [kBM][E + 1] logits / scores
   float* xs = reinterpret_cast<float*>(lg + kBM * (E + 1));  // [kBM][kBK + 1]
@@ -132,18 +134,13 @@ cudaError_t launch_router_simt(const void* x, const void* W_r, const Shape& s, n
   size_t smem = sizeof(double) * (size_t)kBM * (s.E + 1) +
                 sizeof(float) * (size_t)(kBM * (kBK + 1) + kBK * s.E);
   dim3 grid((unsigned)ceil_div(s.T, kBM));
-  if (dt == NMOE_F32) {
-    auto k = router_simt_kernel<float>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, kThreads, smem, st>>>((const float*)x, (const float*)W_r, s.T, s.d, s.E, s.S,
-                                    (int)fn, bias, scores, scores_t);
-  } else {
-    auto k = router_simt_kernel<__nv_bfloat16>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, kThreads, smem, st>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)W_r, s.T,
-                                    s.d, s.E, s.S, (int)fn, bias, scores, scores_t);
-  }
-  return cudaGetLastError();
+  if (dt == NMOE_F32)
+    return launch_kernel(router_simt_kernel<float>, grid, dim3(kThreads), smem, st, s.pdl, 1,
+                         (const float*)x, (const float*)W_r, s.T, s.d, s.E, s.S, (int)fn, bias,
+                         scores, scores_t);
+  return launch_kernel(router_simt_kernel<__nv_bfloat16>, grid, dim3(kThreads), smem, st, s.pdl,
+                       1, (const __nv_bfloat16*)x, (const __nv_bfloat16*)W_r, s.T, s.d, s.E, s.S,
+                       (int)fn, bias, scores, scores_t);
 }
 
 }  // namespace nmoe

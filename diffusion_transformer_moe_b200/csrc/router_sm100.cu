@@ -6,9 +6,9 @@
 // Precision: the scores must match an fp64 reference to 1e-5 relative, and with
 // LogNormal-scaled tokens the logits reach |l| ~ 30, where a single fp32 accumulator
 // over d = 2048 drifts by more than that (tensor-core accumulation also truncates). So
-// the MMAs accumulate only 32-long k-chunks in TMEM (two chunk slices per 64-wide
-// k-block), and the epilogue warps read every chunk back with tcgen05.ld and add it to
-// fp64 running sums in registers. Max, exp and the normalisation run in fp64; each
+// the MMAs accumulate only one 64-long k-chunk per TMEM slice, and the epilogue warps
+// read every chunk back with tcgen05.ld (two chunks per round trip) and add it to
+// Kahan-compensated fp32 running sums, taken in fp64 at the end. Max, exp and the normalisation run in fp64; each
 // score is rounded once to fp32.
 //
 // Each 128-token tile is split along d between the two CTAs of a cluster (so T = 8192
@@ -48,7 +48,7 @@ struct Params {
   int T, d, E, S;
   int epad;         // N of the MMA: E rounded up to 64
   int nbox;         // epad / 64
-  int nbuf;         // TMEM chunk buffers of 2 * epad columns
+  int nbuf;         // TMEM chunk buffers of epad columns (even)
   int score_fn;
   const float* bias;
   float* scores;
@@ -65,12 +65,14 @@ __device__ __forceinline__ double exp_f64_arg(double a) {
   return (double)expf(hi) * (1.0 + (a - (double)hi));
 }
 
-// CW: experts per epilogue thread (16 or 32); G = ceil(E / CW) column groups, so the
-// epilogue has 4 G warps (one per TMEM lane quarter and group).
+// Each epilogue thread owns CW experts (16 up to E = 64, else 32) of one token row;
+// G = ceil(E / CW) column groups, so the epilogue has 4 G warps (one per TMEM lane
+// quarter and group).
 template <int G, int CW>
 __global__ void __launch_bounds__(64 + 128 * G, 1)
 router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
                     const __grid_constant__ CUtensorMap map_w, const Params p) {
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -104,6 +106,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
   volatile int* abort_v = &abort_flag;
+  pdl_wait();  // x, W_r and the bias are complete; earlier readers of the outputs are done
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -141,13 +144,13 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sA + stage * kABytes);
         const uint32_t b_addr = smem_u32(sB + stage * b_bytes);
-        const uint32_t d0 = tmem_base + buf * 2 * p.epad;
+        const uint32_t d0 = tmem_base + buf * p.epad;
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, kBBoxBytes, 1024);
-          // chunk slice kk / 2, restarted at the first MMA of each slice
-          mma_bf16(d0 + (kk >> 1) * p.epad, ad, bd, idesc, kk & 1);
+          // one chunk slice per k-block, restarted at the block's first MMA
+          mma_bf16(d0, ad, bd, idesc, kk != 0);
         }
         mma_commit(&empty_bar[stage]);
         mma_commit(&tfull_bar[buf]);
@@ -164,49 +167,69 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
     const int g = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const int e0 = g * CW;
-    double acc[CW];
+    // Kahan-compensated fp32 sums of the 32-long chunk sums: hi accumulates, lo keeps
+    // what each addition rounded away (error ~2 ulp of the total, however many chunks);
+    // hi + lo is taken in fp64 once at the end.
+    float hi[CW], lo[CW];
 #pragma unroll
-    for (int j = 0; j < CW; ++j) acc[j] = 0.0;
+    for (int j = 0; j < CW; ++j) { hi[j] = 0.f; lo[j] = 0.f; }
     int buf = 0;
     uint32_t buf_phase = 0;
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
+    // two k-blocks (two chunk slices) per TMEM-load round trip
+    for (int kb = 0; kb < nk; kb += 2) {
+      const bool two = kb + 1 < nk;
       int w = 1;
-      if (lane == 0) w = mbar_wait(&tfull_bar[buf], buf_phase, abort_v, kWaitNs);
+      if (lane == 0) {
+        w = mbar_wait(&tfull_bar[buf], buf_phase, abort_v, kWaitNs);
+        if (w && two) w = mbar_wait(&tfull_bar[buf + 1], buf_phase, abort_v, kWaitNs);
+      }
       if (__shfl_sync(0xffffffffu, w, 0) == 0) { ok = false; break; }
       tc_fence_after();
-      const uint32_t taddr =
-          tmem_base + ((uint32_t)(q * 32) << 16) + buf * 2 * p.epad + e0;
-      // both 32-long chunk slices of this thread's experts, 16 columns at a time; the
-      // two chunk sums are added in fp32 (one rounding), then into fp64
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * p.epad + e0;
 #pragma unroll
       for (int h = 0; h < CW / 16; ++h) {
         uint32_t c0[16], c1[16];
         tmem_ld16(taddr + h * 16, c0);
-        tmem_ld16(taddr + p.epad + h * 16, c1);
+        if (two) tmem_ld16(taddr + p.epad + h * 16, c1);
         tmem_ld_wait();
         if (h == CW / 16 - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+          if (lane == 0) {
+            mbar_arrive(&tempty_bar[buf]);
+            if (two) mbar_arrive(&tempty_bar[buf + 1]);
+          }
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          acc[h * 16 + j] += (double)(__uint_as_float(c0[j]) + __uint_as_float(c1[j]));
+        for (int j = 0; j < 16; ++j) {
+          // the k-blocks' two 64-long chunk sums (one rounding), then Kahan
+          const float c = two ? __uint_as_float(c0[j]) + __uint_as_float(c1[j])
+                              : __uint_as_float(c0[j]);
+          const float y = c - lo[h * 16 + j];
+          const float t = hi[h * 16 + j] + y;
+          lo[h * 16 + j] = (t - hi[h * 16 + j]) - y;
+          hi[h * 16 + j] = t;
+        }
       }
-      if (++buf == p.nbuf) { buf = 0; buf_phase ^= 1; }
+      buf += 2;
+      if (buf >= p.nbuf) { buf -= p.nbuf; buf_phase ^= 1; }
     }
+    double acc[CW];
+#pragma unroll
+    for (int j = 0; j < CW; ++j) acc[j] = (double)hi[j] - (double)lo[j];
     // After the cluster barrier both CTAs' stage rings are idle. The second CTA adds its
     // half-d sums into the first CTA's ring laid out [E][128] (a warp writes 32
     // consecutive doubles per expert), then the first CTA finishes in registers.
     double* part = reinterpret_cast<double*>(smem);
     double* red = part + (size_t)kMaxE * kBM;   // [2][G][128]: row max, then row sum
     cluster.sync();                       // (1) every ring is idle
+    // expert pair (e, e+1) of token row at part[((e / 2) * 128 + row) * 2 + (e & 1)]
     if (rank != 0) {
-      double* remote = cluster.map_shared_rank(part, 0);
+      double2* remote = reinterpret_cast<double2*>(cluster.map_shared_rank(part, 0));
 #pragma unroll
-      for (int j = 0; j < CW; ++j)
-        if (e0 + j < p.E) remote[(e0 + j) * kBM + row] = acc[j];
+      for (int j = 0; j < CW; j += 2)
+        if (e0 + j < p.E) remote[((e0 + j) >> 1) * kBM + row] = make_double2(acc[j], acc[j + 1]);
     }
     cluster.sync();                       // (2) the second half's sums have landed
     if (rank == 0) {
@@ -214,12 +237,19 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       const int t = t0 + row;
       const bool live = t < p.T;
       const float* b = (p.bias != nullptr && live) ? p.bias + (int64_t)(t / p.S) * p.E : nullptr;
+      const double2* pp = reinterpret_cast<const double2*>(part);
 #pragma unroll
-      for (int j = 0; j < CW; ++j) {
+      for (int j = 0; j < CW; j += 2) {
         if (e0 + j < p.E) {
-          acc[j] += part[(e0 + j) * kBM + row];
-          if (b) acc[j] += (double)b[e0 + j];
+          const double2 v = pp[((e0 + j) >> 1) * kBM + row];
+          acc[j] += v.x;
+          acc[j + 1] += v.y;
         }
+      }
+      if (b) {
+#pragma unroll
+        for (int j = 0; j < CW; ++j)
+          if (e0 + j < p.E) acc[j] += (double)b[e0 + j];
       }
       if (p.score_fn == NMOE_SCORE_SOFTMAX) {
         double m = -INFINITY;
@@ -323,7 +353,7 @@ cudaError_t launch_router_sm100(const void* x, const void* W_r, const Shape& s,
   p.T = s.T; p.d = s.d; p.E = s.E; p.S = s.S;
   p.epad = (int)ceil_div(s.E, 64) * 64;
   p.nbox = p.epad / 64;
-  p.nbuf = 512 / (2 * p.epad);
+  p.nbuf = 512 / p.epad;   // one epad-wide chunk slice per k-block: 8 (E <= 64) or 4
   if (p.nbuf > 8) p.nbuf = 8;
   p.score_fn = (int)fn;
   p.bias = bias; p.scores = scores; p.scores_t = scores_t; p.err = err;
@@ -343,23 +373,8 @@ cudaError_t launch_router_sm100(const void* x, const void* W_r, const Shape& s,
                      : G == 3 ? router_sm100_kernel<3, 16>
                               : router_sm100_kernel<4, 16>)
                     : (G == 3 ? router_sm100_kernel<3, 32> : router_sm100_kernel<4, 32>);
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(ceil_div(s.T, kBM) * kSplit));
-  cfg.blockDim = dim3(64 + 128 * G);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kSplit;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, k, mx, mw, p);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_kernel(k, dim3((unsigned)(ceil_div(s.T, kBM) * kSplit)), dim3(64 + 128 * G), smem,
+                       st, s.pdl, kSplit, mx, mw, p);
 }
 
 }  // namespace nmoe

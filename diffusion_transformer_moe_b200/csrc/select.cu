@@ -14,7 +14,9 @@
 // csr_kernel: one CTA per 32 consecutive tokens. Because each expert's list is sorted,
 // the number of entries that belong to tokens before t0 is sum_e lower_bound(idx[e], t0),
 // so every CTA finds its output offset with E binary searches: no global scan, no
-// atomics, and every output element has exactly one writer.
+// atomics, and every output element has exactly one writer. It also records, for every
+// (expert, slot), its position in that token-major order (ent_pos), where the down-
+// projection writes the row so that the combine reads each token's rows contiguously.
 #include "nmoe_internal.cuh"
 
 namespace nmoe {
@@ -66,6 +68,8 @@ __global__ void __launch_bounds__(kSelThreads)
 select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int Ce,
               int cached, int32_t* __restrict__ idx, float* __restrict__ gate,
               unsigned* __restrict__ err) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ uint32_t s_keys[];
   __shared__ unsigned s_hist[256];
   __shared__ int s_scan[2 * kSelWarps + 2];
@@ -185,8 +189,10 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
 
 __global__ void __launch_bounds__(kCsrThreads)
 csr_kernel(const int32_t* __restrict__ idx, int Tn, int E, int Ce, int32_t* __restrict__ tok_ptr,
-           int32_t* __restrict__ tok_ent, float* __restrict__ gate, int normalize,
-           float route_scale, unsigned* __restrict__ err) {
+           int32_t* __restrict__ tok_ent, int32_t* __restrict__ ent_pos, float* __restrict__ gate,
+           int normalize, float route_scale, unsigned* __restrict__ err) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ int s_slot[];  // [kCsrTok][E]: slot of (token, expert) or -1
   __shared__ int s_lo[256], s_hi[256];
   __shared__ int s_base_part[kCsrThreads / 32];
@@ -250,7 +256,11 @@ csr_kernel(const int32_t* __restrict__ idx, int Tn, int E, int Ce, int32_t* __re
       int e = e0 + lane;
       int sl = e < E ? srow[e] : -1;
       unsigned m = __ballot_sync(0xffffffffu, sl >= 0);
-      if (sl >= 0) tok_ent[out + __popc(m & ((1u << lane) - 1u))] = e * Ce + sl;
+      if (sl >= 0) {
+        const int at = out + __popc(m & ((1u << lane) - 1u));
+        tok_ent[at] = e * Ce + sl;
+        if (ent_pos != nullptr) ent_pos[e * Ce + sl] = at;
+      }
       out += __popc(m);
     }
     if (normalize) {
@@ -274,24 +284,19 @@ cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, f
                           unsigned* err, cudaStream_t st) {
   int cached = s.S <= kSelMaxCached;
   size_t smem = cached ? sizeof(uint32_t) * (size_t)s.S : 0;
-  cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)(sizeof(uint32_t) * kSelMaxCached));
   dim3 grid((unsigned)s.E, (unsigned)s.n_seg);
-  select_kernel<<<grid, kSelThreads, smem, st>>>(scores_t, s.T, s.S, s.C, s.Ce, cached, idx,
-                                                 gate, err);
-  return cudaGetLastError();
+  return launch_kernel(select_kernel, grid, dim3(kSelThreads), smem, st, s.pdl, 1, scores_t,
+                       (int64_t)s.T, s.S, s.C, s.Ce, cached, idx, gate, err);
 }
 
 cudaError_t launch_csr(const int32_t* idx, const Shape& s, int32_t* tok_ptr, int32_t* tok_ent,
-                       float* gate, nmoe_combine combine, float route_scale, unsigned* err,
-                       cudaStream_t st) {
+                       int32_t* ent_pos, float* gate, nmoe_combine combine, float route_scale,
+                       unsigned* err, cudaStream_t st) {
   size_t smem = sizeof(int) * (size_t)kCsrTok * s.E;
-  cudaFuncSetAttribute(csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((unsigned)ceil_div(s.T, kCsrTok));
-  csr_kernel<<<grid, kCsrThreads, smem, st>>>(idx, s.T, s.E, s.Ce, tok_ptr, tok_ent, gate,
-                                              combine == NMOE_COMBINE_NORMALIZED, route_scale,
-                                              err);
-  return cudaGetLastError();
+  return launch_kernel(csr_kernel, grid, dim3(kCsrThreads), smem, st, s.pdl, 1, idx, s.T, s.E,
+                       s.Ce, tok_ptr, tok_ent, ent_pos, gate,
+                       (int)(combine == NMOE_COMBINE_NORMALIZED), route_scale, err);
 }
 
 }  // namespace nmoe

@@ -83,7 +83,7 @@ def test_workspace_size_accounts_for_every_buffer():
     n = nm.workspace_size(T, d, E, F, C_)
     Ce = E * C_
     # default (split) intermediates: H as a bf16 hi/lo pair, Y in fp32 -> 4 bytes each
-    minimum = 4 * T * E * 2 + 4 * Ce * 3 + 4 * (T + 1) + 4 * Ce * F + 4 * Ce * d
+    minimum = 4 * T * E * 2 + 4 * Ce * 4 + 4 * (T + 1) + 4 * Ce * F + 4 * Ce * d
     assert minimum <= n <= minimum + 16 * 256
     small = nm.workspace_size(T, d, E, F, C_, intermediate="bf16")
     assert small == n - 2 * Ce * F - 2 * Ce * d
