@@ -86,10 +86,11 @@ struct Params {
   unsigned* err;
 };
 
-// silu(g) = g * sigmoid(g); the reciprocal is correctly rounded and exp's error is a
-// few ulp, far below the hi/lo split's 16 bits. g -> -inf gives -0, g -> +inf gives g.
+// silu(g) = g * sigmoid(g) = g / (1 + e^-g) with the fast exp and the fast divide
+// (each within a few ulp of fp32, far below the hi/lo split's 16 bits). g is a finite
+// GEMM output; very negative g gives 0 and g -> +inf gives g.
 __device__ __forceinline__ float silu_f32(float g) {
-  return g * __frcp_rn(1.f + __expf(-g));
+  return __fdividef(g, 1.f + __expf(-g));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
