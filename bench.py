@@ -273,6 +273,24 @@ def run_reference(args, w, rank):
     print(json.dumps(line), flush=True)
 
 
+# ---- multi-rank plumbing (replicas) ---------------------------------------------------------
+
+def max_over_ranks(vals, dist, device):
+    """Element-wise maximum of per-rank timings. Every rank calls it, in the same order."""
+    if dist is None:
+        return [float(v) for v in vals]
+    import torch
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def replica_throughput(T, world, K, ms):
+    """Whole-job tokens/s: every rank ran K batches of T tokens; ms is the slowest rank's
+    total time for them."""
+    return T * world * K / (ms / 1e3)
+
+
 # ---- our CUDA path ---------------------------------------------------------------------
 
 def run_ours(args, w, rank, world, local_rank, dist):
@@ -309,21 +327,29 @@ def run_ours(args, w, rank, world, local_rank, dist):
     if nm.get_last_error() != 0:
         raise RuntimeError("device-side check failed during warm-up")
 
+    def timed(tr):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step(tr)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return sum(s.elapsed_time(e) for s, e in ev)
+
+    # the timed region: K whole-layer steps, launched back to back as a user would
     clocks = ClockSampler(local_rank)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
-    barrier()
-    torch.cuda.synchronize()
     clocks.start()
-    for i in range(K):
-        flush.zero_()
-        ev[i][0].record(stream)
-        step(trace)
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier()
+    ms = timed(None)
     clk = clocks.stop()
-    ms = sum(s.elapsed_time(e) for s, e in ev)
+    # per-stage times: K more steps with CUDA events recorded between the stages (the
+    # events keep the stages from overlapping their launches, so this pass is not the
+    # headline number)
+    traced_ms = timed(trace)
     stage_ms, ncalls = trace.read()
     if nm.get_last_error() != 0:
         raise RuntimeError("device-side check failed during the timed steps")
@@ -349,17 +375,13 @@ def run_ours(args, w, rank, world, local_rank, dist):
     barrier()
     e2e_ms = sum(s.elapsed_time(e) for s, e in e2e_ev)
 
-    if dist is not None:
-        t = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = t.tolist()
+    ms, e2e_ms, traced_ms = max_over_ranks([ms, e2e_ms, traced_ms], dist, dev)
     if rank != 0:
         return
 
     peaks = _peaks()
     per_step_s = ms / 1e3 / K
-    tokens = w.T * world * K
-    value = tokens / (ms / 1e3)
+    value = replica_throughput(w.T, world, K, ms)
     sb = stage_bytes(w, inter)
     sf = stage_flops(w, inter)
     stages = {}
@@ -390,8 +412,9 @@ def run_ours(args, w, rank, world, local_rank, dist):
         "tensor_frac_of_layer": flops / per_step_s / 1e12 / peaks["tensor_sustained"],
         "roofline": roof,
         "stages": stages,
+        "traced_ms_per_step": traced_ms / K,
         "gpu_launches": 6 * K,
-        "e2e": {"value": w.T * world * K / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": replica_throughput(w.T, world, K, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
         "clocks": clk,

@@ -84,6 +84,7 @@ nmoe_status check_shape(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C, i
   if (E < 1 || E > 256) return NMOE_ERR_INVALID_ARG;
   if (n_seg < 1 || n_seg > 65535 || T % n_seg != 0) return NMOE_ERR_INVALID_ARG;
   if (C < 1 || C > T / n_seg) return NMOE_ERR_INVALID_ARG;
+  if (T / n_seg > nmoe::kSelectMaxRow) return NMOE_ERR_UNSUPPORTED;
   if (E * n_seg * C >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
   if (need_dF) {
     if (d < 1 || F < 1) return NMOE_ERR_INVALID_ARG;
@@ -111,7 +112,7 @@ size_t out_size(nmoe_dtype dt, const nmoe_options& o) {
 }
 
 struct Layout {
-  size_t scores, scores_t, idx, gate, tok_ptr, tok_ent, ent_pos, H, Y, xin, xout, total;
+  size_t scores, scores_t, idx, gate, bnd, tok_ptr, tok_ent, ent_pos, H, Y, xin, xout, total;
 };
 
 Layout make_layout(const Shape& s, nmoe_dtype dt, const nmoe_options& o) {
@@ -124,6 +125,7 @@ Layout make_layout(const Shape& s, nmoe_dtype dt, const nmoe_options& o) {
   L.scores_t = take(sizeof(float) * (size_t)s.T * s.E);
   L.idx = o.idx_out ? none : take(sizeof(int32_t) * (size_t)s.E * s.Ce);
   L.gate = take(sizeof(float) * (size_t)s.E * s.Ce);
+  L.bnd = take(sizeof(int32_t) * nmoe::select_bound_entries(s));
   L.tok_ptr = take(sizeof(int32_t) * ((size_t)s.T + 1));
   L.tok_ent = take(sizeof(int32_t) * (size_t)s.E * s.Ce);
   L.ent_pos = take(sizeof(int32_t) * (size_t)s.E * s.Ce);
@@ -203,6 +205,7 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   float* scores_t = reinterpret_cast<float*>(ws + L.scores_t);
   int32_t* idx = o.idx_out ? o.idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
   float* gate = reinterpret_cast<float*>(ws + L.gate);
+  int32_t* bnd = reinterpret_cast<int32_t*>(ws + L.bnd);
   int32_t* tok_ptr = reinterpret_cast<int32_t*>(ws + L.tok_ptr);
   int32_t* tok_ent = reinterpret_cast<int32_t*>(ws + L.tok_ent);
   int32_t* ent_pos = reinterpret_cast<int32_t*>(ws + L.ent_pos);
@@ -237,11 +240,11 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
                                    scores_t, st);
   }
   mark(1);
-  if (e == cudaSuccess) e = nmoe::launch_select(scores_t, s, idx, gate, ds->err, st);
+  if (e == cudaSuccess) e = nmoe::launch_select(scores_t, s, idx, gate, bnd, ds->err, st);
   mark(2);
   if (e == cudaSuccess)
-    e = nmoe::launch_csr(idx, s, tok_ptr, tok_ent, ent_pos, gate, o.combine, o.route_scale,
-                         ds->err, st);
+    e = nmoe::launch_csr(idx, bnd, s, tok_ptr, tok_ent, ent_pos, gate, o.combine,
+                         o.route_scale, ds->err, st);
   mark(3);
   const bool tc = !f32 && nmoe::experts_sm100_supported(s);
   // SPLIT on the tensor cores: H_hi then H_lo, each [E*Ce, F] bf16; on the CUDA cores
@@ -338,10 +341,11 @@ nmoe_status nmoe_select(const float* scores_t, int64_t T, int64_t E, int64_t C,
   if ((v = dev_state(&ds)) != NMOE_OK) return v;
   const Shape s = make_shape(T, 8, E, 8, C, n_segments);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = nmoe::launch_select(scores_t, s, idx, gate, ds->err, st);
+  // no scratch here: the CSR build searches idx instead of reading a boundary table
+  cudaError_t e = nmoe::launch_select(scores_t, s, idx, gate, nullptr, ds->err, st);
   if (e == cudaSuccess && tok_ptr)
-    e = nmoe::launch_csr(idx, s, tok_ptr, tok_ent, nullptr, gate, NMOE_COMBINE_RAW, 1.f, ds->err,
-                         st);
+    e = nmoe::launch_csr(idx, nullptr, s, tok_ptr, tok_ent, nullptr, gate, NMOE_COMBINE_RAW,
+                         1.f, ds->err, st);
   if (e != cudaSuccess) { cudaGetLastError(); return NMOE_ERR_CUDA; }
   return NMOE_OK;
 }

@@ -33,15 +33,17 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Raises a kernel's dynamic shared-memory limit on the current device, once per
-// (kernel, device).
+// Raises a kernel's dynamic shared-memory limit on the current device to at least
+// `bytes`, once per (kernel, device, larger size). The default limit counts the
+// kernel's static shared memory against the same 48 KB, so every launch with dynamic
+// shared memory goes through here, not only those asking for more than 48 KB.
 cudaError_t set_smem_limit(const void* kernel, size_t bytes);
 
 // Launch with programmatic stream serialization (pdl) and an optional 1-D cluster.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                           cudaStream_t st, bool pdl, unsigned cluster_x, Args&&... args) {
-  if (smem > 48 * 1024) {
+  if (smem > 0) {
     cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(kernel), smem);
     if (e != cudaSuccess) return e;
   }
@@ -89,15 +91,24 @@ cudaError_t launch_router_simt(const void* x, const void* W_r, const Shape& s, n
                                nmoe_score_fn fn, const float* bias, float* scores,
                                float* scores_t, cudaStream_t st);
 
-cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, float* gate,
-                          unsigned* err, cudaStream_t st);
+// Longest segment (tokens per expert row) the selection takes: its per-row bitmaps live
+// in shared memory.
+constexpr int kSelectMaxRow = 1 << 19;
 
+// bnd (may be NULL) receives the block boundary table the CSR build reads: for every
+// block of 32 tokens b and expert e, bnd[b*E + e] = number of e's entries whose token
+// comes before the block; select_bound_entries(s) int32 entries.
+size_t select_bound_entries(const Shape& s);
+cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, float* gate,
+                          int32_t* bnd, unsigned* err, cudaStream_t st);
+
+// bnd: the table launch_select wrote, or NULL to search idx instead.
 // combine == NMOE_COMBINE_NORMALIZED rewrites gate[] in place to
 // route_scale * gate / (sum of the token's gates). ent_pos (may be NULL) receives, for
 // each entry e*Ce + slot, its index in the token-major order of tok_ent.
-cudaError_t launch_csr(const int32_t* idx, const Shape& s, int32_t* tok_ptr, int32_t* tok_ent,
-                       int32_t* ent_pos, float* gate, nmoe_combine combine, float route_scale,
-                       unsigned* err, cudaStream_t st);
+cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, int32_t* tok_ptr,
+                       int32_t* tok_ent, int32_t* ent_pos, float* gate, nmoe_combine combine,
+                       float route_scale, unsigned* err, cudaStream_t st);
 
 // CUDA-core expert GEMMs. dt is the type of x and the weights; h_f32 / y_f32 select
 // fp32 (else dt) for the H and Y intermediates.

@@ -6,17 +6,27 @@
 // the lower token index, and the chosen tokens are written in ascending token order.
 //
 // select_kernel: one CTA per (expert, segment). Scores are non-negative floats, so their
-// bit patterns order like unsigned integers. The CTA finds the exact C-th largest key
-// with an MSB-first radix select (four 8-bit digits; warp-aggregated shared-memory
-// histograms built with __match_any_sync), then compacts in token order: every key
-// above the threshold, plus the first (C - #above) keys equal to it.
+// bit patterns order like unsigned integers. The CTA stages its row of keys in shared
+// memory with 16-byte loads and finds the exact C-th largest key with an MSB-first radix
+// select over three digits (bits 31..20, 19..8, 7..0; shared-memory histograms). The
+// first digit splits fp32 scores into bins an eighth of an octave wide, so the bin
+// holding the threshold is a small share of the row: its keys are copied to a candidate
+// list and the last two digits are counted over that list alone (a list of at most
+// kRankMax keys is instead ranked directly, each key against all). One more sweep of the
+// row records, 32 tokens to a word, which keys lie above the threshold and which equal
+// it; a block-wide scan over the words' popcounts then gives every chosen key (each key
+// above the threshold, plus the first C - #above keys equal to it) its position in
+// ascending token order, and, for every block of kBlockTok tokens, how many of the
+// expert's entries come before the block (the boundary table).
 //
-// csr_kernel: one CTA per 32 consecutive tokens. Because each expert's list is sorted,
-// the number of entries that belong to tokens before t0 is sum_e lower_bound(idx[e], t0),
-// so every CTA finds its output offset with E binary searches: no global scan, no
-// atomics, and every output element has exactly one writer. It also records, for every
-// (expert, slot), its position in that token-major order (ent_pos), where the down-
-// projection writes the row so that the combine reads each token's rows contiguously.
+// csr_kernel: one CTA per kBlockTok consecutive tokens. The boundary table gives, for
+// every expert, the slot range [lo, hi) of its entries inside the block, and the sum of
+// the lo's is the block's offset in the token-major order: one coalesced load round, no
+// global scan and no atomics on global memory. Without the table (the standalone
+// selection call, which has no scratch) the same ranges come from binary searches of
+// each expert's ascending token list. The CTA also records, for every (expert, slot),
+// its position in that token-major order (ent_pos), where the down projection writes
+// the row so that the combine reads each token's rows contiguously.
 #include "nmoe_internal.cuh"
 
 namespace nmoe {
@@ -26,9 +36,38 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 // Rows up to this many keys are staged in shared memory; longer rows are read from
 // global memory (L2) on every pass.
-constexpr int kSelMaxCached = 48 * 1024;
+constexpr int kSelMaxCached = 40 * 1024;
+constexpr int kBins = 4096;     // 12-bit digits; thread t owns bins [4t, 4t + 4)
+constexpr int kCandMax = 4096;  // capacity of the candidate list
+constexpr int kRankMax = 256;   // candidate lists up to this long are ranked directly
+static_assert(kBins == 4 * kSelThreads, "four histogram bins per thread");
 
-__device__ __forceinline__ uint32_t load_key(const uint32_t* p) { return *p; }
+constexpr int kBlockTok = 32;   // tokens per CSR block (one warp lane per token)
+static_assert(kBlockTok == 32, "one bitmap word per CSR block");
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ __forceinline__ unsigned is_bad(uint32_t key) {
+  return key >= 0x7f800000u;  // negative, +inf or NaN
+}
+
+// Adds to hist[] the digit (key >> shift) & dmask of every key in src[0, n) whose bits
+// under pmask equal prefix: one shared-memory atomic per key. The loop is bound by
+// instruction issue, not by address conflicts: grouping equal digits first (with
+// __match_any_sync, or a ballot on the first lane's digit) costs more than the
+// conflicts it saves, even on rows full of equal scores.
+__device__ __forceinline__ void histogram(const uint32_t* src, int n, uint32_t pmask,
+                                          uint32_t prefix, int shift, uint32_t dmask,
+                                          unsigned* hist) {
+  for (int i = threadIdx.x; i < n; i += kSelThreads) {
+    const uint32_t key = src[i];
+    if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+  }
+}
 
 // Exclusive block scan of two counters at once; returns the block totals.
 __device__ __forceinline__ void block_scan2(int a, int b, int* ex_a, int* ex_b, int* tot_a,
@@ -37,146 +76,251 @@ __device__ __forceinline__ void block_scan2(int a, int b, int* ex_a, int* ex_b, 
   int ia = a, ib = b;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int va = __shfl_up_sync(0xffffffffu, ia, o);
-    int vb = __shfl_up_sync(0xffffffffu, ib, o);
-    if (lane >= o) { ia += va; ib += vb; }
-  }
-  if (lane == 31) { sh[warp] = ia; sh[kSelWarps + warp] = ib; }
-  __syncthreads();
-  if (warp == 0) {
-    int wa = lane < kSelWarps ? sh[lane] : 0;
-    int wb = lane < kSelWarps ? sh[kSelWarps + lane] : 0;
-    int sa = wa, sb = wb;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int va = __shfl_up_sync(0xffffffffu, sa, o);
-      int vb = __shfl_up_sync(0xffffffffu, sb, o);
-      if (lane >= o) { sa += va; sb += vb; }
+    const int va = __shfl_up_sync(0xffffffffu, ia, o);
+    const int vb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += va;
+      ib += vb;
     }
-    if (lane < kSelWarps) { sh[lane] = sa - wa; sh[kSelWarps + lane] = sb - wb; }
-    if (lane == kSelWarps - 1) { sh[2 * kSelWarps] = sa; sh[2 * kSelWarps + 1] = sb; }
+  }
+  if (lane == 31) {
+    sh[warp] = ia;
+    sh[kSelWarps + warp] = ib;
   }
   __syncthreads();
-  *ex_a = sh[warp] + ia - a;
-  *ex_b = sh[kSelWarps + warp] + ib - b;
-  *tot_a = sh[2 * kSelWarps];
-  *tot_b = sh[2 * kSelWarps + 1];
+  int wa = sh[lane], wb = sh[kSelWarps + lane];  // kSelWarps == 32
+  int sa = wa, sb = wb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int va = __shfl_up_sync(0xffffffffu, sa, o);
+    const int vb = __shfl_up_sync(0xffffffffu, sb, o);
+    if (lane >= o) {
+      sa += va;
+      sb += vb;
+    }
+  }
+  *ex_a = __shfl_sync(0xffffffffu, sa - wa, warp) + ia - a;
+  *ex_b = __shfl_sync(0xffffffffu, sb - wb, warp) + ib - b;
+  *tot_a = __shfl_sync(0xffffffffu, sa, 31);
+  *tot_b = __shfl_sync(0xffffffffu, sb, 31);
+}
+
+// The bin d that holds the k-th largest of the counted keys (bins in descending order):
+// res[0] = d, res[1] = number of counted keys in higher bins, res[2] = hist[d]. Exactly
+// one thread writes res; the caller synchronises before reading it.
+__device__ __forceinline__ void find_digit(const unsigned* hist, unsigned k, unsigned* wsum,
+                                           unsigned* res) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint4 c = reinterpret_cast<const uint4*>(hist)[tid];
+  const unsigned mine = c.x + c.y + c.z + c.w;
+  unsigned suf = mine;  // bins of this lane and the higher lanes of the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned v = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += v;
+  }
+  if (lane == 0) wsum[warp] = suf;
   __syncthreads();
+  unsigned wsuf = wsum[lane];  // then: warps lane .. 31
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned v = __shfl_down_sync(0xffffffffu, wsuf, o);
+    if (lane + o < 32) wsuf += v;
+  }
+  const unsigned higher_warps = __shfl_sync(0xffffffffu, wsuf, (warp + 1) & 31);
+  unsigned above = (warp == kSelWarps - 1 ? 0u : higher_warps) + (suf - mine);
+  const unsigned cnt[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int j = 3; j >= 0; --j) {
+    if (above < k && above + cnt[j] >= k) {
+      res[0] = (unsigned)(4 * tid + j);
+      res[1] = above;
+      res[2] = cnt[j];
+    }
+    above += cnt[j];
+  }
 }
 
 __global__ void __launch_bounds__(kSelThreads)
-select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int Ce,
+select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int Ce, int E,
               int cached, int32_t* __restrict__ idx, float* __restrict__ gate,
-              unsigned* __restrict__ err) {
+              int32_t* __restrict__ bnd, unsigned* __restrict__ err) {
   pdl_launch_dependents();
-  pdl_wait();
-  extern __shared__ uint32_t s_keys[];
-  __shared__ unsigned s_hist[256];
-  __shared__ int s_scan[2 * kSelWarps + 2];
-  __shared__ unsigned s_digit, s_above, s_bad;
+  // dynamic: [keys, cached ? S (rounded up to 4) : 0][gt words, nw4][eq words, nw4]
+  extern __shared__ __align__(16) uint32_t s_dyn[];
+  __shared__ __align__(16) unsigned s_hist[kBins];
+  __shared__ uint32_t s_cand[kCandMax];
+  __shared__ unsigned s_wsum[kSelWarps];
+  __shared__ int s_scan[2 * kSelWarps];
+  __shared__ unsigned s_res[3];
+  __shared__ unsigned s_ncand;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int e = blockIdx.x, g = blockIdx.y;
+  const int nw = (S + 31) >> 5, nw4 = (nw + 3) & ~3;
+  uint32_t* s_keys = s_dyn;
+  uint32_t* s_gtw = s_dyn + (cached ? ((S + 3) & ~3) : 0);
+  uint32_t* s_eqw = s_gtw + nw4;
+
+  reinterpret_cast<uint4*>(s_hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
+  if (tid == 0) s_ncand = 0;
+  pdl_wait();
+
   const uint32_t* row =
       reinterpret_cast<const uint32_t*>(scores_t + (int64_t)e * Tn + (int64_t)g * S);
-
-  if (tid == 0) s_bad = 0;
-  __syncthreads();
   const uint32_t* keys = row;
-  {
-    // Non-negative finite scores only: sign bit clear and below +inf.
-    unsigned bad = 0;
-    if (cached) {
-      for (int i = tid; i < S; i += kSelThreads) {
-        uint32_t k = row[i];
-        bad |= (k >= 0x7f800000u);
-        s_keys[i] = k;
+  // Non-negative finite scores only: sign bit clear and below +inf.
+  unsigned bad = 0;
+  if (cached) {
+    int head = 0;
+    if ((reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+      const int n4 = S >> 2;
+      const uint4* r4 = reinterpret_cast<const uint4*>(row);
+      uint4* k4 = reinterpret_cast<uint4*>(s_keys);
+#pragma unroll 4
+      for (int i = tid; i < n4; i += kSelThreads) {
+        const uint4 v = r4[i];
+        bad |= is_bad(v.x) | is_bad(v.y) | is_bad(v.z) | is_bad(v.w);
+        k4[i] = v;
       }
-      keys = s_keys;
-    } else {
-      for (int i = tid; i < S; i += kSelThreads) bad |= (row[i] >= 0x7f800000u);
+      head = 4 * n4;
     }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&s_bad, 1u);
+#pragma unroll 4
+    for (int i = head + tid; i < S; i += kSelThreads) {
+      const uint32_t v = row[i];
+      bad |= is_bad(v);
+      s_keys[i] = v;
+    }
+    keys = s_keys;
+  } else {
+#pragma unroll 4
+    for (int i = tid; i < S; i += kSelThreads) bad |= is_bad(row[i]);
   }
-  __syncthreads();
-  if (s_bad) {
-    if (tid == 0) atomicOr(err, kErrDeviceCheck);
-  }
+  if (__syncthreads_or((int)bad) && tid == 0) atomicOr(err, kErrDeviceCheck);
 
   // MSB-first radix select of the C-th largest key.
+  const uint32_t* src = keys;
+  int n = S;
   uint32_t prefix = 0, pmask = 0;
   int k = C;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kSelThreads) s_hist[i] = 0;
+  bool ranked = false;
+#pragma unroll 1
+  for (int pass = 0; pass < 3 && !ranked; ++pass) {
+    const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
+    const uint32_t dmask = pass == 2 ? 0xffu : 0xfffu;
+    histogram(src, n, pmask, prefix, shift, dmask, s_hist);
     __syncthreads();
-    for (int i0 = 0; i0 < S; i0 += kSelThreads) {
-      int i = i0 + tid;
-      uint32_t key = i < S ? load_key(keys + i) : 0u;
-      bool in = (i < S) && ((key & pmask) == prefix);
-      unsigned digit = in ? ((key >> shift) & 255u) : 256u;
-      unsigned peers = __match_any_sync(0xffffffffu, digit);
-      if (in && lane == __ffs(peers) - 1) atomicAdd(&s_hist[digit], (unsigned)__popc(peers));
-    }
+    find_digit(s_hist, (unsigned)k, s_wsum, s_res);
     __syncthreads();
-    if (warp == 0) {
-      // lane L owns bins [8L, 8L+8); count of keys with a larger digit than each bin
-      unsigned c[8], mine = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { c[j] = s_hist[lane * 8 + j]; mine += c[j]; }
-      // inclusive suffix sum over lanes (higher lanes hold higher digits)
-      unsigned suf = mine;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        unsigned v = __shfl_down_sync(0xffffffffu, suf, o);
-        if (lane + o < 32) suf += v;
-      }
-      unsigned above = suf - mine;  // keys in bins owned by higher lanes
-#pragma unroll
-      for (int j = 7; j >= 0; --j) {
-        if (above < (unsigned)k && above + c[j] >= (unsigned)k) {
-          s_digit = (unsigned)(lane * 8 + j);
-          s_above = above;
+    prefix |= s_res[0] << shift;
+    pmask |= dmask << shift;
+    k -= (int)s_res[1];
+    const int nbin = (int)s_res[2];
+    reinterpret_cast<uint4*>(s_hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
+    if (pass == 0 && nbin <= kCandMax) {
+      // keys of the threshold's bin; their order is irrelevant to the histograms
+      for (int i0 = 0; i0 < S; i0 += kSelThreads) {
+        const int i = i0 + tid;
+        const uint32_t key = i < S ? keys[i] : 0u;
+        const bool in = i < S && (key & pmask) == prefix;
+        const unsigned b = __ballot_sync(0xffffffffu, in);
+        if (b != 0u) {
+          unsigned base = 0;
+          if (lane == 0) base = atomicAdd(&s_ncand, (unsigned)__popc(b));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          const unsigned at = base + (unsigned)__popc(b & lanemask_lt());
+          if (in && at < (unsigned)kCandMax) s_cand[at] = key;
         }
-        above += c[j];
+      }
+      src = s_cand;
+      n = nbin;
+      if (nbin <= kRankMax) {
+        // Few candidates: rank them directly instead of two more digits. The k-th
+        // largest candidate c has #{> c} < k <= #{>= c}; equal candidates agree.
+        __syncthreads();
+        if (tid < nbin) {
+          const uint32_t c = s_cand[tid];
+          int gt = 0, ge = 0;
+          for (int j = 0; j < nbin; ++j) {
+            const uint32_t o = s_cand[j];
+            gt += o > c;
+            ge += o >= c;
+          }
+          if (gt < k && k <= ge) {
+            s_res[0] = c;
+            s_res[1] = (unsigned)gt;
+          }
+        }
+        __syncthreads();
+        prefix = s_res[0];
+        k -= (int)s_res[1];
+        ranked = true;
       }
     }
-    __syncthreads();
-    k -= (int)s_above;
-    prefix |= s_digit << shift;
-    pmask |= 255u << shift;
     __syncthreads();
   }
   const uint32_t thr = prefix;  // the C-th largest key; take k keys equal to it
 
-  // Ordered compaction: thread tid owns a contiguous run of keys.
-  const int per = (S + kSelThreads - 1) / kSelThreads;
-  const int b0 = min(S, tid * per), b1 = min(S, b0 + per);
-  int n_gt = 0, n_eq = 0;
-  for (int i = b0; i < b1; ++i) {
-    uint32_t key = load_key(keys + i);
-    n_gt += key > thr;
-    n_eq += key == thr;
-  }
-  int ex_gt, ex_eq, tot_gt, tot_eq;
-  block_scan2(n_gt, n_eq, &ex_gt, &ex_eq, &tot_gt, &tot_eq, s_scan);
-  int eq_seen = ex_eq;
-  int pos = ex_gt + min(ex_eq, k);
-  int32_t* out_idx = idx + (int64_t)e * Ce + (int64_t)g * C;
-  float* out_gate = gate + (int64_t)e * Ce + (int64_t)g * C;
-  for (int i = b0; i < b1; ++i) {
-    uint32_t key = load_key(keys + i);
-    bool take = key > thr;
-    if (key == thr) { take = eq_seen < k; ++eq_seen; }
-    if (take) {
-      out_idx[pos] = g * S + i;
-      out_gate[pos] = __uint_as_float(key);
-      ++pos;
+  // Word w of the bitmaps covers keys [32w, 32w + 32): bit b set if key 32w + b is
+  // above (gt) or equal to (eq) the threshold.
+  for (int w = warp; w < nw; w += kSelWarps) {
+    const int i = 32 * w + lane;
+    const uint32_t key = i < S ? keys[i] : 0u;
+    const unsigned gw = __ballot_sync(0xffffffffu, i < S && key > thr);
+    const unsigned qw = __ballot_sync(0xffffffffu, i < S && key == thr);
+    if (lane == 0) {
+      s_gtw[w] = gw;
+      s_eqw[w] = qw;
     }
   }
-  if (tid == 0 && tot_gt + min(tot_eq, k) != C) atomicOr(err, kErrDeviceCheck);
+  __syncthreads();
+
+  // Thread tid owns words [w0, w1); a scan of their popcounts places every chosen key.
+  const int wpt = (nw + kSelThreads - 1) / kSelThreads;
+  const int w0 = min(nw, tid * wpt), w1 = min(nw, w0 + wpt);
+  int n_gt = 0, n_eq = 0;
+  for (int w = w0; w < w1; ++w) {
+    n_gt += __popc(s_gtw[w]);
+    n_eq += __popc(s_eqw[w]);
+  }
+  int gt_run, eq_run, tot_gt, tot_eq;
+  block_scan2(n_gt, n_eq, &gt_run, &eq_run, &tot_gt, &tot_eq, s_scan);
+
+  const int tok0 = g * S;
+  // the bit of each word whose token starts a CSR block
+  const int rb = (kBlockTok - tok0 % kBlockTok) % kBlockTok;
+  int32_t* out_idx = idx + (int64_t)e * Ce + (int64_t)g * C;
+  float* out_gate = gate + (int64_t)e * Ce + (int64_t)g * C;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t gw = s_gtw[w], qw = s_eqw[w];
+    if (bnd != nullptr && 32 * w + rb < S) {
+      const uint32_t m = (1u << rb) - 1u;
+      const int before = gt_run + __popc(gw & m) + min(eq_run + __popc(qw & m), k);
+      bnd[(int64_t)((tok0 + 32 * w + rb) / kBlockTok) * E + e] = g * C + before;
+    }
+    for (uint32_t bits = gw | qw; bits != 0u; bits &= bits - 1u) {
+      const int b = __ffs(bits) - 1;
+      const uint32_t m = (1u << b) - 1u;
+      const int gt_before = gt_run + __popc(gw & m);
+      const int eq_before = eq_run + __popc(qw & m);
+      const int pos = gt_before + min(eq_before, k);
+      if ((((gw >> b) & 1u) != 0u || eq_before < k) && pos < C) {
+        out_idx[pos] = tok0 + 32 * w + b;
+        out_gate[pos] = __uint_as_float(keys[32 * w + b]);
+      }
+    }
+    gt_run += __popc(gw);
+    eq_run += __popc(qw);
+  }
+  if (tid == 0) {
+    if (bnd != nullptr && g == (int)gridDim.y - 1)
+      bnd[((Tn + kBlockTok - 1) / kBlockTok) * E + e] = Ce;
+    if (tot_gt + min(tot_eq, k) != C) atomicOr(err, kErrDeviceCheck);
+  }
 }
 
-constexpr int kCsrTok = 32;
 constexpr int kCsrThreads = 256;
+constexpr int kCsrWarps = kCsrThreads / 32;
+static_assert(kCsrThreads >= 256, "one thread per expert (E <= 256)");
 
 __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
   int lo = 0, hi = n;
@@ -188,91 +332,127 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
 }
 
 __global__ void __launch_bounds__(kCsrThreads)
-csr_kernel(const int32_t* __restrict__ idx, int Tn, int E, int Ce, int32_t* __restrict__ tok_ptr,
-           int32_t* __restrict__ tok_ent, int32_t* __restrict__ ent_pos, float* __restrict__ gate,
-           int normalize, float route_scale, unsigned* __restrict__ err) {
+csr_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ bnd, int Tn, int E,
+           int Ce, int32_t* __restrict__ tok_ptr, int32_t* __restrict__ tok_ent,
+           int32_t* __restrict__ ent_pos, float* __restrict__ gate, int normalize,
+           float route_scale, unsigned* __restrict__ err) {
   pdl_launch_dependents();
-  pdl_wait();
-  extern __shared__ int s_slot[];  // [kCsrTok][E]: slot of (token, expert) or -1
-  __shared__ int s_lo[256], s_hi[256];
-  __shared__ int s_base_part[kCsrThreads / 32];
-  __shared__ int s_cnt[kCsrTok], s_off[kCsrTok];
+  extern __shared__ int s_slot[];  // [kBlockTok][E]: slot of (token, expert) or -1
+  __shared__ int s_lo[256], s_beg[256];
+  __shared__ int s_wlo[kCsrWarps], s_wcnt[kCsrWarps];
+  __shared__ int s_cnt[kBlockTok], s_off[kBlockTok];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = blockIdx.x * kCsrTok;
-  const int t1 = min(Tn, t0 + kCsrTok);
+  const int blk = blockIdx.x;
+  const int t0 = blk * kBlockTok;
+  const int t1 = min(Tn, t0 + kBlockTok);
 
-  for (int i = tid; i < kCsrTok * E; i += kCsrThreads) s_slot[i] = -1;
-  int part = 0;
-  for (int e = tid; e < E; e += kCsrThreads) {
-    const int32_t* row = idx + (int64_t)e * Ce;
-    int lo = lower_bound_i32(row, Ce, t0);
-    int hi = lower_bound_i32(row, Ce, t1);
-    s_lo[e] = lo;
-    s_hi[e] = hi;
-    part += lo;
+  for (int i = tid; i < kBlockTok * E; i += kCsrThreads) s_slot[i] = -1;
+  if (tid < kBlockTok) s_cnt[tid] = 0;
+  pdl_wait();
+
+  // slot range [lo, lo + cnt) of expert `tid` inside the block
+  int lo = 0, cnt = 0;
+  if (tid < E) {
+    if (bnd != nullptr) {
+      lo = bnd[(int64_t)blk * E + tid];
+      cnt = bnd[(int64_t)(blk + 1) * E + tid] - lo;
+    } else {
+      const int32_t* row = idx + (int64_t)tid * Ce;
+      lo = lower_bound_i32(row, Ce, t0);
+      cnt = lower_bound_i32(row, Ce, t1) - lo;
+    }
+    if (lo < 0 || cnt < 0 || lo + cnt > Ce) {  // not a table the selection wrote
+      atomicOr(err, kErrDeviceCheck);
+      lo = 0;
+      cnt = 0;
+    }
+    s_lo[tid] = lo;
   }
+  // exclusive scan of cnt over the experts; sum of lo = entries before the block
+  int inc = cnt, part = lo;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  if (lane == 0) s_base_part[warp] = part;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
+    part += __shfl_xor_sync(0xffffffffu, part, o);
+  }
+  if (lane == 31) s_wcnt[warp] = inc;
+  if (lane == 0) s_wlo[warp] = part;
   __syncthreads();
-  int base = 0;
+  int base = 0, total = 0, before = 0;
 #pragma unroll
-  for (int w = 0; w < kCsrThreads / 32; ++w) base += s_base_part[w];
+  for (int w = 0; w < kCsrWarps; ++w) {
+    base += s_wlo[w];
+    total += s_wcnt[w];
+    if (w < warp) before += s_wcnt[w];
+  }
+  if (tid < E) s_beg[tid] = before + inc - cnt;
+  __syncthreads();
 
-  // scatter this block's entries into the (token, expert) slot map
-  for (int e = warp; e < E; e += kCsrThreads / 32) {
-    const int32_t* row = idx + (int64_t)e * Ce;
-    for (int s = s_lo[e] + lane; s < s_hi[e]; s += 32) {
-      int t = row[s];
-      if (t >= t0 && t < t1) s_slot[(t - t0) * E + e] = s;
-      else atomicOr(err, kErrDeviceCheck);
+  // scatter the block's entries into the (token, expert) slot map, one per thread
+  for (int j = tid; j < total; j += kCsrThreads) {
+    int a = 0, b = E - 1;  // last expert whose first flat entry is <= j
+    while (a < b) {
+      const int mid = (a + b + 1) >> 1;
+      if (s_beg[mid] <= j) a = mid; else b = mid - 1;
+    }
+    const int sl = s_lo[a] + (j - s_beg[a]);
+    const int t = idx[(int64_t)a * Ce + sl];
+    if (t >= t0 && t < t1) {
+      s_slot[(t - t0) * E + a] = sl;
+      atomicAdd(&s_cnt[t - t0], 1);
+    } else {
+      atomicOr(err, kErrDeviceCheck);
     }
   }
   __syncthreads();
 
-  // per-token counts and their exclusive scan (one warp: kCsrTok == 32)
+  // per-token offsets (one warp: kBlockTok == 32)
   if (warp == 0) {
-    int c = 0;
-    if (t0 + lane < t1)
-      for (int e = 0; e < E; ++e) c += s_slot[lane * E + e] >= 0;
-    int inc = c;
+    const int c = s_cnt[lane];
+    int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int v = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += v;
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
-    s_cnt[lane] = c;
-    s_off[lane] = inc - c;
-    if (t0 + lane < t1) tok_ptr[t0 + lane] = base + inc - c;
-    if (t0 + lane == Tn - 1) tok_ptr[Tn] = base + inc;
+    s_off[lane] = incl - c;
+    if (t0 + lane < t1) tok_ptr[t0 + lane] = base + incl - c;
+    if (t0 + lane == Tn - 1) tok_ptr[Tn] = base + incl;
   }
   __syncthreads();
 
   // entries of each token in ascending expert order: one warp per token
-  for (int r = warp; r < t1 - t0; r += kCsrThreads / 32) {
+  const unsigned lt = lanemask_lt();
+  for (int r = warp; r < t1 - t0; r += kCsrWarps) {
     int out = base + s_off[r];
     const int* srow = s_slot + r * E;
+    float tot = 0.f;  // the token's gates summed in ascending expert order, fp32
     for (int e0 = 0; e0 < E; e0 += 32) {
-      int e = e0 + lane;
-      int sl = e < E ? srow[e] : -1;
-      unsigned m = __ballot_sync(0xffffffffu, sl >= 0);
+      const int e = e0 + lane;
+      const int sl = e < E ? srow[e] : -1;
+      const unsigned m = __ballot_sync(0xffffffffu, sl >= 0);
       if (sl >= 0) {
-        const int at = out + __popc(m & ((1u << lane) - 1u));
+        const int at = out + __popc(m & lt);
         tok_ent[at] = e * Ce + sl;
         if (ent_pos != nullptr) ent_pos[e * Ce + sl] = at;
+      }
+      if (normalize) {
+        const float v = sl >= 0 ? gate[(int64_t)e * Ce + sl] : 0.f;
+        for (unsigned mm = m; mm != 0u; mm &= mm - 1u)
+          tot += __shfl_sync(0xffffffffu, v, __ffs(mm) - 1);
       }
       out += __popc(m);
     }
     if (normalize) {
-      __syncwarp();
-      // fixed order: ascending expert, fp32
-      float tot = 0.f;
-      int beg = base + s_off[r], n = s_cnt[r];
-      for (int j = 0; j < n; ++j) tot += gate[tok_ent[beg + j]];
-      __syncwarp();  // every lane has read the raw gates before any is overwritten
-      for (int j = lane; j < n; j += 32) {
-        int v = tok_ent[beg + j];
-        gate[v] = route_scale * (gate[v] / tot);
+      // every entry belongs to one token, so this lane alone reads and rewrites it
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const int sl = e < E ? srow[e] : -1;
+        if (sl >= 0) {
+          float* gp = gate + (int64_t)e * Ce + sl;
+          *gp = route_scale * (*gp / tot);
+        }
       }
     }
   }
@@ -280,22 +460,28 @@ csr_kernel(const int32_t* __restrict__ idx, int Tn, int E, int Ce, int32_t* __re
 
 }  // namespace
 
-cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, float* gate,
-                          unsigned* err, cudaStream_t st) {
-  int cached = s.S <= kSelMaxCached;
-  size_t smem = cached ? sizeof(uint32_t) * (size_t)s.S : 0;
-  dim3 grid((unsigned)s.E, (unsigned)s.n_seg);
-  return launch_kernel(select_kernel, grid, dim3(kSelThreads), smem, st, s.pdl, 1, scores_t,
-                       (int64_t)s.T, s.S, s.C, s.Ce, cached, idx, gate, err);
+size_t select_bound_entries(const Shape& s) {
+  return ((size_t)ceil_div(s.T, kBlockTok) + 1) * (size_t)s.E;
 }
 
-cudaError_t launch_csr(const int32_t* idx, const Shape& s, int32_t* tok_ptr, int32_t* tok_ent,
-                       int32_t* ent_pos, float* gate, nmoe_combine combine, float route_scale,
-                       unsigned* err, cudaStream_t st) {
-  size_t smem = sizeof(int) * (size_t)kCsrTok * s.E;
-  dim3 grid((unsigned)ceil_div(s.T, kCsrTok));
-  return launch_kernel(csr_kernel, grid, dim3(kCsrThreads), smem, st, s.pdl, 1, idx, s.T, s.E,
-                       s.Ce, tok_ptr, tok_ent, ent_pos, gate,
+cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, float* gate,
+                          int32_t* bnd, unsigned* err, cudaStream_t st) {
+  if (s.S > kSelectMaxRow) return cudaErrorInvalidValue;
+  const int cached = s.S <= kSelMaxCached;
+  const size_t nw4 = (size_t)((ceil_div(s.S, 32) + 3) & ~3);
+  const size_t smem = sizeof(uint32_t) * ((cached ? (size_t)((s.S + 3) & ~3) : 0) + 2 * nw4);
+  dim3 grid((unsigned)s.E, (unsigned)s.n_seg);
+  return launch_kernel(select_kernel, grid, dim3(kSelThreads), smem, st, s.pdl, 1, scores_t,
+                       (int64_t)s.T, s.S, s.C, s.Ce, s.E, cached, idx, gate, bnd, err);
+}
+
+cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, int32_t* tok_ptr,
+                       int32_t* tok_ent, int32_t* ent_pos, float* gate, nmoe_combine combine,
+                       float route_scale, unsigned* err, cudaStream_t st) {
+  size_t smem = sizeof(int) * (size_t)kBlockTok * s.E;
+  dim3 grid((unsigned)ceil_div(s.T, kBlockTok));
+  return launch_kernel(csr_kernel, grid, dim3(kCsrThreads), smem, st, s.pdl, 1, idx, bnd, s.T,
+                       s.E, s.Ce, tok_ptr, tok_ent, ent_pos, gate,
                        (int)(combine == NMOE_COMBINE_NORMALIZED), route_scale, err);
 }
 

@@ -26,7 +26,9 @@
  *     reported by nmoe_get_last_error().
  *   - No CPU fallback exists: every step runs in this library's CUDA kernels.
  *   - Sizes: 1 <= E <= 256, 1 <= C <= T / n_segments, T < 2^31, E * n_segments * C
- *     < 2^31, d and F multiples of 8.
+ *     < 2^31, d and F multiples of 8 (else NMOE_ERR_INVALID_ARG or, for the multiples,
+ *     NMOE_ERR_UNSUPPORTED). T / n_segments <= 2^19 tokens per segment
+ *     (NMOE_ERR_UNSUPPORTED above: the selection keeps a segment's bitmaps on chip).
  */
 #ifndef NMOE_H_
 #define NMOE_H_

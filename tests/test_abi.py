@@ -51,7 +51,7 @@ FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced (checks
 @pytest.mark.parametrize("args,expect", [
     (dict(T=0), 1), (dict(E=0), 1), (dict(E=257), 1), (dict(C=0), 1), (dict(C=65), 1),
     (dict(d=12), 2), (dict(F=20), 2), (dict(x=0), 1), (dict(x=FAKE + 8), 1),
-    (dict(out=FAKE), 1),
+    (dict(out=FAKE), 1), (dict(T=(1 << 19) + 64, C=8), 2),
 ])
 def test_forward_rejects_bad_arguments_on_host(args, expect):
     a = dict(x=FAKE, W_r=FAKE + 4096, W1=FAKE + 8192, W3=FAKE + 12288, W2=FAKE + 16384,
@@ -83,7 +83,9 @@ def test_workspace_size_accounts_for_every_buffer():
     n = nm.workspace_size(T, d, E, F, C_)
     Ce = E * C_
     # default (split) intermediates: H as a bf16 hi/lo pair, Y in fp32 -> 4 bytes each
-    minimum = 4 * T * E * 2 + 4 * Ce * 4 + 4 * (T + 1) + 4 * Ce * F + 4 * Ce * d
+    blocks = (T + 31) // 32 + 1  # per-expert boundary table of the CSR build
+    minimum = (4 * T * E * 2 + 4 * Ce * 4 + 4 * blocks * E + 4 * (T + 1) + 4 * Ce * F
+               + 4 * Ce * d)
     assert minimum <= n <= minimum + 16 * 256
     small = nm.workspace_size(T, d, E, F, C_, intermediate="bf16")
     assert small == n - 2 * Ce * F - 2 * Ce * d

@@ -1,0 +1,74 @@
+"""bench.py's multi-rank path on the CPU: two gloo ranks started the way torchrun starts
+them (RANK / WORLD_SIZE / MASTER_ADDR / MASTER_PORT in the environment)."""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parents[1]
+sys.path.insert(0, str(ROOT))
+import bench  # noqa: E402
+
+_RANK = """
+import datetime, json, os, sys
+sys.path.insert(0, sys.argv[1])
+import torch.distributed as dist
+import bench
+rank = int(os.environ["RANK"])
+dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+# rank-dependent timings: the job is as slow as its slowest rank, per quantity
+mine = [10.0 + 2.0 * rank, 30.0 - rank, 5.0]
+got = bench.max_over_ranks(mine, dist, "cpu")
+dist.barrier()
+dist.destroy_process_group()
+print(json.dumps({"rank": rank, "got": got}))
+"""
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_two_gloo_ranks_take_the_max_of_every_timing():
+    port = _free_port()
+    procs = []
+    for rank in range(2):
+        env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, "-c", _RANK, str(ROOT)], env=env,
+                                      stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                                      text=True))
+    outs = []
+    for p in procs:
+        try:
+            o, e = p.communicate(timeout=180)
+        except subprocess.TimeoutExpired:
+            for q in procs:
+                q.kill()
+            pytest.fail("a gloo rank did not finish")
+        assert p.returncode == 0, e[-2000:]
+        outs.append(json.loads(o.strip().splitlines()[-1]))
+    for r in outs:
+        assert r["got"] == [12.0, 30.0, 5.0]
+
+
+def test_replica_throughput_counts_every_rank_over_the_slowest_time():
+    # 2 ranks x 10 steps x 8192 tokens in 12 ms (the slowest rank)
+    assert bench.replica_throughput(8192, 2, 10, 12.0) == pytest.approx(8192 * 20 / 0.012)
+    assert bench.max_over_ranks([1.5, 2], None, "cpu") == [1.5, 2.0]
+
+
+def test_reference_arm_on_a_non_zero_rank_exits_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""

@@ -150,6 +150,13 @@ def test_routing_options_match_oracle(opts, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_segments_not_aligned_to_token_blocks(dtype):
+    # 3 segments of 100 tokens: segment edges fall inside the CSR's 32-token blocks
+    a = I.make_small(300, 136, 6, 104, dtype, seed=23)
+    _full_parity(a, 20, dtype, dict(n_segments=3))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_router_bias_matches_oracle(dtype):
     a = I.make_small(192, 64, 6, 64, dtype, seed=22)
     bias = torch.randn(3, 6, generator=torch.Generator().manual_seed(5))
@@ -224,6 +231,29 @@ def test_select_edge_sizes(T, E, C_, nseg):
     ptr, ent = O.token_lists(want, T)
     assert np.array_equal(tok_ptr.cpu().numpy(), ptr)
     assert np.array_equal(tok_ent.cpu().numpy(), ent)
+
+
+_FRESH_SELECT = """
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import diffusion_transformer_moe_b200 as nm
+from oracle import nmoe_oracle as O
+p = torch.rand(8192, 4, generator=torch.Generator().manual_seed(3))
+idx, _, _, _ = nm.select(p.t().contiguous().cuda(), 128)
+torch.cuda.synchronize()
+assert np.array_equal(idx.cpu().numpy(), O.select(p.numpy(), 128))
+"""
+
+
+def test_first_large_row_select_in_a_fresh_process():
+    # the first selection of a process, with a row that needs its shared-memory opt-in
+    import subprocess
+    import sys
+    from pathlib import Path
+    root = str(Path(__file__).resolve().parents[1])
+    r = subprocess.run([sys.executable, "-c", _FRESH_SELECT, root], capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
 
 
 def test_nan_scores_raise_the_device_check():
