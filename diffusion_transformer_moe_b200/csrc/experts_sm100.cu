@@ -70,7 +70,11 @@ struct Cfg {
   static constexpr int kEpiWarp0 = 2 + kAWarps;
   static constexpr int kThreads = 32 * (2 + kAWarps + kEpiWarps);
   static constexpr int kFullCount = 1 + 32 * kAWarps;    // TMA arrive + one per gather thread
-  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
+  // staging block per epilogue warp: gemm2 with fp32 Y, 32 rows x 32 fp32; gemm1, 32
+  // rows x 32 bf16 of H (and as much again for H lo)
+  static constexpr int kEpiStage =
+      MODE == kGemm2 ? (SPLIT ? 32 * 32 * 4 : 0) : (SPLIT ? 2 * 32 * 64 : 32 * 64);
+  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + kEpiWarps * kEpiStage + 1024;
 };
 
 struct Params {
@@ -324,8 +328,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       const int64_t ent = (int64_t)e * p.Ce + (valid ? s : 0);
       const int64_t orow = (MODE == kGemm2 ? (int64_t)p.ent_pos[ent] : ent) * p.N;
       if (MODE == kGemm1) {
-        __nv_bfloat16* hi = static_cast<__nv_bfloat16*>(p.out) + orow;
-        __nv_bfloat16* lo = static_cast<__nv_bfloat16*>(p.out_lo) + orow;
+        // staging blocks of this warp, 32 rows x 64 bytes each (H, then H lo): 16-byte
+        // chunk c of row r at r * 64 + (c ^ ((r / 2) % 4)) * 16
+        uint8_t* sh = smem + kStages * C::kStageBytes + (warp - C::kEpiWarp0) * C::kEpiStage;
+        uint8_t* sl = sh + 32 * 64;
+        const int sw = (lane >> 1) & 3;
 #pragma unroll 1
         for (int j0 = 64 * half; j0 < 64 * half + 64; j0 += 32) {
           uint32_t g[32], u[32];
@@ -339,44 +346,74 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
           uint32_t ph[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) ph[i] = pack_bf16x2(h[2 * i], h[2 * i + 1]);
-          if (valid) {
+          // this row's 32 values into the staging blocks ...
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int f = n0 + j0 + 8 * v;
-              if (f < p.N) {
-                *reinterpret_cast<uint4*>(hi + f) =
-                    make_uint4(ph[4 * v], ph[4 * v + 1], ph[4 * v + 2], ph[4 * v + 3]);
-                if (SPLIT) {
-                  uint4 l;
-                  l.x = pack_lo_bf16x2(h[8 * v + 0], h[8 * v + 1], ph[4 * v + 0]);
-                  l.y = pack_lo_bf16x2(h[8 * v + 2], h[8 * v + 3], ph[4 * v + 1]);
-                  l.z = pack_lo_bf16x2(h[8 * v + 4], h[8 * v + 5], ph[4 * v + 2]);
-                  l.w = pack_lo_bf16x2(h[8 * v + 6], h[8 * v + 7], ph[4 * v + 3]);
-                  *reinterpret_cast<uint4*>(lo + f) = l;
-                }
-              }
+          for (int v = 0; v < 4; ++v) {
+            const int off = lane * 64 + ((v ^ sw) << 4);
+            *reinterpret_cast<uint4*>(sh + off) =
+                make_uint4(ph[4 * v], ph[4 * v + 1], ph[4 * v + 2], ph[4 * v + 3]);
+            if (SPLIT) {
+              uint4 l;
+              l.x = pack_lo_bf16x2(h[8 * v + 0], h[8 * v + 1], ph[4 * v + 0]);
+              l.y = pack_lo_bf16x2(h[8 * v + 2], h[8 * v + 3], ph[4 * v + 1]);
+              l.z = pack_lo_bf16x2(h[8 * v + 4], h[8 * v + 5], ph[4 * v + 2]);
+              l.w = pack_lo_bf16x2(h[8 * v + 6], h[8 * v + 7], ph[4 * v + 3]);
+              *reinterpret_cast<uint4*>(sl + off) = l;
             }
           }
+          __syncwarp();
+          // ... then out 8 rows per store, 64 contiguous bytes per row
+          const int c = lane & 3;
+          const int f = n0 + j0 + 8 * c;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = 8 * i + (lane >> 2);
+            const int64_t ro = __shfl_sync(0xffffffffu, orow, r);
+            const int rv = __shfl_sync(0xffffffffu, (int)valid, r);
+            const int off = r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+            if (rv && f < p.N) {
+              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ro + f) =
+                  *reinterpret_cast<const uint4*>(sh + off);
+              if (SPLIT)
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out_lo) + ro + f) =
+                    *reinterpret_cast<const uint4*>(sl + off);
+            }
+          }
+          __syncwarp();  // the blocks are read before the next chunk overwrites them
         }
       } else {
         const float gw = valid ? p.gate[(int64_t)e * p.Ce + s] : 0.f;
+        // staging block of this warp: 16-byte chunk c of row r at r * 128 + (c ^ (r % 8)) * 16
+        float* sb = reinterpret_cast<float*>(smem + kStages * C::kStageBytes +
+                                             (warp - C::kEpiWarp0) * C::kEpiStage);
 #pragma unroll 1
         for (int j0 = 128 * half; j0 < 128 * half + 128; j0 += 32) {
           uint32_t y[32];
           tmem_ld32(taddr + j0, y);
           tmem_ld_wait();
           if (SPLIT) {
-            float* yr = static_cast<float*>(p.out) + orow;
-            if (valid) {
+            // Each thread holds one row's 32 values; written straight out, one warp store
+            // would touch 32 rows. Through the staging block, a store covers 4 rows with
+            // 128 contiguous bytes each.
 #pragma unroll
-              for (int v = 0; v < 8; ++v) {
-                const int c = n0 + j0 + 4 * v;
-                if (c < p.N)
-                  *reinterpret_cast<float4*>(yr + c) = make_float4(
-                      gw * __uint_as_float(y[4 * v]), gw * __uint_as_float(y[4 * v + 1]),
-                      gw * __uint_as_float(y[4 * v + 2]), gw * __uint_as_float(y[4 * v + 3]));
-              }
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<float4*>(sb + lane * 32 + ((c ^ (lane & 7)) << 2)) = make_float4(
+                  gw * __uint_as_float(y[4 * c]), gw * __uint_as_float(y[4 * c + 1]),
+                  gw * __uint_as_float(y[4 * c + 2]), gw * __uint_as_float(y[4 * c + 3]));
+            __syncwarp();
+            const int c = lane & 7;
+            const int col = n0 + j0 + 4 * c;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = 4 * i + (lane >> 3);
+              const int64_t ro = __shfl_sync(0xffffffffu, orow, r);
+              const int rv = __shfl_sync(0xffffffffu, (int)valid, r);
+              const float4 v =
+                  *reinterpret_cast<const float4*>(sb + r * 32 + ((c ^ (r & 7)) << 2));
+              if (rv && col < p.N)
+                *reinterpret_cast<float4*>(static_cast<float*>(p.out) + ro + col) = v;
             }
+            __syncwarp();  // the block is read before the next chunk overwrites it
           } else {
             __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.out) + orow;
             uint32_t h[16];

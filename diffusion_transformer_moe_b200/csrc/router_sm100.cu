@@ -6,9 +6,12 @@
 // Precision: the scores must match an fp64 reference to 1e-5 relative, and with
 // LogNormal-scaled tokens the logits reach |l| ~ 30, where a single fp32 accumulator
 // over d = 2048 drifts by more than that (tensor-core accumulation also truncates). So
-// the MMAs accumulate only one 64-long k-chunk per TMEM slice, and the epilogue warps
-// read every chunk back with tcgen05.ld (two chunks per round trip) and add it to
-// Kahan-compensated fp32 running sums, taken in fp64 at the end. Max, exp and the normalisation run in fp64; each
+// the MMAs accumulate only one 128-long k-chunk (two k-blocks) per TMEM slice, and the
+// epilogue warps read every chunk back with tcgen05.ld (two chunks per round trip) and
+// add it to Kahan-compensated fp32 running sums, taken in fp64 at the end. (Modelled on
+// the 1024 px workload with round-toward-zero accumulation, 128-long chunks keep the
+// scores within ~3e-6 of fp64, 256-long ones ~8e-6; 64-long ones took twice the
+// read-back round trips, which bound the kernel.) Max, exp and the normalisation run in fp64; each
 // score is rounded once to fp32.
 //
 // Each 128-token tile is split along d between the two CTAs of a cluster (so T = 8192
@@ -41,6 +44,7 @@ constexpr int kABytes = kBM * kBK * 2;     // 16 KB
 constexpr int kBBoxBytes = 64 * kBK * 2;   // 8 KB: 64 experts x 64 k
 constexpr int kMaxE = 128;
 constexpr int kSplit = 2;   // CTAs per token tile (one cluster), each owning half of d
+constexpr int kChunkKB = 2; // k-blocks accumulated per TMEM chunk slice (128-long chunks)
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint64_t kDrainNs = 20000000ull;
 
@@ -90,6 +94,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
   const int nk_all = (p.d + kBK - 1) / kBK;
   const int kb0 = rank == 0 ? 0 : (nk_all + 1) / 2;
   const int nk = rank == 0 ? (nk_all + 1) / 2 : nk_all - (nk_all + 1) / 2;
+  const int nch = (nk + kChunkKB - 1) / kChunkKB;  // chunk slices this CTA fills
   const int t0 = (blockIdx.x / kSplit) * kBM;
 
   if (threadIdx.x == 0) {
@@ -139,7 +144,9 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       int stage = 0, buf = 0;
       uint32_t phase = 0, buf_phase = 0;
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait(&tempty_bar[buf], buf_phase ^ 1, abort_v, kWaitNs)) break;
+        const bool first = kb % kChunkKB == 0;
+        const bool last = kb % kChunkKB == kChunkKB - 1 || kb == nk - 1;
+        if (first && !mbar_wait(&tempty_bar[buf], buf_phase ^ 1, abort_v, kWaitNs)) break;
         if (!mbar_wait(&full_bar[stage], phase, abort_v, kWaitNs)) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sA + stage * kABytes);
@@ -149,13 +156,15 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, kBBoxBytes, 1024);
-          // one chunk slice per k-block, restarted at the block's first MMA
-          mma_bf16(d0, ad, bd, idesc, kk != 0);
+          // one chunk slice per kChunkKB k-blocks, restarted at the chunk's first MMA
+          mma_bf16(d0, ad, bd, idesc, !(first && kk == 0));
         }
         mma_commit(&empty_bar[stage]);
-        mma_commit(&tfull_bar[buf]);
         if (++stage == kStages) { stage = 0; phase ^= 1; }
-        if (++buf == p.nbuf) { buf = 0; buf_phase ^= 1; }
+        if (last) {
+          mma_commit(&tfull_bar[buf]);
+          if (++buf == p.nbuf) { buf = 0; buf_phase ^= 1; }
+        }
       }
       mma_commit(&drain_bar);
       int dummy = 0;
@@ -167,7 +176,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
     const int g = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const int e0 = g * CW;
-    // Kahan-compensated fp32 sums of the 32-long chunk sums: hi accumulates, lo keeps
+    // Kahan-compensated fp32 sums of the chunk sums: hi accumulates, lo keeps
     // what each addition rounded away (error ~2 ulp of the total, however many chunks);
     // hi + lo is taken in fp64 once at the end.
     float hi[CW], lo[CW];
@@ -176,9 +185,9 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
     int buf = 0;
     uint32_t buf_phase = 0;
     bool ok = true;
-    // two k-blocks (two chunk slices) per TMEM-load round trip
-    for (int kb = 0; kb < nk; kb += 2) {
-      const bool two = kb + 1 < nk;
+    // two chunk slices per TMEM-load round trip
+    for (int ch = 0; ch < nch; ch += 2) {
+      const bool two = ch + 1 < nch;
       int w = 1;
       if (lane == 0) {
         w = mbar_wait(&tfull_bar[buf], buf_phase, abort_v, kWaitNs);
@@ -203,7 +212,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          // the k-blocks' two 64-long chunk sums (one rounding), then Kahan
+          // the round's two chunk sums (one rounding), then Kahan
           const float c = two ? __uint_as_float(c0[j]) + __uint_as_float(c1[j])
                               : __uint_as_float(c0[j]);
           const float y = c - lo[h * 16 + j];
