@@ -82,6 +82,9 @@ struct Params {
   int K;           // reduction length (d for gemm1, F for gemm2)
   int N;           // output row length (F for gemm1, d for gemm2)
   int tiles_m, tiles_n, num_tiles;
+  // Work items: tiles [0, num_full) whole, then every remaining tile as two items, each
+  // half of its N range (so a last, partial wave of tiles runs on twice the SMs).
+  int num_full, num_items;
   const int32_t* idx;    // gemm1: chosen tokens [E, Ce]
   const float* gate;     // gemm2: combine weights [E, Ce]
   const int32_t* ent_pos;  // gemm2: Y row of entry e*Ce + s (token-major order)
@@ -95,6 +98,29 @@ struct Params {
 // GEMM output; very negative g gives 0 and g -> +inf gives g.
 __device__ __forceinline__ float silu_f32(float g) {
   return __fdividef(g, 1.f + __expf(-g));
+}
+
+// Work item -> tile: expert, first row, first column of its N range, and whether it
+// covers half of the tile's N range. n_per_tile: gemm1 128 columns of F (gate and up
+// each), gemm2 256 columns of d.
+struct Tile {
+  int e, m0, n0;
+  bool half;
+};
+__device__ __forceinline__ Tile tile_of(int item, const Params& p, int n_per_tile) {
+  int t = item, part = -1;
+  if (item >= p.num_full) {
+    t = p.num_full + ((item - p.num_full) >> 1);
+    part = (item - p.num_full) & 1;
+  }
+  Tile r;
+  r.e = t / (p.tiles_m * p.tiles_n);
+  const int rem = t % (p.tiles_m * p.tiles_n);
+  r.m0 = (rem / p.tiles_n) * kBM;
+  r.n0 = (rem % p.tiles_n) * n_per_tile;
+  r.half = part >= 0;
+  if (r.half) r.n0 += part * (n_per_tile / 2);
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -163,11 +189,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // per stage: ever issued / parity of last issue
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const int e = tile / (p.tiles_m * p.tiles_n);
-      const int rem = tile % (p.tiles_m * p.tiles_n);
-      const int m0 = (rem / p.tiles_n) * kBM;
-      const int n0 = (rem % p.tiles_n) * n_per_tile;
+    for (int item = blockIdx.x; item < p.num_items; item += gridDim.x) {
+      const Tile tl = tile_of(item, p, n_per_tile);
+      const int e = tl.e, m0 = tl.m0, n0 = tl.n0;
+      const int nbox = tl.half ? 2 : 4;  // 64-column boxes of B
+      const uint32_t b_bytes = (uint32_t)(nbox * kBBoxBytes);
       int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
       if (MODE == kGemm1 && !C::kLsuA) {
         const int32_t* ir = p.idx + (int64_t)e * p.Ce;
@@ -185,7 +211,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         if (!ok) break;
         if (lane == 0)
           mbar_arrive_expect_tx(&full_bar[stage],
-                                C::kLsuA ? (uint32_t)kBBytes : (uint32_t)C::kStageBytes);
+                                C::kLsuA ? b_bytes : C::kATiles * kABytes + b_bytes);
         __syncwarp();
         const int k0 = kb * kBK;
         uint8_t* b_dst = b_tile(stage);
@@ -193,9 +219,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
           if (!C::kLsuA)
             tma_gather4(a_tile(stage, 0) + lane * 512, &map_a, &full_bar[stage], k0, r0, r1,
                         r2, r3);
-          if (lane < 4) {
-            const CUtensorMap* mb = lane < 2 ? &map_b0 : &map_b1;
-            tma_load_3d(b_dst + lane * kBBoxBytes, mb, &full_bar[stage], n0 + 64 * (lane & 1),
+          // boxes: gate columns, then up columns (two of each, or one of each for a half)
+          if (lane < nbox) {
+            const int per = nbox / 2;
+            const CUtensorMap* mb = lane < per ? &map_b0 : &map_b1;
+            tma_load_3d(b_dst + lane * kBBoxBytes, mb, &full_bar[stage], n0 + 64 * (lane % per),
                         k0, e);
           }
         } else {
@@ -203,7 +231,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
             tma_load_2d(a_tile(stage, 0), &map_a, &full_bar[stage], k0, e * p.Ce + m0);
           if (C::kATiles == 2 && lane == 1)
             tma_load_2d(a_tile(stage, 1), &map_a2, &full_bar[stage], k0, e * p.Ce + m0);
-          if (lane < 4)
+          if (lane < nbox)
             tma_load_3d(b_dst + lane * kBBoxBytes, &map_b0, &full_bar[stage], n0 + 64 * lane,
                         k0, e);
         }
@@ -233,10 +261,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-      const int e = tile / (p.tiles_m * p.tiles_n);
-      const int rem = tile % (p.tiles_m * p.tiles_n);
-      const int m0 = (rem / p.tiles_n) * kBM;
+    for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+      const Tile tl = tile_of(item, p, n_per_tile);
+      const int e = tl.e, m0 = tl.m0;
       const __nv_bfloat16* src[8];
       uint32_t dst_off[8];
 #pragma unroll
@@ -271,11 +298,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
   } else if (warp == 1) {
     // ---------------- MMA issuer (one thread) ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kBM, 256, 1);
+      constexpr uint32_t idesc_full = idesc_bf16(kBM, 256, 1);
+      constexpr uint32_t idesc_half = idesc_bf16(kBM, 128, 1);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+        const uint32_t idesc = tile_of(item, p, n_per_tile).half ? idesc_half : idesc_full;
         if (!(ok = mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_v, kWaitNs))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
@@ -313,11 +342,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     const int row = q * 32 + lane;                  // accumulator row = tile row
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const int e = tile / (p.tiles_m * p.tiles_n);
-      const int rem = tile % (p.tiles_m * p.tiles_n);
-      const int m0 = (rem / p.tiles_n) * kBM;
-      const int n0 = (rem % p.tiles_n) * n_per_tile;
+    for (int item = blockIdx.x; item < p.num_items; item += gridDim.x) {
+      const Tile tl = tile_of(item, p, n_per_tile);
+      const int e = tl.e, m0 = tl.m0, n0 = tl.n0;
+      // accumulator columns this warp drains: [c_lo, c_lo + c_n) (gemm1: gate columns,
+      // the matching up columns sit `up` further on)
+      const int acc_n = tl.half ? 128 : 256;
+      const int up = acc_n / 2;
+      const int c_n = MODE == kGemm1 ? acc_n / 4 : acc_n / 2;
+      const int c_lo = half * c_n;
       int w = 1;
       if (lane == 0) w = mbar_wait(&tfull_bar[acc], acc_phase, abort_v, kWaitNs);
       if (__shfl_sync(0xffffffffu, w, 0) == 0) break;
@@ -334,10 +367,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         uint8_t* sl = sh + 32 * 64;
         const int sw = (lane >> 1) & 3;
 #pragma unroll 1
-        for (int j0 = 64 * half; j0 < 64 * half + 64; j0 += 32) {
+        for (int j0 = c_lo; j0 < c_lo + c_n; j0 += 32) {
           uint32_t g[32], u[32];
           tmem_ld32(taddr + j0, g);
-          tmem_ld32(taddr + 128 + j0, u);
+          tmem_ld32(taddr + up + j0, u);
           tmem_ld_wait();
           float h[32];
 #pragma unroll
@@ -387,7 +420,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         float* sb = reinterpret_cast<float*>(smem + kStages * C::kStageBytes +
                                              (warp - C::kEpiWarp0) * C::kEpiStage);
 #pragma unroll 1
-        for (int j0 = 128 * half; j0 < 128 * half + 128; j0 += 32) {
+        for (int j0 = c_lo; j0 < c_lo + c_n; j0 += 32) {
           uint32_t y[32];
           tmem_ld32(taddr + j0, y);
           tmem_ld_wait();
@@ -493,12 +526,22 @@ bool rows_map(CUtensorMap* m, const void* base, int64_t rows, int cols, uint32_t
   return make_map(m, base, 2, dims, strides, box);
 }
 
+// With one persistent CTA per SM, the last wave of tiles is partial. When it fills at
+// most half of the SMs, its tiles run as two half-width items each, so that wave takes
+// half as long on up to twice the SMs.
+void split_tail(Params& p, int sm_count) {
+  const int r = p.num_tiles % sm_count;
+  p.num_full = p.num_tiles;
+  if (r > 0 && 2 * r <= sm_count) p.num_full = p.num_tiles - r;
+  p.num_items = p.num_full + 2 * (p.num_tiles - p.num_full);
+}
+
 template <int MODE, bool SPLIT, int GATHER>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b0,
                    const CUtensorMap& b1, const __nv_bfloat16* x, const Params& p,
                    int sm_count, cudaStream_t st, bool pdl) {
   using C = Cfg<MODE, SPLIT, GATHER>;
-  const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
+  const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   return launch_kernel(grouped_gemm_kernel<MODE, SPLIT, GATHER>, dim3(grid), dim3(C::kThreads),
                        C::kSmem, st, pdl, 1, a, a2, b0, b1, x, p);
 }
@@ -523,6 +566,7 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
   p.tiles_m = (int)ceil_div(s.Ce, kBM);
   p.tiles_n = (int)ceil_div(s.F, 128);
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
+  split_tail(p, sm_count);
   p.idx = idx; p.gate = nullptr; p.ent_pos = nullptr; p.out = H_hi; p.out_lo = H_lo;
   p.err = err;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
@@ -547,6 +591,7 @@ cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* 
   p.tiles_m = (int)ceil_div(s.Ce, kBM);
   p.tiles_n = (int)ceil_div(s.d, 256);
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
+  split_tail(p, sm_count);
   p.idx = nullptr; p.gate = gate; p.ent_pos = ent_pos; p.out = Y; p.out_lo = nullptr;
   p.err = err;
   return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl)
