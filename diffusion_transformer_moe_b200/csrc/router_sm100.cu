@@ -8,21 +8,21 @@
 // over d = 2048 drifts by more than that (tensor-core accumulation also truncates). So
 // the MMAs accumulate only one 128-long k-chunk (two k-blocks) per TMEM slice, and the
 // epilogue warps read every chunk back with tcgen05.ld (two chunks per round trip) and
-// add it to Kahan-compensated fp32 running sums, taken in fp64 at the end. (Modelled on
-// the 1024 px workload with round-toward-zero accumulation, 128-long chunks keep the
-// scores within ~3e-6 of fp64, 256-long ones ~8e-6; 64-long ones took twice the
-// read-back round trips, which bound the kernel.) Max, exp and the normalisation run in fp64; each
-// score is rounded once to fp32.
+// add it to Kahan-compensated fp32 running sums. (Modelled on the 1024 px workload with
+// round-toward-zero accumulation, 128-long chunks keep the scores within ~3e-6 of fp64,
+// 256-long ones ~8e-6; 64-long ones took twice the read-back round trips.) From there
+// each logit is an unevaluated pair of fp32 numbers h + l, and the score function works
+// on the pairs: two-sum for every shift, exp(h + l) = exp(h) (1 + l), compensated sums,
+// one fp32 division (relative error a few 1e-7).
 //
 // Each 128-token tile is split along d between the two CTAs of a cluster (so T = 8192
 // fills 128 SMs, not 64). In each CTA, warp 0 streams x and W_r tiles with TMA into a
 // 6-stage ring; warp 1 (one thread) issues tcgen05.mma (M = 128, N = E rounded up to
-// 64, K = 16) into a ring of TMEM chunk buffers; 4*G epilogue warps (G = ceil(E/32))
-// each own 32 tokens x 32 experts and keep fp64 sums. The second CTA then adds its sums
-// into the first CTA's shared memory (distributed shared memory, no global traffic),
-// and the first CTA applies the score function and writes both score layouts. exp runs
-// in fp32 on the high part of the fp64 argument, corrected to first order by the low
-// part (relative error ~3e-7); every wait is bounded.
+// 64, K = 16) into a ring of TMEM chunk buffers; 4*G epilogue warps (G = ceil(E/CW))
+// each own 32 tokens x CW experts. Then each CTA sends its sums for the partner's half
+// of the tokens to the partner's shared memory (distributed shared memory, no global
+// traffic), and each finishes the score function and both score layouts for its 64
+// tokens. Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <cooperative_groups.h>
@@ -60,13 +60,12 @@ struct Params {
   unsigned* err;
 };
 
-// exp(a) for an fp64 argument: fp32 exp of the high part times (1 + low part). The low
-// part is below 2^-24 |a|, so dropping its square leaves ~1e-11; expf adds ~2 ulp.
-// Arguments beyond the fp32 exp range use the fp64 exp.
-__device__ __forceinline__ double exp_f64_arg(double a) {
-  if (a < -80.0 || a > 80.0) return exp(a);
-  const float hi = (float)a;
-  return (double)expf(hi) * (1.0 + (a - (double)hi));
+// a + b = s + e exactly (Knuth's two-sum; no operation here may be contracted or
+// reassociated, which nvcc does not do to plain adds).
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
+  s = a + b;
+  const float bb = s - a;
+  e = (a - (s - bb)) + (b - bb);
 }
 
 // Each epilogue thread owns CW experts (16 up to E = 64, else 32) of one token row;
@@ -224,85 +223,139 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       buf += 2;
       if (buf >= p.nbuf) { buf -= p.nbuf; buf_phase ^= 1; }
     }
-    double acc[CW];
+    // Each logit as an unevaluated fp32 pair h + l (l below half an ulp of h): the
+    // compensated sum hi - lo, renormalised.
+    float* h = hi;  // renormalised in place
+    float* l = lo;
 #pragma unroll
-    for (int j = 0; j < CW; ++j) acc[j] = (double)hi[j] - (double)lo[j];
-    // After the cluster barrier both CTAs' stage rings are idle. The second CTA adds its
-    // half-d sums into the first CTA's ring laid out [E][128] (a warp writes 32
-    // consecutive doubles per expert), then the first CTA finishes in registers.
-    double* part = reinterpret_cast<double*>(smem);
-    double* red = part + (size_t)kMaxE * kBM;   // [2][G][128]: row max, then row sum
-    cluster.sync();                       // (1) every ring is idle
-    // expert pair (e, e+1) of token row at part[((e / 2) * 128 + row) * 2 + (e & 1)]
-    if (rank != 0) {
-      double2* remote = reinterpret_cast<double2*>(cluster.map_shared_rank(part, 0));
-#pragma unroll
-      for (int j = 0; j < CW; j += 2)
-        if (e0 + j < p.E) remote[((e0 + j) >> 1) * kBM + row] = make_double2(acc[j], acc[j + 1]);
+    for (int j = 0; j < CW; ++j) {
+      float s_, e_;
+      two_sum(hi[j], -lo[j], s_, e_);
+      h[j] = s_;
+      l[j] = e_;
     }
-    cluster.sync();                       // (2) the second half's sums have landed
-    if (rank == 0) {
-      const int nthreads = 128 * G;
+    // Tokens 0..63 of the tile are finished by the first CTA, 64..127 by the second:
+    // each sends its half-d sums of the partner's rows to the partner's shared memory
+    // (laid out [expert][64 rows], (h, l) pairs), after the first cluster barrier has
+    // left both stage rings idle.
+    const bool mine = (q >> 1) == rank;     // this warp's rows are finished here
+    const int r64 = row & 63;
+    float2* xch = reinterpret_cast<float2*>(smem);
+    float* red_m = reinterpret_cast<float*>(xch + (size_t)kMaxE * 64);  // [G][64]
+    float2* red_z = reinterpret_cast<float2*>(red_m + 4 * 64);          // [G][64]
+    cluster.sync();                         // (1) every ring is idle
+    if (!mine) {
+      float2* remote = cluster.map_shared_rank(xch, rank ^ 1);
+#pragma unroll
+      for (int j = 0; j < CW; ++j)
+        if (e0 + j < p.E) remote[(e0 + j) * 64 + r64] = make_float2(h[j], l[j]);
+    }
+    cluster.sync();                         // (2) the partner's sums have landed
+    if (mine) {
+      const int nfin = 64 * G;               // threads finishing this CTA's 64 tokens
       const int t = t0 + row;
       const bool live = t < p.T;
-      const float* b = (p.bias != nullptr && live) ? p.bias + (int64_t)(t / p.S) * p.E : nullptr;
-      const double2* pp = reinterpret_cast<const double2*>(part);
+      const float* b =
+          (p.bias != nullptr && live) ? p.bias + (int64_t)(t / p.S) * p.E : nullptr;
 #pragma unroll
-      for (int j = 0; j < CW; j += 2) {
+      for (int j = 0; j < CW; ++j) {
         if (e0 + j < p.E) {
-          const double2 v = pp[((e0 + j) >> 1) * kBM + row];
-          acc[j] += v.x;
-          acc[j + 1] += v.y;
+          const float2 v = xch[(e0 + j) * 64 + r64];
+          float s_, e_;
+          two_sum(h[j], v.x, s_, e_);
+          two_sum(s_, e_ + (l[j] + v.y), h[j], l[j]);
+          if (b) {
+            two_sum(h[j], b[e0 + j], s_, e_);
+            two_sum(s_, e_ + l[j], h[j], l[j]);
+          }
         }
       }
-      if (b) {
-#pragma unroll
-        for (int j = 0; j < CW; ++j)
-          if (e0 + j < p.E) acc[j] += (double)b[e0 + j];
-      }
+      float pr[CW];
       if (p.score_fn == NMOE_SCORE_SOFTMAX) {
-        double m = -INFINITY;
+        // shift by the largest high part; exp(h - m + l) = exp(d) (1 + t) with
+        // d + t = h - m + l exactly up to t's rounding (|t| < 1e-6, so the dropped t^2 is
+        // far below fp32)
+        float m = -INFINITY;
 #pragma unroll
         for (int j = 0; j < CW; ++j)
-          if (e0 + j < p.E) m = fmax(m, acc[j]);
-        red[g * kBM + row] = m;
-        asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-        m = red[row];
+          if (e0 + j < p.E) m = fmaxf(m, h[j]);
+        red_m[g * 64 + r64] = m;
+        asm volatile("bar.sync 1, %0;" ::"r"(nfin) : "memory");
 #pragma unroll
-        for (int h = 1; h < G; ++h) m = fmax(m, red[h * kBM + row]);
-        double z = 0.0;
+        for (int k = 0; k < G; ++k) m = fmaxf(m, red_m[k * 64 + r64]);
+        bool deep = false;                   // some argument below -80
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
-          acc[j] = (e0 + j < p.E) ? exp_f64_arg(acc[j] - m) : 0.0;
-          z += acc[j];
+          float dd, tt;                      // exp argument: dd + tt
+          two_sum(h[j], -m, dd, tt);
+          tt += l[j];
+          const bool live_e = e0 + j < p.E;
+          deep |= live_e && dd < -80.f;
+          pr[j] = live_e ? expf(dd) * (1.f + tt) : 0.f;
         }
-        red[(G + g) * kBM + row] = z;
-        asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-        z = 0.0;
+        // below e^-80 the fp32 exponential leaves the normal range: fp64 there (rare, and
+        // kept out of the loop above so that it costs nothing otherwise)
+        if (__any_sync(0xffffffffu, deep)) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) z += red[(G + h) * kBM + row];
-        const double rz = 1.0 / z;
+          for (int j = 0; j < CW; ++j) {
+            float dd, tt;
+            two_sum(h[j], -m, dd, tt);
+            if (e0 + j < p.E && dd < -80.f) pr[j] = (float)exp((double)dd + (double)(tt + l[j]));
+          }
+        }
+        float zs = 0.f, zc = 0.f;            // compensated sum of the exponentials
 #pragma unroll
-        for (int j = 0; j < CW; ++j) acc[j] *= rz;
+        for (int j = 0; j < CW; ++j) {
+          float s_, e_;
+          two_sum(zs, pr[j], s_, e_);
+          zs = s_;
+          zc += e_;
+        }
+        red_z[g * 64 + r64] = make_float2(zs, zc);
+        asm volatile("bar.sync 1, %0;" ::"r"(nfin) : "memory");
+        zs = 0.f;
+        zc = 0.f;
+#pragma unroll
+        for (int k = 0; k < G; ++k) {
+          const float2 v = red_z[k * 64 + r64];
+          float s_, e_;
+          two_sum(zs, v.x, s_, e_);
+          zs = s_;
+          zc += e_ + v.y;
+        }
+        const float rz = 1.f / (zs + zc);    // one division; each score 1 ulp from e / z
+#pragma unroll
+        for (int j = 0; j < CW; ++j) pr[j] *= rz;
       } else {
+        // 1 / (1 + exp(-(h + l))), exp(-(h + l)) = exp(-h) (1 - l)
+        bool deep = false;
 #pragma unroll
-        for (int j = 0; j < CW; ++j) acc[j] = 1.0 / (1.0 + exp_f64_arg(-acc[j]));
+        for (int j = 0; j < CW; ++j) {
+          deep |= fabsf(h[j]) > 80.f;
+          pr[j] = 1.f / (1.f + expf(-h[j]) * (1.f - l[j]));
+        }
+        if (__any_sync(0xffffffffu, deep)) {
+#pragma unroll
+          for (int j = 0; j < CW; ++j)
+            if (fabsf(h[j]) > 80.f)
+              pr[j] = (float)(1.0 / (1.0 + exp(-((double)h[j] + (double)l[j]))));
+        }
       }
       if (ok && live) {
         float* srow = p.scores + (int64_t)t * p.E + e0;
         if ((p.E & 3) == 0 && e0 + CW <= p.E) {
 #pragma unroll
           for (int j = 0; j < CW; j += 4)
-            *reinterpret_cast<float4*>(srow + j) = make_float4(
-                (float)acc[j], (float)acc[j + 1], (float)acc[j + 2], (float)acc[j + 3]);
+            *reinterpret_cast<float4*>(srow + j) =
+                make_float4(pr[j], pr[j + 1], pr[j + 2], pr[j + 3]);
         } else {
 #pragma unroll
           for (int j = 0; j < CW; ++j)
-            if (e0 + j < p.E) srow[j] = (float)acc[j];
+            if (e0 + j < p.E) srow[j] = pr[j];
         }
 #pragma unroll
         for (int j = 0; j < CW; ++j)
-          if (e0 + j < p.E) p.scores_t[(int64_t)(e0 + j) * p.T + t] = (float)acc[j];
+          if (e0 + j < p.E) p.scores_t[(int64_t)(e0 + j) * p.T + t] = pr[j];
       }
     }
   }
@@ -372,7 +425,10 @@ cudaError_t launch_router_sm100(const void* x, const void* W_r, const Shape& s,
     // a shape the tensor maps cannot describe: the CUDA-core router computes the same
     return launch_router_simt(x, W_r, s, NMOE_BF16, fn, bias, scores, scores_t, st);
   size_t smem = (size_t)kStages * (kABytes + p.nbox * kBBoxBytes);
-  const size_t red = sizeof(double) * kBM * (size_t)(kMaxE + 2 * 4);
+  // the tail reuses the ring: exchange [kMaxE][64] (h, l) pairs, then [4][64] maxima and
+  // [4][64] (sum, error) pairs
+  const size_t red = sizeof(float2) * 64 * kMaxE + sizeof(float) * 4 * 64 +
+                     sizeof(float2) * 4 * 64;
   smem = (smem > red ? smem : red) + 1024;
   // 16 experts per thread up to E = 64 (up to 16 epilogue warps), 32 beyond
   const int CW = s.E <= 64 ? 16 : 32;
