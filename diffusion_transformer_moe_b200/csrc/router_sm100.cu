@@ -21,8 +21,8 @@
 // 64, K = 16) into a ring of TMEM chunk buffers; 4*G epilogue warps (G = ceil(E/CW))
 // each own 32 tokens x CW experts. Then each CTA sends its sums for the partner's half
 // of the tokens to the partner's shared memory (distributed shared memory, no global
-// traffic), and each finishes the score function and both score layouts for its 64
-// tokens. Every wait is bounded.
+// traffic), and all its epilogue warps finish the score function and both score layouts
+// for its 64 tokens. Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <cooperative_groups.h>
@@ -225,138 +225,136 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
     }
     // Each logit as an unevaluated fp32 pair h + l (l below half an ulp of h): the
     // compensated sum hi - lo, renormalised.
-    float* h = hi;  // renormalised in place
-    float* l = lo;
-#pragma unroll
-    for (int j = 0; j < CW; ++j) {
-      float s_, e_;
-      two_sum(hi[j], -lo[j], s_, e_);
-      h[j] = s_;
-      l[j] = e_;
-    }
-    // Tokens 0..63 of the tile are finished by the first CTA, 64..127 by the second:
-    // each sends its half-d sums of the partner's rows to the partner's shared memory
-    // (laid out [expert][64 rows], (h, l) pairs), after the first cluster barrier has
-    // left both stage rings idle.
-    const bool mine = (q >> 1) == rank;     // this warp's rows are finished here
-    const int r64 = row & 63;
+    // Each logit as an unevaluated fp32 pair h + l (l below half an ulp of h), from the
+    // compensated sum hi - lo. Tokens 0..63 of the tile are finished by the first CTA,
+    // 64..127 by the second. Every thread puts its half-d pairs where the finishing CTA
+    // reads them, laid out [expert][64 tokens]: its own rows in `own`, the partner's rows
+    // in the partner's `xch` (distributed shared memory). The first cluster barrier has
+    // left both stage rings idle for this.
+    const bool mine = (q >> 1) == rank;
     float2* xch = reinterpret_cast<float2*>(smem);
-    float* red_m = reinterpret_cast<float*>(xch + (size_t)kMaxE * 64);  // [G][64]
-    float2* red_z = reinterpret_cast<float2*>(red_m + 4 * 64);          // [G][64]
+    float2* own = xch + (size_t)kMaxE * 64;
+    float* red_m = reinterpret_cast<float*>(own + (size_t)kMaxE * 64);  // [2G][64]
+    float2* red_z = reinterpret_cast<float2*>(red_m + 8 * 64);          // [2G][64]
     cluster.sync();                         // (1) every ring is idle
-    if (!mine) {
-      float2* remote = cluster.map_shared_rank(xch, rank ^ 1);
-#pragma unroll
-      for (int j = 0; j < CW; ++j)
-        if (e0 + j < p.E) remote[(e0 + j) * 64 + r64] = make_float2(h[j], l[j]);
-    }
-    cluster.sync();                         // (2) the partner's sums have landed
-    if (mine) {
-      const int nfin = 64 * G;               // threads finishing this CTA's 64 tokens
-      const int t = t0 + row;
-      const bool live = t < p.T;
-      const float* b =
-          (p.bias != nullptr && live) ? p.bias + (int64_t)(t / p.S) * p.E : nullptr;
+    {
+      float2* dst = mine ? own : cluster.map_shared_rank(xch, rank ^ 1);
+      const int r64 = row & 63;
 #pragma unroll
       for (int j = 0; j < CW; ++j) {
-        if (e0 + j < p.E) {
-          const float2 v = xch[(e0 + j) * 64 + r64];
-          float s_, e_;
-          two_sum(h[j], v.x, s_, e_);
-          two_sum(s_, e_ + (l[j] + v.y), h[j], l[j]);
-          if (b) {
-            two_sum(h[j], b[e0 + j], s_, e_);
-            two_sum(s_, e_ + l[j], h[j], l[j]);
-          }
+        float s_, e_;
+        two_sum(hi[j], -lo[j], s_, e_);
+        if (e0 + j < p.E) dst[(e0 + j) * 64 + r64] = make_float2(s_, e_);
+      }
+    }
+    cluster.sync();                         // (2) the partner's sums have landed
+    // All 4G epilogue warps finish this CTA's 64 tokens: thread et takes token et % 64
+    // and the kEpc experts of group et / 64 (2G groups).
+    constexpr int kEpc = CW / 2;
+    const int nthr = 128 * G;
+    const int et = threadIdx.x - 64;
+    const int tk = et & 63, grp = et >> 6;
+    const int eb = grp * kEpc;
+    const int t = t0 + rank * 64 + tk;
+    const bool live = t < p.T;
+    const float* b = (p.bias != nullptr && live) ? p.bias + (int64_t)(t / p.S) * p.E : nullptr;
+    float h[kEpc], l[kEpc], pr[kEpc];
+#pragma unroll 4
+    for (int j = 0; j < kEpc; ++j) {
+      h[j] = 0.f;
+      l[j] = 0.f;
+      const int e = eb + j;
+      if (e < p.E) {
+        const float2 u = own[e * 64 + tk], v = xch[e * 64 + tk];
+        float s_, e_;
+        two_sum(u.x, v.x, s_, e_);
+        two_sum(s_, e_ + (u.y + v.y), h[j], l[j]);
+        if (b) {
+          two_sum(h[j], b[e], s_, e_);
+          two_sum(s_, e_ + l[j], h[j], l[j]);
         }
       }
-      float pr[CW];
-      if (p.score_fn == NMOE_SCORE_SOFTMAX) {
-        // shift by the largest high part; exp(h - m + l) = exp(d) (1 + t) with
-        // d + t = h - m + l exactly up to t's rounding (|t| < 1e-6, so the dropped t^2 is
-        // far below fp32)
-        float m = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < CW; ++j)
-          if (e0 + j < p.E) m = fmaxf(m, h[j]);
-        red_m[g * 64 + r64] = m;
-        asm volatile("bar.sync 1, %0;" ::"r"(nfin) : "memory");
-#pragma unroll
-        for (int k = 0; k < G; ++k) m = fmaxf(m, red_m[k * 64 + r64]);
-        bool deep = false;                   // some argument below -80
-#pragma unroll
-        for (int j = 0; j < CW; ++j) {
-          float dd, tt;                      // exp argument: dd + tt
+    }
+    if (p.score_fn == NMOE_SCORE_SOFTMAX) {
+      // shift by the largest high part; exp(h - m + l) = exp(d) (1 + t) with d + t =
+      // h - m + l exactly up to t's rounding (|t| < 1e-6, so the dropped t^2 is far
+      // below fp32)
+      float m = -INFINITY;
+#pragma unroll 4
+      for (int j = 0; j < kEpc; ++j)
+        if (eb + j < p.E) m = fmaxf(m, h[j]);
+      red_m[grp * 64 + tk] = m;
+      asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
+      for (int k = 0; k < 2 * G; ++k) m = fmaxf(m, red_m[k * 64 + tk]);
+      bool deep = false;                     // some argument below -80
+      float zs = 0.f, zc = 0.f;              // compensated sum of the exponentials
+#pragma unroll 4
+      for (int j = 0; j < kEpc; ++j) {
+        float dd, tt;                        // exp argument: dd + tt
+        two_sum(h[j], -m, dd, tt);
+        tt += l[j];
+        const bool live_e = eb + j < p.E;
+        deep |= live_e && dd < -80.f;
+        pr[j] = live_e ? expf(dd) * (1.f + tt) : 0.f;
+      }
+      // below e^-80 the fp32 exponential leaves the normal range: fp64 there (rare, and
+      // kept out of the loop above so that it costs nothing otherwise)
+      if (__any_sync(0xffffffffu, deep)) {
+        for (int j = 0; j < kEpc; ++j) {
+          float dd, tt;
           two_sum(h[j], -m, dd, tt);
-          tt += l[j];
-          const bool live_e = e0 + j < p.E;
-          deep |= live_e && dd < -80.f;
-          pr[j] = live_e ? expf(dd) * (1.f + tt) : 0.f;
+          if (eb + j < p.E && dd < -80.f) pr[j] = (float)exp((double)dd + (double)(tt + l[j]));
         }
-        // below e^-80 the fp32 exponential leaves the normal range: fp64 there (rare, and
-        // kept out of the loop above so that it costs nothing otherwise)
-        if (__any_sync(0xffffffffu, deep)) {
+      }
+#pragma unroll 4
+      for (int j = 0; j < kEpc; ++j) {
+        float s_, e_;
+        two_sum(zs, pr[j], s_, e_);
+        zs = s_;
+        zc += e_;
+      }
+      red_z[grp * 64 + tk] = make_float2(zs, zc);
+      asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
+      zs = 0.f;
+      zc = 0.f;
+      for (int k = 0; k < 2 * G; ++k) {
+        const float2 v = red_z[k * 64 + tk];
+        float s_, e_;
+        two_sum(zs, v.x, s_, e_);
+        zs = s_;
+        zc += e_ + v.y;
+      }
+      const float rz = 1.f / (zs + zc);      // one division; each score 1 ulp from e / z
+#pragma unroll 4
+      for (int j = 0; j < kEpc; ++j) pr[j] *= rz;
+    } else {
+      // 1 / (1 + exp(-(h + l))), exp(-(h + l)) = exp(-h) (1 - l)
+      bool deep = false;
+#pragma unroll 4
+      for (int j = 0; j < kEpc; ++j) {
+        deep |= fabsf(h[j]) > 80.f;
+        pr[j] = 1.f / (1.f + expf(-h[j]) * (1.f - l[j]));
+      }
+      if (__any_sync(0xffffffffu, deep)) {
+        for (int j = 0; j < kEpc; ++j)
+          if (fabsf(h[j]) > 80.f)
+            pr[j] = (float)(1.0 / (1.0 + exp(-((double)h[j] + (double)l[j]))));
+      }
+    }
+    if (ok && live && eb < p.E) {
+      float* srow = p.scores + (int64_t)t * p.E + eb;
+      if ((p.E & 3) == 0 && eb + kEpc <= p.E) {
 #pragma unroll
-          for (int j = 0; j < CW; ++j) {
-            float dd, tt;
-            two_sum(h[j], -m, dd, tt);
-            if (e0 + j < p.E && dd < -80.f) pr[j] = (float)exp((double)dd + (double)(tt + l[j]));
-          }
-        }
-        float zs = 0.f, zc = 0.f;            // compensated sum of the exponentials
-#pragma unroll
-        for (int j = 0; j < CW; ++j) {
-          float s_, e_;
-          two_sum(zs, pr[j], s_, e_);
-          zs = s_;
-          zc += e_;
-        }
-        red_z[g * 64 + r64] = make_float2(zs, zc);
-        asm volatile("bar.sync 1, %0;" ::"r"(nfin) : "memory");
-        zs = 0.f;
-        zc = 0.f;
-#pragma unroll
-        for (int k = 0; k < G; ++k) {
-          const float2 v = red_z[k * 64 + r64];
-          float s_, e_;
-          two_sum(zs, v.x, s_, e_);
-          zs = s_;
-          zc += e_ + v.y;
-        }
-        const float rz = 1.f / (zs + zc);    // one division; each score 1 ulp from e / z
-#pragma unroll
-        for (int j = 0; j < CW; ++j) pr[j] *= rz;
+        for (int j = 0; j < kEpc; j += 4)
+          *reinterpret_cast<float4*>(srow + j) =
+              make_float4(pr[j], pr[j + 1], pr[j + 2], pr[j + 3]);
       } else {
-        // 1 / (1 + exp(-(h + l))), exp(-(h + l)) = exp(-h) (1 - l)
-        bool deep = false;
-#pragma unroll
-        for (int j = 0; j < CW; ++j) {
-          deep |= fabsf(h[j]) > 80.f;
-          pr[j] = 1.f / (1.f + expf(-h[j]) * (1.f - l[j]));
-        }
-        if (__any_sync(0xffffffffu, deep)) {
-#pragma unroll
-          for (int j = 0; j < CW; ++j)
-            if (fabsf(h[j]) > 80.f)
-              pr[j] = (float)(1.0 / (1.0 + exp(-((double)h[j] + (double)l[j]))));
-        }
+        for (int j = 0; j < kEpc; ++j)
+          if (eb + j < p.E) srow[j] = pr[j];
       }
-      if (ok && live) {
-        float* srow = p.scores + (int64_t)t * p.E + e0;
-        if ((p.E & 3) == 0 && e0 + CW <= p.E) {
-#pragma unroll
-          for (int j = 0; j < CW; j += 4)
-            *reinterpret_cast<float4*>(srow + j) =
-                make_float4(pr[j], pr[j + 1], pr[j + 2], pr[j + 3]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < CW; ++j)
-            if (e0 + j < p.E) srow[j] = pr[j];
-        }
-#pragma unroll
-        for (int j = 0; j < CW; ++j)
-          if (e0 + j < p.E) p.scores_t[(int64_t)(e0 + j) * p.T + t] = pr[j];
-      }
+#pragma unroll 4
+      for (int j = 0; j < kEpc; ++j)
+        if (eb + j < p.E) p.scores_t[(int64_t)(eb + j) * p.T + t] = pr[j];
     }
   }
   if (warp < 2) {
@@ -425,10 +423,10 @@ cudaError_t launch_router_sm100(const void* x, const void* W_r, const Shape& s,
     // a shape the tensor maps cannot describe: the CUDA-core router computes the same
     return launch_router_simt(x, W_r, s, NMOE_BF16, fn, bias, scores, scores_t, st);
   size_t smem = (size_t)kStages * (kABytes + p.nbox * kBBoxBytes);
-  // the tail reuses the ring: exchange [kMaxE][64] (h, l) pairs, then [4][64] maxima and
-  // [4][64] (sum, error) pairs
-  const size_t red = sizeof(float2) * 64 * kMaxE + sizeof(float) * 4 * 64 +
-                     sizeof(float2) * 4 * 64;
+  // the tail reuses the ring: two [kMaxE][64] arrays of (h, l) pairs, then [8][64] maxima
+  // and [8][64] (sum, error) pairs
+  const size_t red = 2 * sizeof(float2) * 64 * kMaxE + sizeof(float) * 8 * 64 +
+                     sizeof(float2) * 8 * 64;
   smem = (smem > red ? smem : red) + 1024;
   // 16 experts per thread up to E = 64 (up to 16 epilogue warps), 32 beyond
   const int CW = s.E <= 64 ? 16 : 32;
