@@ -104,10 +104,17 @@ def _traffic(kernel_stage, workload):
     h = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
     if not m or not h:
         return None
-    src = os.path.join(ROOT, "diffusion_transformer_moe_b200", "csrc", "experts_sm100.cu")
+    src = os.path.join(ROOT, "diffusion_transformer_moe_b200", "csrc",
+                       STAGE_SOURCE.get(kernel_stage, "experts_sm100.cu"))
     if hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
         return None
     return float(m.group(1))
+
+
+# the source file of each stage's kernel (a summary is stale once its file changes)
+STAGE_SOURCE = {"router": "router_sm100.cu", "select": "select.cu", "csr": "select.cu",
+                "gemm1_swiglu": "experts_sm100.cu", "gemm2_scale": "experts_sm100.cu",
+                "combine": "combine.cu"}
 
 
 # ---- clocks during the timed region ----------------------------------------------------
