@@ -44,11 +44,18 @@ class Workload:
     dtype: str  # "bf16" or "f32"
     lognormal_scale: bool = False
     skewed: bool = False
+    segments: int = 1  # selection runs per segment of T / segments tokens (per image)
 
     @property
     def C(self) -> int:
-        # capacity = ceil(capacity_factor * tokens / experts) (walkthrough section 6.2)
-        return capacity(self.T, self.capacity_factor, self.E)
+        # capacity per segment = ceil(capacity_factor * tokens / experts) (walkthrough
+        # section 6.2, where a segment is one sample)
+        return capacity(self.T // self.segments, self.capacity_factor, self.E)
+
+    @property
+    def Ce(self) -> int:
+        """Entries per expert: C per segment."""
+        return self.segments * self.C
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -56,7 +63,7 @@ class Workload:
 
     def expert_flops(self) -> float:
         # GEMM1 (gate + up) 4*E*C*d*F, GEMM2 2*E*C*F*d
-        return 6.0 * self.E * self.C * self.d * self.F
+        return 6.0 * self.E * self.Ce * self.d * self.F
 
     def router_flops(self) -> float:
         return 2.0 * self.T * self.d * self.E
@@ -77,6 +84,10 @@ WORKLOADS = {
                  dtype="bf16"),
         Workload("skewed_2048px", T=16384, d=2048, E=128, F=768, capacity_factor=1,
                  dtype="bf16", skewed=True),
+        # the model's own layer shape (walkthrough section 6 defaults: 128 experts of
+        # width 1344, capacity factor 8) on a 1024 px CFG pair, selection per image
+        Workload("model_default_1024px_cfg", T=8192, d=2048, E=128, F=1344,
+                 capacity_factor=8, dtype="bf16", segments=2),
     )
 }
 

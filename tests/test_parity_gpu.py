@@ -294,19 +294,21 @@ N_SAMPLE = 192
 
 
 @pytest.mark.parametrize("name", ["512px_cfg", "1024px_cfg", "skewed_2048px",
-                                  "batch4_1024px_cfg"])
+                                  "batch4_1024px_cfg", "model_default_1024px_cfg"])
 def test_full_workload_matches_oracle(name):
     w = I.WORKLOADS[name]
+    nseg = w.segments
     a = I.make_inputs(w)
     dev = {k: v.cuda() for k, v in a.items()}
-    ws = torch.empty(nm.workspace_size(w.T, w.d, w.E, w.F, w.C, out_f32=True),
+    ws = torch.empty(nm.workspace_size(w.T, w.d, w.E, w.F, w.C, out_f32=True,
+                                       n_segments=nseg),
                      dtype=torch.uint8, device="cuda")
     scores = torch.empty(w.T, w.E, device="cuda", dtype=torch.float32)
-    idx = torch.empty(w.E, w.C, device="cuda", dtype=torch.int32)
+    idx = torch.empty(w.E, w.Ce, device="cuda", dtype=torch.int32)
     out = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C,
-                     workspace=ws, scores_out=scores, idx_out=idx)
+                     workspace=ws, scores_out=scores, idx_out=idx, n_segments=nseg)
     out32 = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C,
-                       workspace=ws, out_f32=True)
+                       workspace=ws, out_f32=True, n_segments=nseg)
     torch.cuda.synchronize()
     assert nm.get_last_error() == 0
     # the bf16 output is the fp32 result rounded once
@@ -315,12 +317,12 @@ def test_full_workload_matches_oracle(name):
     x = I.to_numpy_f64(a["x"])
     W_r = I.to_numpy_f64(a["W_r"])
     s_gpu = scores.cpu().numpy()
-    sel = O.select(s_gpu, w.C)
+    sel = O.select(s_gpu, w.C, nseg)
     assert np.array_equal(sel, idx.cpu().numpy())
     p = O.scores_from_logits(O.router_logits(x, W_r))
     _check_scores(scores, p)
     # the oracle's own selection may differ only where scores are within tolerance
-    own = O.select(O.round_f32(p), w.C)
+    own = O.select(O.round_f32(p), w.C, nseg)
     n_diff = sum(len(set(own[e]) ^ set(sel[e])) for e in range(w.E))
     assert n_diff <= 2 * w.E
     rng = np.random.default_rng(0)
@@ -332,7 +334,7 @@ def test_full_workload_matches_oracle(name):
                                      rng.choice(chosen, N_SAMPLE // 3, replace=False),
                                      chosen[np.argsort(-norms)[:N_SAMPLE // 3]]]))
     W1 = a["W1"].float().numpy(); W3 = a["W3"].float().numpy(); W2 = a["W2"].float().numpy()
-    r = O.layer_rows(x, W_r, W1, W3, W2, w.C, toks, selection=sel)
+    r = O.layer_rows(x, W_r, W1, W3, W2, w.C, toks, selection=sel, n_segments=nseg)
     tk = torch.as_tensor(toks, device="cuda")
     _check_out(out[tk], r["out"], w.dtype)
     _check_out(out32[tk], r["out"], "bf16f32" if w.dtype == "bf16" else "f32")
