@@ -36,7 +36,14 @@ Readings taken where the page is silent (each is listed in the design doc as well):
     ascending expert order;
   * the page's router input cat([timestep, hidden]) is exactly a per-segment additive
     logit bias ``router_bias[s, e] = temb_s . W_gate[:d_t, e]``
-    (see :func:`router_logits_concat` for the literal form).
+    (see :func:`router_logits_concat` for the literal form);
+  * the shared expert (section 6.2: one SwiGLU feed-forward over every token, the
+    routed outputs added onto its output) has its own width F_shared, which the page
+    does not give;
+  * the block around the layer (section 6.3: the modulation gates pass through
+    clamp(-2, 2) and then tanh) adds the layer output to its residual stream as
+    ``residual + tanh(clamp(gate2, -2, 2)) * ffn_out``, with one gate vector of d
+    values per segment (sample); see :func:`gated_residual`.
 
 Every floating-point step is done in fp64 on the exact values of the inputs.
 """
@@ -185,15 +192,29 @@ def combine_weights(p, idx, mode: str = "raw", route_scale: float = 1.0) -> np.n
     return out
 
 
+def gated_residual(residual, gate2, ffn_out, n_segments: int = 1) -> np.ndarray:
+    """Section 6.3: residual + tanh(clamp(gate2, -2, 2)) * ffn_out, the gate row of each
+    token's segment (gate2 [n_segments, d]; None means a gate of one)."""
+    out = np.asarray(ffn_out, dtype=F64)
+    if gate2 is not None:
+        g = np.tanh(np.clip(_f64(gate2), -2.0, 2.0))
+        seg = np.arange(out.shape[0]) // (out.shape[0] // n_segments)
+        out = g[seg] * out
+    return _f64(residual) + out
+
+
 def layer(x, W_r, W1, W3, W2, C: int, *, score_fn: str = "softmax",
           combine: str = "raw", route_scale: float = 1.0, n_segments: int = 1,
-          router_bias=None, selection=None, shared=None) -> dict:
+          router_bias=None, selection=None, shared=None, residual=None,
+          gate2=None) -> dict:
     """The whole MoE FFN layer.
 
     ``selection`` injects an expert-choice selection (idx[E, n_segments*C]) instead of
     the oracle's own, so that outputs can be compared given the same integer decisions.
     ``shared`` = (Ws1 [d,Fs], Ws3 [d,Fs], Ws2 [Fs,d]) adds a shared SwiGLU expert that
     every token goes through (section 6.2), onto which the routed outputs are added.
+    ``residual`` [T,d] (and ``gate2`` [n_segments,d]) add the result to the block's
+    residual stream through the gate (section 6.3, :func:`gated_residual`).
 
     Returns dict(out [T,d] fp64, p fp64 [T,E], scores32 [T,E], idx, w).
     """
@@ -213,12 +234,15 @@ def layer(x, W_r, W1, W3, W2, C: int, *, score_fn: str = "softmax",
         rows = idx[e]
         y = swiglu_ffn(x[rows], W1[e], W3[e], W2[e])
         out[rows] += w[e][:, None] * y  # rows within one expert are distinct
+    if residual is not None:
+        out = gated_residual(residual, gate2, out, n_segments)
     return dict(out=out, p=p, scores32=s32, idx=idx, w=w)
 
 
 def layer_rows(x, W_r, W1, W3, W2, C: int, tokens, *, score_fn: str = "softmax",
                combine: str = "raw", route_scale: float = 1.0, n_segments: int = 1,
-               router_bias=None, selection=None, shared=None) -> dict:
+               router_bias=None, selection=None, shared=None, residual=None,
+               gate2=None) -> dict:
     """The layer output for the listed tokens only (for workloads too large to run
     whole). Router, scores and selection still cover every token."""
     x = _f64(x)
@@ -242,4 +266,9 @@ def layer_rows(x, W_r, W1, W3, W2, C: int, tokens, *, score_fn: str = "softmax",
         y = swiglu_ffn(x[idx[e][slots]], np.asarray(W1[e]), np.asarray(W3[e]),
                        np.asarray(W2[e]))
         out[where] += w[e][slots][:, None] * y
+    if residual is not None:
+        T = x.shape[0]
+        g = np.ones((len(tokens), x.shape[1])) if gate2 is None else \
+            np.tanh(np.clip(_f64(gate2), -2.0, 2.0))[tokens // (T // n_segments)]
+        out = _f64(residual)[tokens] + g * out
     return dict(out=out, p=p, scores32=s32, idx=idx, w=w)

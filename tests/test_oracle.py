@@ -238,6 +238,64 @@ def test_shared_expert_adds_dense_ffn():
                                atol=1e-13)
 
 
+# -- the block's gated residual (section 6.3) ----------------------------------------------
+
+def _tanh(a):
+    """tanh from its exponential definition (not numpy's tanh)."""
+    import math
+    return (math.exp(2 * a) - 1.0) / (math.exp(2 * a) + 1.0)
+
+
+def test_gated_residual_with_a_zero_gate_is_the_residual():
+    a = _small(16, 6, 3, 4, seed=30)
+    res = np.random.default_rng(1).standard_normal((16, 6))
+    r = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=5, residual=res,
+                gate2=np.zeros((1, 6)))
+    assert np.array_equal(r["out"], res)
+
+
+def test_gated_residual_clamps_to_two_then_takes_tanh():
+    a = _small(16, 6, 3, 4, seed=31)
+    res = np.random.default_rng(2).standard_normal((16, 6))
+    gate = np.array([[-5.0, -2.0, -0.5, 0.5, 2.0, 7.0]])
+    r0 = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=5)
+    r = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=5, residual=res, gate2=gate)
+    factor = np.array([_tanh(-2.0), _tanh(-2.0), _tanh(-0.5), _tanh(0.5), _tanh(2.0),
+                       _tanh(2.0)])
+    np.testing.assert_allclose(r["out"], res + factor * r0["out"], rtol=1e-14, atol=1e-15)
+    assert abs(factor[-1] - 0.9640275800758169) < 1e-15  # tanh(2), not tanh(7)
+
+
+def test_gated_residual_takes_each_segments_gate_row():
+    a = _small(24, 4, 3, 4, seed=32)
+    res = np.zeros((24, 4))
+    gate = np.array([[0.3, 0.3, 0.3, 0.3], [-1.0, -1.0, -1.0, -1.0], [1.5, 1.5, 1.5, 1.5]])
+    r0 = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=3, n_segments=3)
+    r = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=3, n_segments=3,
+                residual=res, gate2=gate)
+    for seg, gval in enumerate((0.3, -1.0, 1.5)):
+        rows = slice(8 * seg, 8 * seg + 8)
+        np.testing.assert_allclose(r["out"][rows], _tanh(gval) * r0["out"][rows],
+                                   rtol=1e-14, atol=1e-15)
+
+
+def test_gated_residual_wraps_shared_plus_routed_and_rows_agree():
+    a = _small(20, 6, 3, 4, seed=33)
+    sh = (a["W1"][1], a["W3"][1], a["W2"][1])
+    res = np.random.default_rng(3).standard_normal((20, 6))
+    gate = np.random.default_rng(4).standard_normal((2, 6))
+    routed = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=4, n_segments=2)["out"]
+    r = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=4, n_segments=2, shared=sh,
+                residual=res, gate2=gate)
+    g = np.array([[_tanh(min(2.0, max(-2.0, v))) for v in row] for row in gate])
+    want = res + g[np.arange(20) // 10] * (_dense_ffn(a["x"], *sh) + routed)
+    np.testing.assert_allclose(r["out"], want, rtol=1e-12, atol=1e-13)
+    toks = [0, 7, 10, 19]
+    rr = O.layer_rows(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], 4, toks, n_segments=2,
+                      shared=sh, residual=res, gate2=gate)
+    np.testing.assert_allclose(rr["out"], r["out"][toks], rtol=1e-13, atol=1e-14)
+
+
 # -- the skewed workload has what it promises ---------------------------------------------
 
 @pytest.mark.slow
