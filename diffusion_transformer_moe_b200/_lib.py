@@ -49,7 +49,9 @@ class Options(C.Structure):
         ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t),
         ("scores_out", C.c_void_p), ("idx_out", C.c_void_p), ("host_io", C.c_int),
         ("trace", C.c_void_p), ("intermediate", C.c_int), ("out_f32", C.c_int),
-        ("tma_gather", C.c_int),
+        ("tma_gather", C.c_int), ("shared_w1", C.c_void_p), ("shared_w3", C.c_void_p),
+        ("shared_w2", C.c_void_p), ("shared_f", C.c_int64), ("residual", C.c_void_p),
+        ("gate2", C.c_void_p),
     ]
 
 
@@ -139,7 +141,12 @@ def _dev(t: torch.Tensor, name: str) -> None:
 def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
             n_segments=1, router_bias=None, workspace=None, scores_out=None, idx_out=None,
             host_io=False, trace=None, intermediate="split", out_f32=False,
-            tma_gather=False) -> Options:
+            tma_gather=False, shared=None, shared_f=None, residual=None,
+            gate2=None) -> Options:
+    """nmoe_options from keyword arguments. ``shared`` = (Ws1 [d,Fs], Ws3 [d,Fs],
+    Ws2 [Fs,d]) device tensors adds the shared expert; ``shared_f`` alone (no tensors)
+    only sizes a workspace for one. ``residual`` [T,d] and ``gate2`` fp32
+    [n_segments,d] add the block's gated residual."""
     o = Options()
     lib().nmoe_options_init(C.byref(o))
     o.dtype = dtype
@@ -158,6 +165,18 @@ def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
     o.intermediate = INTERMEDIATE[intermediate]
     o.out_f32 = 1 if out_f32 else 0
     o.tma_gather = 1 if tma_gather else 0
+    if shared is not None:
+        Ws1, Ws3, Ws2 = shared
+        for n, t in (("shared Ws1", Ws1), ("shared Ws3", Ws3), ("shared Ws2", Ws2)):
+            _dev(t, n)
+        o.shared_w1, o.shared_w3, o.shared_w2 = Ws1.data_ptr(), Ws3.data_ptr(), Ws2.data_ptr()
+        o.shared_f = int(Ws1.shape[1])
+    elif shared_f is not None:
+        # sizing only (nmoe_workspace_size reads no weight): non-null placeholders
+        o.shared_w1 = o.shared_w3 = o.shared_w2 = 256
+        o.shared_f = int(shared_f)
+    o.residual = _ptr(residual)
+    o.gate2 = _ptr(gate2)
     return o
 
 
@@ -193,8 +212,8 @@ def select(scores_t, C_: int, n_segments=1, csr=True, stream=None):
 def forward(x, W_r, W1, W3, W2, C_: int, out=None, stream=None, **opts):
     """The whole layer. ``opts`` are the nmoe_options fields (score_fn, combine,
     route_scale, n_segments, router_bias, workspace, scores_out, idx_out, trace,
-    intermediate, out_f32, tma_gather). With ``host_io=True`` x and out are pinned CPU
-    tensors."""
+    intermediate, out_f32, tma_gather, shared=(Ws1, Ws3, Ws2), residual, gate2). With
+    ``host_io=True`` x and out are pinned CPU tensors."""
     host_io = bool(opts.get("host_io", False))
     for n, t in (("W_r", W_r), ("W1", W1), ("W3", W3), ("W2", W2)):
         _dev(t, n)

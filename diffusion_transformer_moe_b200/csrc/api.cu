@@ -112,7 +112,8 @@ size_t out_size(nmoe_dtype dt, const nmoe_options& o) {
 }
 
 struct Layout {
-  size_t scores, scores_t, idx, gate, bnd, tok_ptr, tok_ent, ent_pos, H, Y, xin, xout, total;
+  size_t scores, scores_t, idx, gate, bnd, tok_ptr, tok_ent, ent_pos, H, Hs, Y, xin, xout,
+      total;
 };
 
 Layout make_layout(const Shape& s, nmoe_dtype dt, const nmoe_options& o) {
@@ -126,11 +127,14 @@ Layout make_layout(const Shape& s, nmoe_dtype dt, const nmoe_options& o) {
   L.idx = o.idx_out ? none : take(sizeof(int32_t) * (size_t)s.E * s.Ce);
   L.gate = take(sizeof(float) * (size_t)s.E * s.Ce);
   L.bnd = take(sizeof(int32_t) * nmoe::select_bound_entries(s));
+  // with a shared expert every token has one more entry (and Y row): its shared row
+  const size_t shared_rows = o.shared_w1 ? (size_t)s.T : 0;
   L.tok_ptr = take(sizeof(int32_t) * ((size_t)s.T + 1));
-  L.tok_ent = take(sizeof(int32_t) * (size_t)s.E * s.Ce);
+  L.tok_ent = take(sizeof(int32_t) * ((size_t)s.E * s.Ce + shared_rows));
   L.ent_pos = take(sizeof(int32_t) * (size_t)s.E * s.Ce);
   L.H = take(is * (size_t)s.E * s.Ce * s.F);
-  L.Y = take(is * (size_t)s.E * s.Ce * s.d);
+  L.Hs = o.shared_w1 ? take(is * (size_t)s.T * (size_t)o.shared_f) : none;
+  L.Y = take(is * ((size_t)s.E * s.Ce + shared_rows) * s.d);
   L.xin = o.host_io ? take(esize(dt) * (size_t)s.T * s.d) : none;
   L.xout = o.host_io ? take(out_size(dt, o) * (size_t)s.T * s.d) : none;
   L.total = off;
@@ -151,6 +155,18 @@ nmoe_status options_ok(const nmoe_options& o) {
     return NMOE_ERR_INVALID_ARG;
   if (o.intermediate != NMOE_INTERMEDIATE_SPLIT && o.intermediate != NMOE_INTERMEDIATE_BF16)
     return NMOE_ERR_INVALID_ARG;
+  const int n_shared = (o.shared_w1 != nullptr) + (o.shared_w3 != nullptr) +
+                       (o.shared_w2 != nullptr);
+  if (n_shared != 0 && n_shared != 3) return NMOE_ERR_INVALID_ARG;
+  if (n_shared == 3) {
+    if (!aligned16(o.shared_w1) || !aligned16(o.shared_w3) || !aligned16(o.shared_w2))
+      return NMOE_ERR_INVALID_ARG;
+    if (o.shared_f < 1 || o.shared_f >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
+    if (o.shared_f % 8 != 0) return NMOE_ERR_UNSUPPORTED;
+  }
+  if (o.gate2 && !o.residual) return NMOE_ERR_INVALID_ARG;
+  if (o.residual && !aligned16(o.residual)) return NMOE_ERR_INVALID_ARG;
+  if (o.gate2 && !aligned16(o.gate2)) return NMOE_ERR_INVALID_ARG;
   return NMOE_OK;
 }
 
@@ -180,11 +196,14 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
     return NMOE_ERR_INVALID_ARG;
   if (!o.host_io && (!aligned16(x) || !aligned16(out))) return NMOE_ERR_INVALID_ARG;
   if (x == out) return NMOE_ERR_INVALID_ARG;
+  if (o.residual != nullptr && o.residual == out) return NMOE_ERR_INVALID_ARG;
 
   DevState* ds = nullptr;
   if ((v = dev_state(&ds)) != NMOE_OK) return v;
   Shape s = make_shape(T, d, E, F, C, o.n_segments);
   if (s.Ce > 65535 * 64) return NMOE_ERR_UNSUPPORTED;
+  const bool has_shared = o.shared_w1 != nullptr;
+  if (has_shared && (int64_t)s.E * s.Ce + s.T >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
   // per-stage events sit between the launches, so traced calls run without overlap
   s.pdl = o.trace == nullptr;
   const Layout L = make_layout(s, o.dtype, o);
@@ -211,6 +230,14 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   int32_t* ent_pos = reinterpret_cast<int32_t*>(ws + L.ent_pos);
   void* H = ws + L.H;
   void* Y = ws + L.Y;
+  // the shared expert: one "expert" over all T tokens in token order (identity row map,
+  // weight 1), whose row of Y for token t is the first of t's span (tok_ptr[t])
+  Shape sh = s;
+  sh.E = 1; sh.F = (int)o.shared_f; sh.C = s.T; sh.n_seg = 1; sh.S = s.T; sh.Ce = s.T;
+  void* Hs = has_shared ? static_cast<void*>(ws + L.Hs) : nullptr;
+  void* Hs_lo = has_shared ? static_cast<void*>(ws + L.Hs + sizeof(uint16_t) * (size_t)s.T *
+                                                               (size_t)o.shared_f)
+                           : nullptr;
   const size_t xbytes = esize(o.dtype) * (size_t)s.T * s.d;
   const size_t obytes = out_size(o.dtype, o) * (size_t)s.T * s.d;
   const bool f32 = o.dtype == NMOE_F32;
@@ -243,9 +270,15 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   if (e == cudaSuccess) e = nmoe::launch_select(scores_t, s, idx, gate, bnd, ds->err, st);
   mark(2);
   if (e == cudaSuccess)
-    e = nmoe::launch_csr(idx, bnd, s, tok_ptr, tok_ent, ent_pos, gate, o.combine,
+    e = nmoe::launch_csr(idx, bnd, s, has_shared, tok_ptr, tok_ent, ent_pos, gate, o.combine,
                          o.route_scale, ds->err, st);
   mark(3);
+  const bool tc_sh = has_shared && !f32 && nmoe::experts_sm100_supported(sh);
+  if (has_shared && e == cudaSuccess)
+    e = tc_sh ? nmoe::launch_gemm1_sm100(xd, nullptr, o.shared_w1, o.shared_w3, sh, split,
+                                         false, Hs, Hs_lo, ds->err, ds->sm_count, st)
+              : nmoe::launch_gemm1_simt(xd, nullptr, o.shared_w1, o.shared_w3, sh, o.dtype,
+                                        split, Hs, st);
   const bool tc = !f32 && nmoe::experts_sm100_supported(s);
   // SPLIT on the tensor cores: H_hi then H_lo, each [E*Ce, F] bf16; on the CUDA cores
   // (shapes the tcgen05 kernels do not take) H is one fp32 array of the same size.
@@ -255,13 +288,19 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
                                       ds->err, ds->sm_count, st)
            : nmoe::launch_gemm1_simt(xd, idx, W1, W3, s, o.dtype, split, H, st);
   mark(4);
+  if (has_shared && e == cudaSuccess)
+    e = tc_sh ? nmoe::launch_gemm2_sm100(Hs, Hs_lo, nullptr, tok_ptr, o.shared_w2, sh, split,
+                                         Y, ds->err, ds->sm_count, st)
+              : nmoe::launch_gemm2_simt(Hs, nullptr, o.shared_w2, tok_ptr, sh, o.dtype, split,
+                                        y_f32, Y, st);
   if (e == cudaSuccess)
     e = tc ? nmoe::launch_gemm2_sm100(H, H_lo, gate, ent_pos, W2, s, split, Y, ds->err,
                                       ds->sm_count, st)
            : nmoe::launch_gemm2_simt(H, gate, W2, ent_pos, s, o.dtype, split, y_f32, Y, st);
   mark(5);
   if (e == cudaSuccess)
-    e = nmoe::launch_combine(Y, tok_ptr, s, y_f32, out_f32, outd, ds->err, ds->sm_count, st);
+    e = nmoe::launch_combine(Y, tok_ptr, s, y_f32, out_f32, outd, o.residual, !f32, o.gate2,
+                             ds->err, ds->sm_count, st);
   mark(6);
   if (o.host_io && e == cudaSuccess)
     e = cudaMemcpyAsync(out, outd, obytes, cudaMemcpyDeviceToHost, st);
@@ -297,6 +336,12 @@ void nmoe_options_init(nmoe_options* o) {
   o->intermediate = NMOE_INTERMEDIATE_SPLIT;
   o->out_f32 = 0;
   o->tma_gather = 0;
+  o->shared_w1 = nullptr;
+  o->shared_w3 = nullptr;
+  o->shared_w2 = nullptr;
+  o->shared_f = 0;
+  o->residual = nullptr;
+  o->gate2 = nullptr;
 }
 
 nmoe_status nmoe_router(const void* x, const void* W_r, int64_t T, int64_t d, int64_t E,
@@ -344,8 +389,8 @@ nmoe_status nmoe_select(const float* scores_t, int64_t T, int64_t E, int64_t C,
   // no scratch here: the CSR build searches idx instead of reading a boundary table
   cudaError_t e = nmoe::launch_select(scores_t, s, idx, gate, nullptr, ds->err, st);
   if (e == cudaSuccess && tok_ptr)
-    e = nmoe::launch_csr(idx, nullptr, s, tok_ptr, tok_ent, nullptr, gate, NMOE_COMBINE_RAW,
-                         1.f, ds->err, st);
+    e = nmoe::launch_csr(idx, nullptr, s, false, tok_ptr, tok_ent, nullptr, gate,
+                         NMOE_COMBINE_RAW, 1.f, ds->err, st);
   if (e != cudaSuccess) { cudaGetLastError(); return NMOE_ERR_CUDA; }
   return NMOE_OK;
 }

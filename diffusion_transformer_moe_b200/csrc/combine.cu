@@ -9,6 +9,11 @@
 // in ascending expert order (the order of the token lists), accumulated in fp32 and
 // rounded once to the output type. A token no expert chose gets an exact zero row.
 //
+// With the surrounding block's residual (section 6.3 of the walkthrough: the modulation
+// gates go through clamp(-2, 2) and tanh), each stored sum becomes
+//   out[t, :] = residual[t, :] + tanh(clamp(gate2[t / S, :], -2, 2)) * sum,
+// in fp32 before the one rounding.
+//
 // Each CTA owns a contiguous token range, whose rows of Y form one contiguous span.
 // Every thread owns one 16-byte column group and walks the span row by row with eight
 // independent loads in flight, adding into the current token's sum and storing it when
@@ -62,10 +67,57 @@ __device__ __forceinline__ void store_out(__nv_bfloat16* dst, const float* a) {
   }
 }
 
+// n residual values (of x's type) from p, as fp32
+template <int N>
+__device__ __forceinline__ void load_res(const void* p, bool bf16, float* r) {
+  if (bf16) {
+    const __nv_bfloat162* h = static_cast<const __nv_bfloat162*>(p);
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      r[2 * i] = f.x;
+      r[2 * i + 1] = f.y;
+    }
+  } else {
+    const float4* f = static_cast<const float4*>(p);
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const float4 v = f[i];
+      r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
+    }
+  }
+}
+
+// residual + tanh(clamp(gate, -2, 2)) * sum, on the N columns of one group
+template <int N>
+struct Gated {
+  const void* res;     // NULL: plain sum
+  bool res_bf16;
+  const float* gate2;  // [n_seg, d] or NULL (gate 1)
+  int d, S, col;
+  int seg = -1;
+  float g[N];
+  __device__ __forceinline__ void apply(int t, float* acc) {
+    if (res == nullptr) return;
+    if (gate2 != nullptr && t / S != seg) {
+      seg = t / S;
+#pragma unroll
+      for (int i = 0; i < N; ++i)
+        g[i] = tanhf(fminf(fmaxf(gate2[(int64_t)seg * d + col + i], -2.f), 2.f));
+    }
+    float r[N];
+    const size_t esz = res_bf16 ? 2 : 4;
+    load_res<N>(static_cast<const char*>(res) + ((int64_t)t * d + col) * esz, res_bf16, r);
+#pragma unroll
+    for (int i = 0; i < N; ++i) acc[i] = r[i] + (gate2 != nullptr ? g[i] : 1.f) * acc[i];
+  }
+};
+
 template <typename TY, typename TO>
 __global__ void __launch_bounds__(512)
 combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, int Tn, int d,
-               int tok_per_cta, TO* __restrict__ out) {
+               int tok_per_cta, TO* __restrict__ out, const void* __restrict__ residual,
+               int res_bf16, const float* __restrict__ gate2, int S) {
   constexpr int N = Vec<TY>::N;          // columns per 16-byte group
   pdl_launch_dependents();
   __shared__ int s_ptr[kMaxTokPerCta + 1];
@@ -79,6 +131,7 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
   const int64_t stride = d / N;          // 16-byte groups per row
   for (int grp = threadIdx.x; grp < ngroups; grp += blockDim.x) {
     const int col = grp * N;
+    Gated<N> gt{residual, res_bf16 != 0, gate2, d, S, col};
     const uint4* src = reinterpret_cast<const uint4*>(Y) + grp;
     float acc[N];
 #pragma unroll
@@ -94,6 +147,7 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
       for (int k = 0; k < kAhead; ++k) {
         if (r + k < r1) {
           while (r + k >= tend) {         // token t is complete (or had no rows)
+            gt.apply(t, acc);
             store_out<N>(out + (int64_t)t * d + col, acc);
 #pragma unroll
             for (int i = 0; i < N; ++i) acc[i] = 0.f;
@@ -105,6 +159,7 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
       }
     }
     for (; t < t1; ++t) {                  // the last token and any empty ones after it
+      gt.apply(t, acc);
       store_out<N>(out + (int64_t)t * d + col, acc);
 #pragma unroll
       for (int i = 0; i < N; ++i) acc[i] = 0.f;
@@ -114,6 +169,7 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
 
 template <typename TY, typename TO>
 cudaError_t launch_typed(const void* Y, const int32_t* tok_ptr, const Shape& s, void* out,
+                         const void* residual, bool res_bf16, const float* gate2,
                          int sm_count, cudaStream_t st) {
   constexpr int N = Vec<TY>::N;
   const int ngroups = s.d / N;
@@ -128,21 +184,26 @@ cudaError_t launch_typed(const void* Y, const int32_t* tok_ptr, const Shape& s, 
     grid = (int)ceil_div(s.T, per);
   }
   return launch_kernel(combine_kernel<TY, TO>, dim3(grid), dim3(threads), 0, st, s.pdl, 1,
-                       (const TY*)Y, tok_ptr, s.T, s.d, per, (TO*)out);
+                       (const TY*)Y, tok_ptr, s.T, s.d, per, (TO*)out, residual,
+                       (int)res_bf16, gate2, s.S);
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const Shape& s, bool y_f32,
-                           bool out_f32, void* out, unsigned* err, int sm_count,
-                           cudaStream_t st) {
+                           bool out_f32, void* out, const void* residual, bool res_bf16,
+                           const float* gate2, unsigned* err, int sm_count, cudaStream_t st) {
   (void)err;
   using bf = __nv_bfloat16;
   if (s.d % 8 != 0) return cudaErrorInvalidValue;
-  if (y_f32 && out_f32) return launch_typed<float, float>(Y, tok_ptr, s, out, sm_count, st);
-  if (y_f32) return launch_typed<float, bf>(Y, tok_ptr, s, out, sm_count, st);
-  if (out_f32) return launch_typed<bf, float>(Y, tok_ptr, s, out, sm_count, st);
-  return launch_typed<bf, bf>(Y, tok_ptr, s, out, sm_count, st);
+  if (y_f32 && out_f32)
+    return launch_typed<float, float>(Y, tok_ptr, s, out, residual, res_bf16, gate2, sm_count,
+                                      st);
+  if (y_f32)
+    return launch_typed<float, bf>(Y, tok_ptr, s, out, residual, res_bf16, gate2, sm_count, st);
+  if (out_f32)
+    return launch_typed<bf, float>(Y, tok_ptr, s, out, residual, res_bf16, gate2, sm_count, st);
+  return launch_typed<bf, bf>(Y, tok_ptr, s, out, residual, res_bf16, gate2, sm_count, st);
 }
 
 }  // namespace nmoe

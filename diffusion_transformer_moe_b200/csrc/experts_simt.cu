@@ -28,7 +28,9 @@ gemm1_simt_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
   pdl_wait();
   const int e = blockIdx.z, m0 = blockIdx.y * kBM, n0 = blockIdx.x * kBN;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  if (tid < kBM) rows[tid] = (m0 + tid < Ce) ? idx[(int64_t)e * Ce + m0 + tid] : -1;
+  // NULL idx: identity row map (the shared expert)
+  if (tid < kBM)
+    rows[tid] = (m0 + tid < Ce) ? (idx ? idx[(int64_t)e * Ce + m0 + tid] : m0 + tid) : -1;
   __syncthreads();
   const T* w1 = W1 + (int64_t)e * d * F;
   const T* w3 = W3 + (int64_t)e * d * F;
@@ -124,7 +126,7 @@ gemm2_simt_kernel(const TH* __restrict__ H, const float* __restrict__ gate,
   for (int i = 0; i < 4; ++i) {
     int s = m0 + ty * 4 + i;
     if (s >= Ce) continue;
-    float w = gate[(int64_t)e * Ce + s];
+    float w = gate ? gate[(int64_t)e * Ce + s] : 1.f;  // NULL gate: weight 1
     const int64_t yrow = ent_pos[(int64_t)e * Ce + s];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {

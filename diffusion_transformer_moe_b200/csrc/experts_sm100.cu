@@ -196,12 +196,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       const uint32_t b_bytes = (uint32_t)(nbox * kBBoxBytes);
       int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
       if (MODE == kGemm1 && !C::kLsuA) {
-        const int32_t* ir = p.idx + (int64_t)e * p.Ce;
+        const int32_t* ir = p.idx + (int64_t)e * p.Ce;  // NULL idx: identity (shared)
         const int s = m0 + 4 * lane;
-        r0 = s + 0 < p.Ce ? ir[s + 0] : 0;
-        r1 = s + 1 < p.Ce ? ir[s + 1] : 0;
-        r2 = s + 2 < p.Ce ? ir[s + 2] : 0;
-        r3 = s + 3 < p.Ce ? ir[s + 3] : 0;
+        r0 = s + 0 < p.Ce ? (p.idx ? ir[s + 0] : s + 0) : 0;
+        r1 = s + 1 < p.Ce ? (p.idx ? ir[s + 1] : s + 1) : 0;
+        r2 = s + 2 < p.Ce ? (p.idx ? ir[s + 2] : s + 2) : 0;
+        r3 = s + 3 < p.Ce ? (p.idx ? ir[s + 3] : s + 3) : 0;
       }
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
@@ -270,7 +270,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       for (int i = 0; i < 8; ++i) {
         const int r = pw * 32 + i * 4 + sub;
         const int s = m0 + r;
-        const int t = s < p.Ce ? p.idx[(int64_t)e * p.Ce + s] : 0;
+        const int t = s < p.Ce ? (p.idx ? p.idx[(int64_t)e * p.Ce + s] : s) : 0;
         src[i] = x + (int64_t)t * p.K + c * 8;
         dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
       }
@@ -415,7 +415,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
           __syncwarp();  // the blocks are read before the next chunk overwrites them
         }
       } else {
-        const float gw = valid ? p.gate[(int64_t)e * p.Ce + s] : 0.f;
+        const float gw = valid ? (p.gate ? p.gate[(int64_t)e * p.Ce + s] : 1.f) : 0.f;
         // staging block of this warp: 16-byte chunk c of row r at r * 128 + (c ^ (r % 8)) * 16
         float* sb = reinterpret_cast<float*>(smem + kStages * C::kStageBytes +
                                              (warp - C::kEpiWarp0) * C::kEpiStage);

@@ -11,6 +11,8 @@ bool experts_sm100_supported(const Shape& s);
 // cp.async (default) or by TMA tile::gather4 (tma_gather).
 // split: H is written as bf16 hi = bf16(h) to H_hi and lo = bf16(h - hi) to H_lo;
 // otherwise only H_hi (bf16(h)) is written.
+// idx NULL: row s of the single expert is token s (the shared expert); gate NULL in
+// gemm2: weight 1.
 cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1,
                                const void* W3, const Shape& s, bool split, bool tma_gather,
                                void* H_hi, void* H_lo, unsigned* err, int sm_count,

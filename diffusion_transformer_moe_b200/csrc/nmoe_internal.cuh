@@ -105,26 +105,33 @@ cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, f
 // bnd: the table launch_select wrote, or NULL to search idx instead.
 // combine == NMOE_COMBINE_NORMALIZED rewrites gate[] in place to
 // route_scale * gate / (sum of the token's gates). ent_pos (may be NULL) receives, for
-// each entry e*Ce + slot, its index in the token-major order of tok_ent.
-cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, int32_t* tok_ptr,
-                       int32_t* tok_ent, int32_t* ent_pos, float* gate, nmoe_combine combine,
-                       float route_scale, unsigned* err, cudaStream_t st);
+// each entry e*Ce + slot, its index in the token-major order of tok_ent. With `shared`,
+// every token's span starts with one more entry, its shared-expert row (tok_ent value
+// E*Ce + t), so tok_ptr[T] = E*Ce + T.
+cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, bool shared,
+                       int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
+                       nmoe_combine combine, float route_scale, unsigned* err,
+                       cudaStream_t st);
 
 // CUDA-core expert GEMMs. dt is the type of x and the weights; h_f32 / y_f32 select
 // fp32 (else dt) for the H and Y intermediates.
+// idx NULL: row s of the single expert is token s (the shared expert).
 cudaError_t launch_gemm1_simt(const void* x, const int32_t* idx, const void* W1, const void* W3,
                               const Shape& s, nmoe_dtype dt, bool h_f32, void* H,
                               cudaStream_t st);
 
-// Row e*Ce + s of the product goes to Y row ent_pos[e*Ce + s] (token-major order).
+// Row e*Ce + s of the product goes to Y row ent_pos[e*Ce + s] (token-major order);
+// gate NULL: weight 1.
 cudaError_t launch_gemm2_simt(const void* H, const float* gate, const void* W2,
                               const int32_t* ent_pos, const Shape& s, nmoe_dtype dt, bool h_f32,
                               bool y_f32, void* Y, cudaStream_t st);
 
 // out[t] = sum of Y rows tok_ptr[t] .. tok_ptr[t+1]-1 (token-major Y, ascending expert);
 // Y is fp32 if y_f32 (else bf16), out fp32 if out_f32.
+// With residual (x's dtype: bf16 if res_bf16, else fp32), out[t] = residual[t] +
+// tanh(clamp(gate2[t / S], -2, 2)) * (that sum), gate2 NULL meaning a gate of 1.
 cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const Shape& s, bool y_f32,
-                           bool out_f32, void* out, unsigned* err, int sm_count,
-                           cudaStream_t st);
+                           bool out_f32, void* out, const void* residual, bool res_bf16,
+                           const float* gate2, unsigned* err, int sm_count, cudaStream_t st);
 
 }  // namespace nmoe

@@ -26,7 +26,8 @@
 // selection call, which has no scratch) the same ranges come from binary searches of
 // each expert's ascending token list. The CTA also records, for every (expert, slot),
 // its position in that token-major order (ent_pos), where the down projection writes
-// the row so that the combine reads each token's rows contiguously.
+// the row so that the combine reads each token's rows contiguously. With a shared expert
+// every token's span starts with its shared-expert row.
 #include "nmoe_internal.cuh"
 
 namespace nmoe {
@@ -333,7 +334,7 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
 
 __global__ void __launch_bounds__(kCsrThreads)
 csr_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ bnd, int Tn, int E,
-           int Ce, int32_t* __restrict__ tok_ptr, int32_t* __restrict__ tok_ent,
+           int Ce, int shared, int32_t* __restrict__ tok_ptr, int32_t* __restrict__ tok_ent,
            int32_t* __restrict__ ent_pos, float* __restrict__ gate, int normalize,
            float route_scale, unsigned* __restrict__ err) {
   pdl_launch_dependents();
@@ -387,6 +388,7 @@ csr_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ bnd, int
     if (w < warp) before += s_wcnt[w];
   }
   if (tid < E) s_beg[tid] = before + inc - cnt;
+  base += shared * t0;  // with a shared expert, one more entry for every earlier token
   __syncthreads();
 
   // scatter the block's entries into the (token, expert) slot map, one per thread
@@ -416,9 +418,9 @@ csr_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ bnd, int
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    s_off[lane] = incl - c;
-    if (t0 + lane < t1) tok_ptr[t0 + lane] = base + incl - c;
-    if (t0 + lane == Tn - 1) tok_ptr[Tn] = base + incl;
+    s_off[lane] = incl - c + shared * lane;   // start of the token's span
+    if (t0 + lane < t1) tok_ptr[t0 + lane] = base + s_off[lane];
+    if (t0 + lane == Tn - 1) tok_ptr[Tn] = base + incl + shared * (lane + 1);
   }
   __syncthreads();
 
@@ -426,6 +428,10 @@ csr_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ bnd, int
   const unsigned lt = lanemask_lt();
   for (int r = warp; r < t1 - t0; r += kCsrWarps) {
     int out = base + s_off[r];
+    if (shared) {  // the shared-expert row comes first
+      if (lane == 0) tok_ent[out] = E * Ce + t0 + r;
+      ++out;
+    }
     const int* srow = s_slot + r * E;
     float tot = 0.f;  // the token's gates summed in ascending expert order, fp32
     for (int e0 = 0; e0 < E; e0 += 32) {
@@ -475,13 +481,14 @@ cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, f
                        (int64_t)s.T, s.S, s.C, s.Ce, s.E, cached, idx, gate, bnd, err);
 }
 
-cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, int32_t* tok_ptr,
-                       int32_t* tok_ent, int32_t* ent_pos, float* gate, nmoe_combine combine,
-                       float route_scale, unsigned* err, cudaStream_t st) {
+cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, bool shared,
+                       int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
+                       nmoe_combine combine, float route_scale, unsigned* err,
+                       cudaStream_t st) {
   size_t smem = sizeof(int) * (size_t)kBlockTok * s.E;
   dim3 grid((unsigned)ceil_div(s.T, kBlockTok));
   return launch_kernel(csr_kernel, grid, dim3(kCsrThreads), smem, st, s.pdl, 1, idx, bnd, s.T,
-                       s.E, s.Ce, tok_ptr, tok_ent, ent_pos, gate,
+                       s.E, s.Ce, (int)shared, tok_ptr, tok_ent, ent_pos, gate,
                        (int)(combine == NMOE_COMBINE_NORMALIZED), route_scale, err);
 }
 

@@ -119,6 +119,22 @@ typedef struct nmoe_options {
   int tma_gather;            /* nonzero: the gate/up GEMM fetches its token rows with TMA
                                 tile::gather4 instead of cp.async (about 2x slower on
                                 B200; kept for comparison) */
+  /* Shared expert (section 6.2: one SwiGLU feed-forward that every token goes through;
+   * the routed, weighted outputs are added onto its output). All NULL: none. Otherwise
+   * device arrays in `dtype`: shared_w1, shared_w3 [d, shared_f], shared_w2
+   * [shared_f, d], row-major, 16-byte aligned; shared_f a multiple of 8 (else
+   * NMOE_ERR_UNSUPPORTED). The page does not give the width; the caller does. */
+  const void* shared_w1;
+  const void* shared_w3;
+  const void* shared_w2;
+  int64_t shared_f;
+  /* Gated residual of the surrounding block (section 6.3: the modulation gates are
+   * clamped to [-2, 2] and passed through tanh). NULL: out = the layer output. Else a
+   * device array [T, d] in `dtype` (it may be x; it must not overlap out), and
+   *   out = residual + tanh(clamp(gate2[segment], -2, 2)) * (layer output),
+   * with gate2 NULL (a gate of 1) or device fp32 [n_segments, d], 16-byte aligned. */
+  const void* residual;
+  const float* gate2;
 } nmoe_options;
 
 /* Fills `o` with the defaults: bf16, softmax, raw combine, route_scale 1, one segment,

@@ -96,6 +96,40 @@ def test_workspace_size_accounts_for_every_buffer():
     assert host32 >= n + 2 * T * d + 4 * T * d
 
 
+def test_workspace_grows_by_the_shared_expert():
+    T, d, E, F, C_, Fs = 8192, 2048, 64, 1024, 128, 1024
+    n = nm.workspace_size(T, d, E, F, C_)
+    m = nm.workspace_size(T, d, E, F, C_, shared_f=Fs)
+    # H hi + lo of the shared expert, one more fp32 Y row and list entry per token
+    extra = 4 * T * Fs + 4 * T * d + 4 * T
+    assert extra <= m - n <= extra + 3 * 256
+
+
+def _forward_ex_status(**kw):
+    a = dict(x=FAKE, W_r=FAKE + 4096, W1=FAKE + 8192, W3=FAKE + 12288, W2=FAKE + 16384,
+             out=FAKE + 32768)
+    o = L.Options()
+    nm.lib().nmoe_options_init(C.byref(o))
+    for k, v in kw.items():
+        setattr(o, k, v)
+    return nm.lib().nmoe_forward_ex(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], 64, 16, 4,
+                                    16, 8, a["out"], None, C.byref(o))
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(shared_w1=FAKE + 65536, shared_f=16), 1),                     # one of three
+    (dict(shared_w1=FAKE + 65536, shared_w3=FAKE + 69632, shared_w2=FAKE + 73728,
+          shared_f=12), 2),                                              # width % 8
+    (dict(shared_w1=FAKE + 65536, shared_w3=FAKE + 69632, shared_w2=FAKE + 73728,
+          shared_f=0), 1),
+    (dict(gate2=FAKE + 65536), 1),                                       # gate without residual
+    (dict(residual=FAKE + 65544), 1),                                    # misaligned
+    (dict(residual=FAKE + 32768), 1),                                    # residual is out
+])
+def test_block_options_are_checked_on_host(kw, expect):
+    assert _forward_ex_status(**kw) == expect
+
+
 def test_missing_gpu_is_reported_not_crashed():
     import torch
     if torch.cuda.is_available():

@@ -163,6 +163,83 @@ def test_router_bias_matches_oracle(dtype):
     _full_parity(a, 16, dtype, dict(n_segments=3, router_bias=bias))
 
 
+# -- shared expert and the block's gated residual (walkthrough sections 6.2 and 6.3) -----
+
+def _block_case(T, d, E, F, Fs, dtype, seed, nseg):
+    a = I.make_small(T, d, E, F, dtype, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    sh = tuple((torch.randn(*shape, generator=g) / shape[0] ** 0.5).to(tdt)
+               for shape in ((d, Fs), (d, Fs), (Fs, d)))
+    res = torch.randn(T, d, generator=g).to(tdt)
+    gate2 = 3.0 * torch.randn(nseg, d, generator=g)  # many gates beyond the +-2 clamp
+    return a, sh, res, gate2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T,d,E,F,Fs,C_,nseg,parts", [
+    (256, 128, 8, 96, 64, 24, 1, ("shared",)),
+    (300, 136, 5, 200, 104, 20, 3, ("shared", "residual", "gate2")),
+    (512, 256, 6, 128, 256, 40, 2, ("residual", "gate2")),
+    (520, 264, 12, 328, 136, 65, 2, ("shared", "residual")),
+    (64, 64, 3, 64, 8, 16, 1, ("shared", "residual", "gate2")),   # CUDA-core shared expert
+])
+def test_shared_expert_and_gated_residual_match_oracle(dtype, T, d, E, F, Fs, C_, nseg, parts):
+    a, sh, res, gate2 = _block_case(T, d, E, F, Fs, dtype, T + Fs, nseg)
+    opts = dict(n_segments=nseg)
+    ref = dict(n_segments=nseg)
+    if "shared" in parts:
+        opts["shared"] = tuple(t.cuda() for t in sh)
+        ref["shared"] = tuple(I.to_numpy_f64(t) for t in sh)
+    if "residual" in parts:
+        opts["residual"] = res.cuda()
+        ref["residual"] = I.to_numpy_f64(res)
+    if "gate2" in parts:
+        opts["gate2"] = gate2.cuda()
+        ref["gate2"] = gate2.double().numpy()
+    out, scores, idx = _run(a, C_, **opts)
+    sel = O.select(scores.cpu().numpy(), C_, nseg)
+    assert np.array_equal(sel, idx.cpu().numpy())
+    r = O.layer(I.to_numpy_f64(a["x"]), I.to_numpy_f64(a["W_r"]), I.to_numpy_f64(a["W1"]),
+                I.to_numpy_f64(a["W3"]), I.to_numpy_f64(a["W2"]), C_, selection=sel, **ref)
+    _check_out(out, r["out"], dtype)
+
+
+def test_residual_may_be_x_and_a_zero_gate_returns_it():
+    a, sh, res, gate2 = _block_case(256, 128, 8, 96, 64, "bf16", 5, 2)
+    x = a["x"].cuda()
+    out = nm.forward(x, a["W_r"].cuda(), a["W1"].cuda(), a["W3"].cuda(), a["W2"].cuda(), 24,
+                     n_segments=2, shared=tuple(t.cuda() for t in sh), residual=x,
+                     gate2=torch.zeros(2, 128, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(out, x)
+
+
+def test_shared_expert_full_1024px_rows_match_oracle():
+    w = I.WORKLOADS["1024px_cfg"]
+    a = I.make_inputs(w)
+    g = torch.Generator().manual_seed(11)
+    Fs = 1024
+    sh = tuple((torch.randn(*shape, generator=g) / shape[0] ** 0.5).to(torch.bfloat16)
+               for shape in ((w.d, Fs), (w.d, Fs), (Fs, w.d)))
+    gate2 = torch.randn(1, w.d, generator=g)
+    dev = {k: v.cuda() for k, v in a.items()}
+    idx = torch.empty(w.E, w.C, device="cuda", dtype=torch.int32)
+    out = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C, idx_out=idx,
+                     shared=tuple(t.cuda() for t in sh), residual=dev["x"],
+                     gate2=gate2.cuda(), out_f32=True)
+    torch.cuda.synchronize()
+    assert nm.get_last_error() == 0
+    sel = idx.cpu().numpy()
+    x = I.to_numpy_f64(a["x"])
+    toks = np.random.default_rng(2).choice(w.T, 96, replace=False)
+    r = O.layer_rows(x, I.to_numpy_f64(a["W_r"]), a["W1"].float().numpy(),
+                     a["W3"].float().numpy(), a["W2"].float().numpy(), w.C, toks,
+                     selection=sel, shared=tuple(I.to_numpy_f64(t) for t in sh),
+                     residual=x, gate2=gate2.double().numpy())
+    _check_out(out[torch.as_tensor(toks, device="cuda")], r["out"], "bf16")
+
+
 # -- invariants on the GPU path --------------------------------------------------------------
 
 def test_unselected_tokens_are_exact_zero_and_each_expert_has_C():
