@@ -46,6 +46,9 @@ def _args():
     ap.add_argument("--intermediate", choices=("split", "bf16"), default="split")
     ap.add_argument("--tma-gather", action="store_true",
                     help="gather the gate/up GEMM's token rows with TMA tile::gather4")
+    ap.add_argument("--shared-f", type=int, default=0,
+                    help="add a shared SwiGLU expert of this width and the block's gated "
+                         "residual (out = x + tanh(clamp(gate2)) * ffn_out)")
     return ap.parse_args()
 
 
@@ -72,11 +75,20 @@ def _workload_config(w, intermediate):
 
 # ---- algorithmic bytes / flops of each stage (minimum traffic the method must move) ----
 
-def stage_bytes(w, intermediate="split"):
-    """Bytes each stage must read + write at least, per layer call."""
+def stage_bytes(w, intermediate="split", shared_f=0):
+    """Bytes each stage must read + write at least, per layer call (with a shared expert
+    of width shared_f: its weights, its H and Y rows, and the residual read)."""
     T, d, E, F, Ce = w.T, w.d, w.E, w.F, w.Ce
     hb = 4 if intermediate == "split" else 2   # H: bf16 hi+lo pair, or bf16
     yb = 4 if intermediate == "split" else 2   # Y: fp32, or bf16
+    Fs = shared_f
+    sh = {"gemm1_swiglu": 2 * 2 * d * Fs + 2 * T * d + hb * T * Fs,
+          "gemm2_scale": 2 * Fs * d + hb * T * Fs + yb * T * d,
+          "combine": yb * T * d + 2 * T * d} if Fs else {}
+    return {k: v + sh.get(k, 0) for k, v in _routed_bytes(T, d, E, F, Ce, hb, yb).items()}
+
+
+def _routed_bytes(T, d, E, F, Ce, hb, yb):
     return {
         "router": 2 * T * d + 2 * d * E + 2 * 4 * T * E,          # x, W_r in; scores, scores_t out
         "select": 4 * T * E + 8 * E * Ce,                          # scores_t in; idx, gate out
@@ -87,12 +99,12 @@ def stage_bytes(w, intermediate="split"):
     }
 
 
-def stage_flops(w, intermediate="split"):
+def stage_flops(w, intermediate="split", shared_f=0):
     """Algorithmic FLOPs of the contractions (the split intermediates' second set of
     down-projection MMAs is executed work, not counted here)."""
-    T, d, E, F, Ce = w.T, w.d, w.E, w.F, w.Ce
-    return {"router": 2 * T * d * E, "gemm1_swiglu": 4 * E * Ce * d * F,
-            "gemm2_scale": 2 * E * Ce * F * d}
+    T, d, E, F, Ce, Fs = w.T, w.d, w.E, w.F, w.Ce, shared_f
+    return {"router": 2 * T * d * E, "gemm1_swiglu": 4 * E * Ce * d * F + 4 * T * d * Fs,
+            "gemm2_scale": 2 * E * Ce * F * d + 2 * T * Fs * d}
 
 
 def _traffic(kernel_stage, workload):
@@ -314,9 +326,18 @@ def run_ours(args, w, rank, world, local_rank, dist):
     W_r, W1, W3, W2 = (a[k].to(dev) for k in ("W_r", "W1", "W3", "W2"))
     inter = args.intermediate
     ws = torch.empty(nm.workspace_size(w.T, w.d, w.E, w.F, w.C, intermediate=inter,
-                                       n_segments=w.segments,
-                                       host_io=True), dtype=torch.uint8, device=dev)
+                                       n_segments=w.segments, host_io=True,
+                                       shared_f=args.shared_f or None),
+                     dtype=torch.uint8, device=dev)
     out = torch.empty_like(x)
+    block = {}
+    if args.shared_f:
+        g = torch.Generator().manual_seed(1000 + rank)
+        Fs = args.shared_f
+        block = dict(shared=tuple((torch.randn(*sh, generator=g) / sh[0] ** 0.5)
+                                  .to(x.dtype).to(dev)
+                                  for sh in ((w.d, Fs), (w.d, Fs), (Fs, w.d))),
+                     residual=x, gate2=torch.randn(w.segments, w.d, generator=g).to(dev))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     K = args.steps
@@ -325,7 +346,7 @@ def run_ours(args, w, rank, world, local_rank, dist):
     def step(tr=None):
         nm.forward(x, W_r, W1, W3, W2, w.C, out=out, workspace=ws, intermediate=inter,
                    n_segments=w.segments,
-                   trace=tr, tma_gather=args.tma_gather)
+                   trace=tr, tma_gather=args.tma_gather, **block)
 
     def barrier():
         if dist is not None:
@@ -371,7 +392,7 @@ def run_ours(args, w, rank, world, local_rank, dist):
     for _ in range(max(1, args.warmup // 2)):
         nm.forward(x_host, W_r, W1, W3, W2, w.C, out=out_host, workspace=ws,
                    n_segments=w.segments,
-                   intermediate=inter, host_io=True, tma_gather=args.tma_gather)
+                   intermediate=inter, host_io=True, tma_gather=args.tma_gather, **block)
     torch.cuda.synchronize()
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
@@ -382,7 +403,7 @@ def run_ours(args, w, rank, world, local_rank, dist):
         e2e_ev[i][0].record(stream)
         nm.forward(x_host, W_r, W1, W3, W2, w.C, out=out_host, workspace=ws,
                    n_segments=w.segments,
-                   intermediate=inter, host_io=True, tma_gather=args.tma_gather)
+                   intermediate=inter, host_io=True, tma_gather=args.tma_gather, **block)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -395,8 +416,8 @@ def run_ours(args, w, rank, world, local_rank, dist):
     peaks = _peaks()
     per_step_s = ms / 1e3 / K
     value = replica_throughput(w.T, world, K, ms)
-    sb = stage_bytes(w, inter)
-    sf = stage_flops(w, inter)
+    sb = stage_bytes(w, inter, args.shared_f)
+    sf = stage_flops(w, inter, args.shared_f)
     stages = {}
     for name, tot in stage_ms.items():
         avg_s = tot / 1e3 / max(ncalls, 1)
@@ -424,13 +445,16 @@ def run_ours(args, w, rank, world, local_rank, dist):
                 "algorithmic_bytes_per_launch": sb[dom],
                 "peak_source": f"{src} hbm_gbs"}
     roof["traffic"] = _traffic(dom, w.name)
-    flops = w.expert_flops() + w.router_flops()
+    flops = w.expert_flops() + w.router_flops() + 6.0 * w.T * w.d * args.shared_f
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(_workload_config(w, inter), parallelism=f"replicas x{world}",
-                       gather="tma gather4" if args.tma_gather else "cp.async"),
+                       gather="tma gather4" if args.tma_gather else "cp.async",
+                       **({"shared_f": args.shared_f,
+                           "block": "x + tanh(clamp(gate2, -2, 2)) * (shared + routed)"}
+                          if args.shared_f else {})),
         "tflops": flops / per_step_s / 1e12,
         "tensor_frac_of_layer": flops / per_step_s / 1e12 / peaks["tensor_sustained"],
         "roofline": roof,
