@@ -10,6 +10,7 @@
 #include <new>
 #include <vector>
 
+#include "csr_block.cuh"
 #include "nmoe_internal.cuh"
 #include "experts_sm100.cuh"
 #include "router_sm100.cuh"
@@ -269,23 +270,28 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   mark(1);
   if (e == cudaSuccess) e = nmoe::launch_select(scores_t, s, idx, gate, bnd, ds->err, st);
   mark(2);
-  if (e == cudaSuccess)
+  const bool tc = !f32 && nmoe::experts_sm100_supported(s);
+  // On the tensor-core path the gate/up GEMM's epilogue warps build the token lists
+  // while their first accumulators fill (no CSR launch); otherwise the CSR kernel does.
+  const bool fuse_csr = tc && nmoe::gemm1_sm100_fuses_csr(s, split);
+  const nmoe::CsrArgs csr = nmoe::csr_args(idx, bnd, s, has_shared, tok_ptr, tok_ent, ent_pos,
+                                           gate, o.combine, o.route_scale, ds->err);
+  if (e == cudaSuccess && !fuse_csr)
     e = nmoe::launch_csr(idx, bnd, s, has_shared, tok_ptr, tok_ent, ent_pos, gate, o.combine,
                          o.route_scale, ds->err, st);
   mark(3);
   const bool tc_sh = has_shared && !f32 && nmoe::experts_sm100_supported(sh);
   if (has_shared && e == cudaSuccess)
     e = tc_sh ? nmoe::launch_gemm1_sm100(xd, nullptr, o.shared_w1, o.shared_w3, sh, split,
-                                         false, Hs, Hs_lo, ds->err, ds->sm_count, st)
+                                         false, Hs, Hs_lo, nullptr, ds->err, ds->sm_count, st)
               : nmoe::launch_gemm1_simt(xd, nullptr, o.shared_w1, o.shared_w3, sh, o.dtype,
                                         split, Hs, st);
-  const bool tc = !f32 && nmoe::experts_sm100_supported(s);
   // SPLIT on the tensor cores: H_hi then H_lo, each [E*Ce, F] bf16; on the CUDA cores
   // (shapes the tcgen05 kernels do not take) H is one fp32 array of the same size.
   void* H_lo = static_cast<char*>(H) + sizeof(uint16_t) * (size_t)s.E * s.Ce * s.F;
   if (e == cudaSuccess)
     e = tc ? nmoe::launch_gemm1_sm100(xd, idx, W1, W3, s, split, o.tma_gather != 0, H, H_lo,
-                                      ds->err, ds->sm_count, st)
+                                      fuse_csr ? &csr : nullptr, ds->err, ds->sm_count, st)
            : nmoe::launch_gemm1_simt(xd, idx, W1, W3, s, o.dtype, split, H, st);
   mark(4);
   if (has_shared && e == cudaSuccess)

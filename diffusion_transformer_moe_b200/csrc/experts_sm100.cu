@@ -38,6 +38,7 @@
 // and returns.
 #include <cudaTypedefs.h>
 
+#include "csr_block.cuh"
 #include "experts_sm100.cuh"
 #include "sm100_ptx.cuh"
 
@@ -90,6 +91,10 @@ struct Params {
   const int32_t* ent_pos;  // gemm2: Y row of entry e*Ce + s (token-major order)
   void* out;             // gemm1: H (hi) [E*Ce, F] bf16; gemm2: Y [E*Ce, d] (fp32 if SPLIT)
   void* out_lo;          // gemm1 with SPLIT: H lo [E*Ce, F] bf16
+  // gemm1: csr_blocks > 0 builds the token lists' blocks in the epilogue warps before
+  // the first tile's accumulator is ready (their staging memory is free until then)
+  CsrArgs csr;
+  int csr_blocks;
   unsigned* err;
 };
 
@@ -337,6 +342,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     __syncwarp();  // the warp reconverges before the block barrier and the TMEM release
   } else if (warp >= C::kEpiWarp0) {
     // ---------------- epilogue: eight warps, two per TMEM lane quarter ----------------
+    if (MODE == kGemm1 && p.csr_blocks > 0) {
+      static_assert(C::kEpiWarps * 32 == kCsrThreads, "one CSR block per epilogue");
+      uint8_t* cs = smem + kStages * C::kStageBytes;
+      const int et = threadIdx.x - 32 * C::kEpiWarp0;
+      for (int blk = blockIdx.x; blk < p.csr_blocks; blk += gridDim.x)
+        csr_block(blk, p.csr, cs, et, []() { asm volatile("bar.sync 1, 256;" ::: "memory"); });
+    }
     const int q = warp & 3;                         // TMEM lane quarter this warp may access
     const int half = (warp - C::kEpiWarp0) >> 2;    // which half of the columns
     const int row = q * 32 + lane;                  // accumulator row = tile row
@@ -553,10 +565,18 @@ bool experts_sm100_supported(const Shape& s) {
          s.F % 8 == 0 && encode_fn() != nullptr;
 }
 
+bool gemm1_sm100_fuses_csr(const Shape& s, bool split) {
+  const size_t room = split ? Cfg<kGemm1, true, kGatherLsu>::kEpiWarps *
+                                  (size_t)Cfg<kGemm1, true, kGatherLsu>::kEpiStage
+                            : Cfg<kGemm1, false, kGatherLsu>::kEpiWarps *
+                                  (size_t)Cfg<kGemm1, false, kGatherLsu>::kEpiStage;
+  return csr_smem_bytes(s.E) <= room;
+}
+
 cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1,
                                const void* W3, const Shape& s, bool split, bool tma_gather,
-                               void* H_hi, void* H_lo, unsigned* err, int sm_count,
-                               cudaStream_t st) {
+                               void* H_hi, void* H_lo, const CsrArgs* csr, unsigned* err,
+                               int sm_count, cudaStream_t st) {
   CUtensorMap ma, mb0, mb1;
   if (!rows_map(&ma, x, s.T, s.d, 1) || !weight_map(&mb0, W1, s.E, s.d, s.F) ||
       !weight_map(&mb1, W3, s.E, s.d, s.F))
@@ -568,6 +588,12 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
   split_tail(p, sm_count);
   p.idx = idx; p.gate = nullptr; p.ent_pos = nullptr; p.out = H_hi; p.out_lo = H_lo;
+  p.csr_blocks = 0;
+  if (csr != nullptr) {
+    if (!gemm1_sm100_fuses_csr(s, split)) return cudaErrorInvalidValue;
+    p.csr = *csr;
+    p.csr_blocks = (int)ceil_div(s.T, kCsrBlockTok);
+  }
   p.err = err;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (tma_gather)
@@ -593,6 +619,7 @@ cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* 
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
   split_tail(p, sm_count);
   p.idx = nullptr; p.gate = gate; p.ent_pos = ent_pos; p.out = Y; p.out_lo = nullptr;
+  p.csr_blocks = 0;
   p.err = err;
   return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl)
                : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl);

@@ -12,14 +12,16 @@ bool experts_sm100_supported(const Shape& s);
 // split: H is written as bf16 hi = bf16(h) to H_hi and lo = bf16(h - hi) to H_lo;
 // otherwise only H_hi (bf16(h)) is written.
 // idx NULL: row s of the single expert is token s (the shared expert); gate NULL in
-// gemm2: weight 1.
+// gemm2: weight 1. csr (may be NULL; only if gemm1_sm100_fuses_csr) also builds the
+// token lists inside the gate/up GEMM, in place of the CSR kernel.
+struct CsrArgs;
+bool gemm1_sm100_fuses_csr(const Shape& s, bool split);
 cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1,
                                const void* W3, const Shape& s, bool split, bool tma_gather,
-                               void* H_hi, void* H_lo, unsigned* err, int sm_count,
-                               cudaStream_t st);
+                               void* H_hi, void* H_lo, const CsrArgs* csr, unsigned* err,
+                               int sm_count, cudaStream_t st);
 
-// Y[ent_pos[e*Ce + s], :] = gate[e, s] * (H[e, s, :] W2_e). split: H = H_hi + H_lo and
-// Y is fp32; otherwise H = H_hi and Y is bf16.
+// Row e*Ce + s of H W2_e, times gate[e, s], goes to Y row ent_pos[e*Ce + s].
 cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
                                const int32_t* ent_pos, const void* W2, const Shape& s,
                                bool split, void* Y, unsigned* err, int sm_count,

@@ -112,6 +112,11 @@ cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, b
                        int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
                        nmoe_combine combine, float route_scale, unsigned* err,
                        cudaStream_t st);
+// The same arguments, for a kernel that builds the lists itself (csr_block.cuh).
+struct CsrArgs;
+CsrArgs csr_args(const int32_t* idx, const int32_t* bnd, const Shape& s, bool shared,
+                 int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
+                 nmoe_combine combine, float route_scale, unsigned* err);
 
 // CUDA-core expert GEMMs. dt is the type of x and the weights; h_f32 / y_f32 select
 // fp32 (else dt) for the H and Y intermediates.

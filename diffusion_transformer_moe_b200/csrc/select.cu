@@ -19,15 +19,11 @@
 // ascending token order, and, for every block of kBlockTok tokens, how many of the
 // expert's entries come before the block (the boundary table).
 //
-// csr_kernel: one CTA per kBlockTok consecutive tokens. The boundary table gives, for
-// every expert, the slot range [lo, hi) of its entries inside the block, and the sum of
-// the lo's is the block's offset in the token-major order: one coalesced load round, no
-// global scan and no atomics on global memory. Without the table (the standalone
-// selection call, which has no scratch) the same ranges come from binary searches of
-// each expert's ascending token list. The CTA also records, for every (expert, slot),
-// its position in that token-major order (ent_pos), where the down projection writes
-// the row so that the combine reads each token's rows contiguously. With a shared expert
-// every token's span starts with its shared-expert row.
+// csr_kernel: one CTA per kBlockTok consecutive tokens runs csr_block (csr_block.cuh)
+// from the boundary table; the standalone selection call, which has no scratch for the
+// table, searches each expert's ascending token list instead. On the tensor-core path
+// of the whole layer the same blocks are built inside the gate/up GEMM instead.
+#include "csr_block.cuh"
 #include "nmoe_internal.cuh"
 
 namespace nmoe {
@@ -319,149 +315,13 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
   }
 }
 
-constexpr int kCsrThreads = 256;
-constexpr int kCsrWarps = kCsrThreads / 32;
-static_assert(kCsrThreads >= 256, "one thread per expert (E <= 256)");
+static_assert(kBlockTok == kCsrBlockTok, "the boundary table is per CSR block");
 
-__device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    int mid = (lo + hi) >> 1;
-    if (a[mid] < v) lo = mid + 1; else hi = mid;
-  }
-  return lo;
-}
-
-__global__ void __launch_bounds__(kCsrThreads)
-csr_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ bnd, int Tn, int E,
-           int Ce, int shared, int32_t* __restrict__ tok_ptr, int32_t* __restrict__ tok_ent,
-           int32_t* __restrict__ ent_pos, float* __restrict__ gate, int normalize,
-           float route_scale, unsigned* __restrict__ err) {
+__global__ void __launch_bounds__(kCsrThreads) csr_kernel(const CsrArgs a) {
   pdl_launch_dependents();
-  extern __shared__ int s_slot[];  // [kBlockTok][E]: slot of (token, expert) or -1
-  __shared__ int s_lo[256], s_beg[256];
-  __shared__ int s_wlo[kCsrWarps], s_wcnt[kCsrWarps];
-  __shared__ int s_cnt[kBlockTok], s_off[kBlockTok];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int blk = blockIdx.x;
-  const int t0 = blk * kBlockTok;
-  const int t1 = min(Tn, t0 + kBlockTok);
-
-  for (int i = tid; i < kBlockTok * E; i += kCsrThreads) s_slot[i] = -1;
-  if (tid < kBlockTok) s_cnt[tid] = 0;
+  extern __shared__ __align__(16) uint8_t s_csr[];
   pdl_wait();
-
-  // slot range [lo, lo + cnt) of expert `tid` inside the block
-  int lo = 0, cnt = 0;
-  if (tid < E) {
-    if (bnd != nullptr) {
-      lo = bnd[(int64_t)blk * E + tid];
-      cnt = bnd[(int64_t)(blk + 1) * E + tid] - lo;
-    } else {
-      const int32_t* row = idx + (int64_t)tid * Ce;
-      lo = lower_bound_i32(row, Ce, t0);
-      cnt = lower_bound_i32(row, Ce, t1) - lo;
-    }
-    if (lo < 0 || cnt < 0 || lo + cnt > Ce) {  // not a table the selection wrote
-      atomicOr(err, kErrDeviceCheck);
-      lo = 0;
-      cnt = 0;
-    }
-    s_lo[tid] = lo;
-  }
-  // exclusive scan of cnt over the experts; sum of lo = entries before the block
-  int inc = cnt, part = lo;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += v;
-    part += __shfl_xor_sync(0xffffffffu, part, o);
-  }
-  if (lane == 31) s_wcnt[warp] = inc;
-  if (lane == 0) s_wlo[warp] = part;
-  __syncthreads();
-  int base = 0, total = 0, before = 0;
-#pragma unroll
-  for (int w = 0; w < kCsrWarps; ++w) {
-    base += s_wlo[w];
-    total += s_wcnt[w];
-    if (w < warp) before += s_wcnt[w];
-  }
-  if (tid < E) s_beg[tid] = before + inc - cnt;
-  base += shared * t0;  // with a shared expert, one more entry for every earlier token
-  __syncthreads();
-
-  // scatter the block's entries into the (token, expert) slot map, one per thread
-  for (int j = tid; j < total; j += kCsrThreads) {
-    int a = 0, b = E - 1;  // last expert whose first flat entry is <= j
-    while (a < b) {
-      const int mid = (a + b + 1) >> 1;
-      if (s_beg[mid] <= j) a = mid; else b = mid - 1;
-    }
-    const int sl = s_lo[a] + (j - s_beg[a]);
-    const int t = idx[(int64_t)a * Ce + sl];
-    if (t >= t0 && t < t1) {
-      s_slot[(t - t0) * E + a] = sl;
-      atomicAdd(&s_cnt[t - t0], 1);
-    } else {
-      atomicOr(err, kErrDeviceCheck);
-    }
-  }
-  __syncthreads();
-
-  // per-token offsets (one warp: kBlockTok == 32)
-  if (warp == 0) {
-    const int c = s_cnt[lane];
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    s_off[lane] = incl - c + shared * lane;   // start of the token's span
-    if (t0 + lane < t1) tok_ptr[t0 + lane] = base + s_off[lane];
-    if (t0 + lane == Tn - 1) tok_ptr[Tn] = base + incl + shared * (lane + 1);
-  }
-  __syncthreads();
-
-  // entries of each token in ascending expert order: one warp per token
-  const unsigned lt = lanemask_lt();
-  for (int r = warp; r < t1 - t0; r += kCsrWarps) {
-    int out = base + s_off[r];
-    if (shared) {  // the shared-expert row comes first
-      if (lane == 0) tok_ent[out] = E * Ce + t0 + r;
-      ++out;
-    }
-    const int* srow = s_slot + r * E;
-    float tot = 0.f;  // the token's gates summed in ascending expert order, fp32
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      const int sl = e < E ? srow[e] : -1;
-      const unsigned m = __ballot_sync(0xffffffffu, sl >= 0);
-      if (sl >= 0) {
-        const int at = out + __popc(m & lt);
-        tok_ent[at] = e * Ce + sl;
-        if (ent_pos != nullptr) ent_pos[e * Ce + sl] = at;
-      }
-      if (normalize) {
-        const float v = sl >= 0 ? gate[(int64_t)e * Ce + sl] : 0.f;
-        for (unsigned mm = m; mm != 0u; mm &= mm - 1u)
-          tot += __shfl_sync(0xffffffffu, v, __ffs(mm) - 1);
-      }
-      out += __popc(m);
-    }
-    if (normalize) {
-      // every entry belongs to one token, so this lane alone reads and rewrites it
-      for (int e0 = 0; e0 < E; e0 += 32) {
-        const int e = e0 + lane;
-        const int sl = e < E ? srow[e] : -1;
-        if (sl >= 0) {
-          float* gp = gate + (int64_t)e * Ce + sl;
-          *gp = route_scale * (*gp / tot);
-        }
-      }
-    }
-  }
+  csr_block(blockIdx.x, a, s_csr, threadIdx.x, []() { __syncthreads(); });
 }
 
 }  // namespace
@@ -485,11 +345,22 @@ cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, b
                        int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
                        nmoe_combine combine, float route_scale, unsigned* err,
                        cudaStream_t st) {
-  size_t smem = sizeof(int) * (size_t)kBlockTok * s.E;
+  const CsrArgs a = csr_args(idx, bnd, s, shared, tok_ptr, tok_ent, ent_pos, gate, combine,
+                             route_scale, err);
   dim3 grid((unsigned)ceil_div(s.T, kBlockTok));
-  return launch_kernel(csr_kernel, grid, dim3(kCsrThreads), smem, st, s.pdl, 1, idx, bnd, s.T,
-                       s.E, s.Ce, (int)shared, tok_ptr, tok_ent, ent_pos, gate,
-                       (int)(combine == NMOE_COMBINE_NORMALIZED), route_scale, err);
+  return launch_kernel(csr_kernel, grid, dim3(kCsrThreads), csr_smem_bytes(s.E), st, s.pdl, 1,
+                       a);
+}
+
+CsrArgs csr_args(const int32_t* idx, const int32_t* bnd, const Shape& s, bool shared,
+                 int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
+                 nmoe_combine combine, float route_scale, unsigned* err) {
+  CsrArgs a;
+  a.idx = idx; a.bnd = bnd; a.T = s.T; a.E = s.E; a.Ce = s.Ce; a.shared = shared ? 1 : 0;
+  a.tok_ptr = tok_ptr; a.tok_ent = tok_ent; a.ent_pos = ent_pos; a.gate = gate;
+  a.normalize = combine == NMOE_COMBINE_NORMALIZED ? 1 : 0;
+  a.route_scale = route_scale; a.err = err;
+  return a;
 }
 
 }  // namespace nmoe
