@@ -32,7 +32,7 @@ EXPORTS = (
     "nmoe_options_init", "nmoe_router", "nmoe_select", "nmoe_forward", "nmoe_forward_ex",
     "nmoe_workspace_size", "nmoe_get_last_error", "nmoe_status_str", "nmoe_trace_create",
     "nmoe_trace_read", "nmoe_trace_reset", "nmoe_trace_destroy", "nmoe_stage_name",
-    "nmoe_build_info", "nmoe_forward_noalloc",
+    "nmoe_build_info", "nmoe_forward_noalloc", "nmoe_kernels_per_call",
 )
 
 
@@ -105,6 +105,8 @@ def lib() -> C.CDLL:
             L.nmoe_build_info.restype = C.c_char_p
             L.nmoe_forward_noalloc.argtypes = [_vp] * 5 + [_i64] * 5 + [_vp, _vp]
             L.nmoe_forward_noalloc.restype = C.c_int
+            L.nmoe_kernels_per_call.argtypes = [_i64] * 5 + [C.POINTER(Options)]
+            L.nmoe_kernels_per_call.restype = C.c_int
             _lib = L
     return _lib
 
@@ -240,6 +242,12 @@ def forward(x, W_r, W1, W3, W2, C_: int, out=None, stream=None, **opts):
 def workspace_size(T, d, E, F, C_, **opts) -> int:
     o = options(**opts)
     return int(lib().nmoe_workspace_size(T, d, E, F, C_, C.byref(o)))
+
+
+def kernels_per_call(T, d, E, F, C_, **opts) -> int:
+    """How many kernels one layer call with these sizes and options launches."""
+    o = options(**opts)
+    return int(lib().nmoe_kernels_per_call(T, d, E, F, C_, C.byref(o)))
 
 
 def get_last_error(stream=None) -> int:

@@ -416,6 +416,19 @@ nmoe_status nmoe_forward_ex(const void* x, const void* W_r, const void* W1, cons
                       static_cast<cudaStream_t>(stream), opts ? *opts : default_options());
 }
 
+int nmoe_kernels_per_call(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
+                          const nmoe_options* opts) {
+  const nmoe_options o = opts ? *opts : default_options();
+  if (check_shape(T, d, E, F, C, o.n_segments, o.dtype, true) != NMOE_OK) return 0;
+  const Shape s = make_shape(T, d, E, F, C, o.n_segments);
+  const bool f32 = o.dtype == NMOE_F32;
+  const bool split = !f32 && o.intermediate == NMOE_INTERMEDIATE_SPLIT;
+  const bool tc = !f32 && nmoe::experts_sm100_supported(s);
+  const bool fuse_csr = tc && nmoe::gemm1_sm100_fuses_csr(s, split);
+  // router, select, (CSR), gate/up, down, combine; two more for a shared expert
+  return 5 + (fuse_csr ? 0 : 1) + (o.shared_w1 != nullptr ? 2 : 0);
+}
+
 size_t nmoe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
                            const nmoe_options* opts) {
   const nmoe_options o = opts ? *opts : default_options();

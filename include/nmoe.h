@@ -185,6 +185,13 @@ NMOE_API nmoe_status nmoe_forward_ex(const void* x, const void* W_r, const void*
 NMOE_API size_t nmoe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
                            const nmoe_options* opts);
 
+/* Number of kernels one nmoe_forward_ex call with these sizes and options launches
+ * (0 for invalid sizes): the router, the selection, the token lists (inside the gate/up
+ * GEMM on the tensor-core path, else a kernel of their own), the gate/up and down GEMMs
+ * (twice with a shared expert) and the combine. Pure host logic; no device access. */
+NMOE_API int nmoe_kernels_per_call(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
+                                   const nmoe_options* opts);
+
 /* Waits for `stream`, then returns and clears the current device's error word
  * (NMOE_OK, NMOE_ERR_TIMEOUT or NMOE_ERR_DEVICE_CHECK), or NMOE_ERR_CUDA if the stream
  * itself reported an error. */

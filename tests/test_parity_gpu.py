@@ -205,6 +205,13 @@ def test_shared_expert_and_gated_residual_match_oracle(dtype, T, d, E, F, Fs, C_
     _check_out(out, r["out"], dtype)
 
 
+def test_tensor_core_path_launches_five_kernels():
+    # router, select, gate/up GEMM (which also builds the token lists), down GEMM, combine
+    assert nm.kernels_per_call(8192, 2048, 64, 1024, 128) == 5
+    assert nm.kernels_per_call(8192, 2048, 64, 1024, 128, shared_f=1024) == 7
+    assert nm.kernels_per_call(256, 256, 8, 512, 32, dtype=1) == 6  # fp32: CSR kernel
+
+
 def test_residual_may_be_x_and_a_zero_gate_returns_it():
     a, sh, res, gate2 = _block_case(256, 128, 8, 96, 64, "bf16", 5, 2)
     x = a["x"].cuda()
