@@ -116,6 +116,7 @@ def _full_parity(a, C_, dtype, opts=None):
     (64, 64, 1, 64, 64),         # one expert, full capacity: the dense SwiGLU
     (96, 32, 7, 40, 1),          # capacity 1
     (128, 512, 3, 136, 128),     # C = T: every expert takes every token
+    (512, 128, 256, 64, 4),      # 256 experts: the token lists need their own kernel
 ])
 def test_small_shapes_match_oracle(dtype, T, d, E, F, C_):
     a = I.make_small(T, d, E, F, dtype, seed=T + d + E)
