@@ -206,6 +206,26 @@ def test_shared_expert_and_gated_residual_match_oracle(dtype, T, d, E, F, Fs, C_
     _check_out(out, r["out"], dtype)
 
 
+def test_repeated_calls_with_and_without_stage_events_stay_clean():
+    # calls back to back (programmatic dependent launch) and with events between the
+    # stages (plain launches): no bounded wait may run out, in either form
+    w = I.WORKLOADS["512px_cfg"]
+    a = I.make_inputs(w)
+    dev = {k: v.cuda() for k, v in a.items()}
+    ws = torch.empty(nm.workspace_size(w.T, w.d, w.E, w.F, w.C), dtype=torch.uint8,
+                     device="cuda")
+    ref = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C, workspace=ws)
+    torch.cuda.synchronize()
+    for traced in (False, True):
+        for _ in range(12):
+            tr = nm.Trace(1) if traced else None
+            out = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C,
+                             workspace=ws, trace=tr)
+            torch.cuda.synchronize()
+            assert nm.get_last_error() == 0
+            assert torch.equal(out, ref)
+
+
 def test_tensor_core_path_launches_five_kernels():
     # router, select, gate/up GEMM (which also builds the token lists), down GEMM, combine
     assert nm.kernels_per_call(8192, 2048, 64, 1024, 128) == 5
