@@ -33,6 +33,8 @@ EXPORTS = (
     "nmoe_workspace_size", "nmoe_get_last_error", "nmoe_status_str", "nmoe_trace_create",
     "nmoe_trace_read", "nmoe_trace_reset", "nmoe_trace_destroy", "nmoe_stage_name",
     "nmoe_build_info", "nmoe_forward_noalloc", "nmoe_kernels_per_call",
+    "nmoe_workspace_offsets", "nmoe_ep_rows", "nmoe_rows_gather", "nmoe_rows_scatter",
+    "nmoe_combine_tokens",
 )
 
 
@@ -51,7 +53,8 @@ class Options(C.Structure):
         ("trace", C.c_void_p), ("intermediate", C.c_int), ("out_f32", C.c_int),
         ("tma_gather", C.c_int), ("shared_w1", C.c_void_p), ("shared_w3", C.c_void_p),
         ("shared_w2", C.c_void_p), ("shared_f", C.c_int64), ("residual", C.c_void_p),
-        ("gate2", C.c_void_p),
+        ("gate2", C.c_void_p), ("expert_begin", C.c_int64), ("expert_end", C.c_int64),
+        ("skip_combine", C.c_int),
     ]
 
 
@@ -107,6 +110,18 @@ def lib() -> C.CDLL:
             L.nmoe_forward_noalloc.restype = C.c_int
             L.nmoe_kernels_per_call.argtypes = [_i64] * 5 + [C.POINTER(Options)]
             L.nmoe_kernels_per_call.restype = C.c_int
+            L.nmoe_workspace_offsets.argtypes = [_i64] * 5 + [C.POINTER(Options)] + [
+                C.POINTER(C.c_size_t)] * 3
+            L.nmoe_workspace_offsets.restype = C.c_int
+            L.nmoe_ep_rows.argtypes = [_vp, _vp] + [_i64] * 7 + [_vp, _vp, _vp]
+            L.nmoe_ep_rows.restype = C.c_int
+            L.nmoe_rows_gather.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp]
+            L.nmoe_rows_gather.restype = C.c_int
+            L.nmoe_rows_scatter.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp]
+            L.nmoe_rows_scatter.restype = C.c_int
+            L.nmoe_combine_tokens.argtypes = [_vp, _vp] + [_i64] * 4 + [C.c_int, C.c_int, _vp,
+                                                                         _vp]
+            L.nmoe_combine_tokens.restype = C.c_int
             _lib = L
     return _lib
 
@@ -122,6 +137,14 @@ def _dt(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return NMOE_F32
     raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dt_code(dtype: torch.dtype) -> int:
+    if dtype == torch.bfloat16:
+        return NMOE_BF16
+    if dtype == torch.float32:
+        return NMOE_F32
+    raise TypeError(f"unsupported dtype {dtype}")
 
 
 def _ptr(t):
@@ -144,7 +167,7 @@ def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
             n_segments=1, router_bias=None, workspace=None, scores_out=None, idx_out=None,
             host_io=False, trace=None, intermediate="split", out_f32=False,
             tma_gather=False, shared=None, shared_f=None, residual=None,
-            gate2=None) -> Options:
+            gate2=None, expert_begin=0, expert_end=0, skip_combine=False) -> Options:
     """nmoe_options from keyword arguments. ``shared`` = (Ws1 [d,Fs], Ws3 [d,Fs],
     Ws2 [Fs,d]) device tensors adds the shared expert; ``shared_f`` alone (no tensors)
     only sizes a workspace for one. ``residual`` [T,d] and ``gate2`` fp32
@@ -179,6 +202,9 @@ def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
         o.shared_f = int(shared_f)
     o.residual = _ptr(residual)
     o.gate2 = _ptr(gate2)
+    o.expert_begin = int(expert_begin)
+    o.expert_end = int(expert_end)
+    o.skip_combine = 1 if skip_combine else 0
     return o
 
 

@@ -166,6 +166,12 @@ nmoe_status options_ok(const nmoe_options& o) {
     if (o.shared_f % 8 != 0) return NMOE_ERR_UNSUPPORTED;
   }
   if (o.gate2 && !o.residual) return NMOE_ERR_INVALID_ARG;
+  const bool ep = o.expert_end > o.expert_begin || o.skip_combine;
+  if (ep && (n_shared != 0 || o.residual != nullptr)) return NMOE_ERR_INVALID_ARG;
+  if (o.expert_begin < 0 || o.expert_end < 0) return NMOE_ERR_INVALID_ARG;
+  if (o.skip_combine && (o.workspace == nullptr || o.host_io)) return NMOE_ERR_INVALID_ARG;
+  // a rank's partial rows are only a layer output after the exchange
+  if (o.expert_end > o.expert_begin && !o.skip_combine) return NMOE_ERR_INVALID_ARG;
   if (o.residual && !aligned16(o.residual)) return NMOE_ERR_INVALID_ARG;
   if (o.gate2 && !aligned16(o.gate2)) return NMOE_ERR_INVALID_ARG;
   return NMOE_OK;
@@ -192,10 +198,12 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   nmoe_status v = check_shape(T, d, E, F, C, o.n_segments, o.dtype, true);
   if (v != NMOE_OK) return v;
   if ((v = options_ok(o)) != NMOE_OK) return v;
-  if (!x || !W_r || !W1 || !W3 || !W2 || !out) return NMOE_ERR_INVALID_ARG;
+  // with skip_combine the call writes no output, and out may be NULL
+  if (!x || !W_r || !W1 || !W3 || !W2 || (!out && !o.skip_combine))
+    return NMOE_ERR_INVALID_ARG;
   if (!aligned16(W_r) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2))
     return NMOE_ERR_INVALID_ARG;
-  if (!o.host_io && (!aligned16(x) || !aligned16(out))) return NMOE_ERR_INVALID_ARG;
+  if (!o.host_io && (!aligned16(x) || (out && !aligned16(out)))) return NMOE_ERR_INVALID_ARG;
   if (x == out) return NMOE_ERR_INVALID_ARG;
   if (o.residual != nullptr && o.residual == out) return NMOE_ERR_INVALID_ARG;
 
@@ -204,6 +212,10 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   Shape s = make_shape(T, d, E, F, C, o.n_segments);
   if (s.Ce > 65535 * 64) return NMOE_ERR_UNSUPPORTED;
   const bool has_shared = o.shared_w1 != nullptr;
+  // the experts this call runs (all, or one rank's range under expert parallelism)
+  const int e_lo = o.expert_end > o.expert_begin ? (int)o.expert_begin : 0;
+  const int e_hi = o.expert_end > o.expert_begin ? (int)o.expert_end : (int)E;
+  if (e_hi > E) return NMOE_ERR_INVALID_ARG;
   if (has_shared && (int64_t)s.E * s.Ce + s.T >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
   // per-stage events sit between the launches, so traced calls run without overlap
   s.pdl = o.trace == nullptr;
@@ -270,7 +282,12 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   mark(1);
   if (e == cudaSuccess) e = nmoe::launch_select(scores_t, s, idx, gate, bnd, ds->err, st);
   mark(2);
-  const bool tc = !f32 && nmoe::experts_sm100_supported(s);
+  // the expert GEMMs cover experts [e_lo, e_hi): their slice of idx, gate and ent_pos
+  Shape sl = s;
+  sl.E = e_hi - e_lo;
+  const int64_t eoff = (int64_t)e_lo * s.Ce;
+  const bool run_experts = sl.E > 0;
+  const bool tc = !f32 && run_experts && nmoe::experts_sm100_supported(sl);
   // On the tensor-core path the gate/up GEMM's epilogue warps build the token lists
   // while their first accumulators fill (no CSR launch); otherwise the CSR kernel does.
   const bool fuse_csr = tc && nmoe::gemm1_sm100_fuses_csr(s, split);
@@ -289,22 +306,24 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   // SPLIT on the tensor cores: H_hi then H_lo, each [E*Ce, F] bf16; on the CUDA cores
   // (shapes the tcgen05 kernels do not take) H is one fp32 array of the same size.
   void* H_lo = static_cast<char*>(H) + sizeof(uint16_t) * (size_t)s.E * s.Ce * s.F;
-  if (e == cudaSuccess)
-    e = tc ? nmoe::launch_gemm1_sm100(xd, idx, W1, W3, s, split, o.tma_gather != 0, H, H_lo,
-                                      fuse_csr ? &csr : nullptr, ds->err, ds->sm_count, st)
-           : nmoe::launch_gemm1_simt(xd, idx, W1, W3, s, o.dtype, split, H, st);
+  if (e == cudaSuccess && run_experts)
+    e = tc ? nmoe::launch_gemm1_sm100(xd, idx + eoff, W1, W3, sl, split, o.tma_gather != 0, H,
+                                      H_lo, fuse_csr ? &csr : nullptr, ds->err, ds->sm_count,
+                                      st)
+           : nmoe::launch_gemm1_simt(xd, idx + eoff, W1, W3, sl, o.dtype, split, H, st);
   mark(4);
   if (has_shared && e == cudaSuccess)
     e = tc_sh ? nmoe::launch_gemm2_sm100(Hs, Hs_lo, nullptr, tok_ptr, o.shared_w2, sh, split,
                                          Y, ds->err, ds->sm_count, st)
               : nmoe::launch_gemm2_simt(Hs, nullptr, o.shared_w2, tok_ptr, sh, o.dtype, split,
                                         y_f32, Y, st);
-  if (e == cudaSuccess)
-    e = tc ? nmoe::launch_gemm2_sm100(H, H_lo, gate, ent_pos, W2, s, split, Y, ds->err,
-                                      ds->sm_count, st)
-           : nmoe::launch_gemm2_simt(H, gate, W2, ent_pos, s, o.dtype, split, y_f32, Y, st);
+  if (e == cudaSuccess && run_experts)
+    e = tc ? nmoe::launch_gemm2_sm100(H, H_lo, gate + eoff, ent_pos + eoff, W2, sl, split, Y,
+                                      ds->err, ds->sm_count, st)
+           : nmoe::launch_gemm2_simt(H, gate + eoff, W2, ent_pos + eoff, sl, o.dtype, split,
+                                     y_f32, Y, st);
   mark(5);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess && !o.skip_combine)
     e = nmoe::launch_combine(Y, tok_ptr, s, y_f32, out_f32, outd, o.residual, !f32, o.gate2,
                              ds->err, ds->sm_count, st);
   mark(6);
@@ -348,6 +367,9 @@ void nmoe_options_init(nmoe_options* o) {
   o->shared_f = 0;
   o->residual = nullptr;
   o->gate2 = nullptr;
+  o->expert_begin = 0;
+  o->expert_end = 0;
+  o->skip_combine = 0;
 }
 
 nmoe_status nmoe_router(const void* x, const void* W_r, int64_t T, int64_t d, int64_t E,
@@ -416,6 +438,94 @@ nmoe_status nmoe_forward_ex(const void* x, const void* W_r, const void* W1, cons
                       static_cast<cudaStream_t>(stream), opts ? *opts : default_options());
 }
 
+nmoe_status nmoe_workspace_offsets(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
+                                   const nmoe_options* opts, size_t* y_offset,
+                                   size_t* tok_ptr_offset, size_t* tok_ent_offset) {
+  const nmoe_options o = opts ? *opts : default_options();
+  if (check_shape(T, d, E, F, C, o.n_segments, o.dtype, true) != NMOE_OK)
+    return NMOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(make_shape(T, d, E, F, C, o.n_segments), o.dtype, o);
+  if (y_offset) *y_offset = L.Y;
+  if (tok_ptr_offset) *tok_ptr_offset = L.tok_ptr;
+  if (tok_ent_offset) *tok_ent_offset = L.tok_ent;
+  return NMOE_OK;
+}
+
+nmoe_status nmoe_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent, int64_t T, int64_t E,
+                         int64_t Ce, int64_t t_begin, int64_t t_end, int64_t e_begin,
+                         int64_t e_end, int32_t* rows, int32_t* count, nmoe_stream_t stream) {
+  if (!tok_ptr || !tok_ent || !rows || !count) return NMOE_ERR_INVALID_ARG;
+  if (T < 1 || E < 1 || Ce < 1 || E * Ce >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
+  if (t_begin < 0 || t_end < t_begin || t_end > T) return NMOE_ERR_INVALID_ARG;
+  if (e_begin < 0 || e_end < e_begin || e_end > E) return NMOE_ERR_INVALID_ARG;
+  DevState* ds = nullptr;
+  nmoe_status v = dev_state(&ds);
+  if (v != NMOE_OK) return v;
+  if (nmoe::launch_ep_rows(tok_ptr, tok_ent, (int)E, (int)Ce, (int)t_begin, (int)t_end,
+                           (int)e_begin, (int)e_end, rows, count,
+                           static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return NMOE_ERR_CUDA;
+  }
+  return NMOE_OK;
+}
+
+namespace {
+nmoe_status rows_copy(const void* src, const int32_t* rows, int64_t n, int64_t row_bytes,
+                      void* dst, bool gather, nmoe_stream_t stream) {
+  if (n < 0 || row_bytes < 16 || row_bytes % 16 != 0) return NMOE_ERR_INVALID_ARG;
+  if (n > 0 && (!src || !rows || !dst || !aligned16(src) || !aligned16(dst)))
+    return NMOE_ERR_INVALID_ARG;
+  DevState* ds = nullptr;
+  nmoe_status v = dev_state(&ds);
+  if (v != NMOE_OK) return v;
+  if (nmoe::launch_rows_copy(src, rows, n, row_bytes, dst, gather, ds->sm_count,
+                             static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return NMOE_ERR_CUDA;
+  }
+  return NMOE_OK;
+}
+}  // namespace
+
+nmoe_status nmoe_rows_gather(const void* src, const int32_t* rows, int64_t n, int64_t row_bytes,
+                             void* dst, nmoe_stream_t stream) {
+  return rows_copy(src, rows, n, row_bytes, dst, true, stream);
+}
+
+nmoe_status nmoe_rows_scatter(const void* src, const int32_t* rows, int64_t n,
+                              int64_t row_bytes, void* dst, nmoe_stream_t stream) {
+  return rows_copy(src, rows, n, row_bytes, dst, false, stream);
+}
+
+nmoe_status nmoe_combine_tokens(const void* Y, const int32_t* tok_ptr, int64_t T, int64_t d,
+                                int64_t t_begin, int64_t t_end, nmoe_dtype y_dtype,
+                                nmoe_dtype out_dtype, void* out, nmoe_stream_t stream) {
+  if (!Y || !tok_ptr || !out) return NMOE_ERR_INVALID_ARG;
+  if (T < 1 || T >= (int64_t(1) << 31) || d < 8 || d >= (int64_t(1) << 31))
+    return NMOE_ERR_INVALID_ARG;
+  if (d % 8 != 0) return NMOE_ERR_UNSUPPORTED;
+  if (t_begin < 0 || t_end < t_begin || t_end > T) return NMOE_ERR_INVALID_ARG;
+  if ((y_dtype != NMOE_F32 && y_dtype != NMOE_BF16) ||
+      (out_dtype != NMOE_F32 && out_dtype != NMOE_BF16))
+    return NMOE_ERR_INVALID_ARG;
+  if (!aligned16(Y) || !aligned16(out)) return NMOE_ERR_INVALID_ARG;
+  if (t_end == t_begin) return NMOE_OK;
+  DevState* ds = nullptr;
+  nmoe_status v = dev_state(&ds);
+  if (v != NMOE_OK) return v;
+  // the token range as a layer of its own: its tok_ptr entries, its output rows
+  Shape s = make_shape(t_end - t_begin, d, 1, 8, 1, 1);
+  s.pdl = false;
+  if (nmoe::launch_combine(Y, tok_ptr + t_begin, s, y_dtype == NMOE_F32,
+                           out_dtype == NMOE_F32, out, nullptr, false, nullptr, ds->err,
+                           ds->sm_count, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return NMOE_ERR_CUDA;
+  }
+  return NMOE_OK;
+}
+
 int nmoe_kernels_per_call(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
                           const nmoe_options* opts) {
   const nmoe_options o = opts ? *opts : default_options();
@@ -423,10 +533,14 @@ int nmoe_kernels_per_call(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
   const Shape s = make_shape(T, d, E, F, C, o.n_segments);
   const bool f32 = o.dtype == NMOE_F32;
   const bool split = !f32 && o.intermediate == NMOE_INTERMEDIATE_SPLIT;
-  const bool tc = !f32 && nmoe::experts_sm100_supported(s);
+  Shape sl = s;
+  if (o.expert_end > o.expert_begin) sl.E = (int)(o.expert_end - o.expert_begin);
+  const bool run_experts = sl.E > 0;
+  const bool tc = !f32 && run_experts && nmoe::experts_sm100_supported(sl);
   const bool fuse_csr = tc && nmoe::gemm1_sm100_fuses_csr(s, split);
-  // router, select, (CSR), gate/up, down, combine; two more for a shared expert
-  return 5 + (fuse_csr ? 0 : 1) + (o.shared_w1 != nullptr ? 2 : 0);
+  // router, select, (CSR), gate/up, down, (combine); two more for a shared expert
+  return 2 + (fuse_csr ? 0 : 1) + (run_experts ? 2 : 0) + (o.skip_combine ? 0 : 1) +
+         (o.shared_w1 != nullptr ? 2 : 0);
 }
 
 size_t nmoe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,

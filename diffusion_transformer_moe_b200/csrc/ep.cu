@@ -1,0 +1,95 @@
+// Expert-parallel pieces: the row lists one rank owes another, row gather/scatter, and
+// the combine of a token range.
+//
+// With experts split into contiguous ranges, one per rank, every rank computes the same
+// routing and token lists, runs the expert GEMMs for its own range (each row landing at
+// its token-major position in Y), and the owner of a token range needs exactly the rows
+// of its tokens that each other rank computed: ep_rows_kernel lists them, in ascending
+// row order, from the token lists alone, so sender and receiver agree without exchanging
+// counts. The rows travel packed (rows_copy_kernel gathers before the all-to-all and
+// scatters after it), and the owner's combine of its range then equals one GPU's.
+#include "nmoe_internal.cuh"
+
+namespace nmoe {
+namespace {
+
+constexpr int kRowsThreads = 1024;
+
+// One CTA: ordered compaction of the rows [tok_ptr[t_begin], tok_ptr[t_end]) whose entry
+// e*Ce + slot has e in [e_begin, e_end).
+__global__ void __launch_bounds__(kRowsThreads)
+ep_rows_kernel(const int32_t* __restrict__ tok_ptr, const int32_t* __restrict__ tok_ent,
+               int E, int Ce, int t_begin, int t_end, int e_begin, int e_end,
+               int32_t* __restrict__ rows, int32_t* __restrict__ count) {
+  __shared__ int s_warp[kRowsThreads / 32];
+  __shared__ int s_base;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r0 = tok_ptr[t_begin], r1 = tok_ptr[t_end];
+  if (tid == 0) s_base = 0;
+  __syncthreads();
+  for (int c0 = r0; c0 < r1; c0 += kRowsThreads) {
+    const int r = c0 + tid;
+    bool keep = false;
+    if (r < r1) {
+      const int v = tok_ent[r];
+      keep = v >= 0 && v < E * Ce && v / Ce >= e_begin && v / Ce < e_end;
+    }
+    const unsigned b = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) s_warp[warp] = __popc(b);
+    __syncthreads();
+    int before = s_base, total = 0;
+    for (int w = 0; w < kRowsThreads / 32; ++w) {
+      if (w < warp) before += s_warp[w];
+      total += s_warp[w];
+    }
+    if (keep) rows[before + __popc(b & ((1u << lane) - 1u))] = r;
+    __syncthreads();
+    if (tid == 0) s_base += total;
+    __syncthreads();
+  }
+  if (tid == 0) *count = s_base;
+}
+
+// dst[i] = src[rows[i]] (GATHER) or dst[rows[i]] = src[i], rows of `chunks` 16-byte units
+template <bool GATHER>
+__global__ void rows_copy_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ rows,
+                                 int64_t n, int chunks, uint4* __restrict__ dst) {
+  const int64_t total = n * chunks;
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < total;
+       k += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = k / chunks, c = k % chunks;
+    const int64_t r = rows[i];
+    if (GATHER)
+      dst[i * chunks + c] = src[r * chunks + c];
+    else
+      dst[r * chunks + c] = src[i * chunks + c];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent, int E, int Ce,
+                           int t_begin, int t_end, int e_begin, int e_end, int32_t* rows,
+                           int32_t* count, cudaStream_t st) {
+  ep_rows_kernel<<<1, kRowsThreads, 0, st>>>(tok_ptr, tok_ent, E, Ce, t_begin, t_end, e_begin,
+                                              e_end, rows, count);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rows_copy(const void* src, const int32_t* rows, int64_t n, int64_t row_bytes,
+                             void* dst, bool gather, int sm_count, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int chunks = (int)(row_bytes / 16);
+  const int64_t total = n * chunks;
+  int64_t grid = (total + 255) / 256;
+  if (grid > 4 * (int64_t)sm_count) grid = 4 * (int64_t)sm_count;
+  if (gather)
+    rows_copy_kernel<true><<<(unsigned)grid, 256, 0, st>>>(
+        static_cast<const uint4*>(src), rows, n, chunks, static_cast<uint4*>(dst));
+  else
+    rows_copy_kernel<false><<<(unsigned)grid, 256, 0, st>>>(
+        static_cast<const uint4*>(src), rows, n, chunks, static_cast<uint4*>(dst));
+  return cudaGetLastError();
+}
+
+}  // namespace nmoe

@@ -139,4 +139,12 @@ cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const Shape& s
                            bool out_f32, void* out, const void* residual, bool res_bf16,
                            const float* gate2, unsigned* err, int sm_count, cudaStream_t st);
 
+// Expert parallelism (ep.cu): rows[0 .. *count) = the token-major rows of tokens
+// [t_begin, t_end) whose expert is in [e_begin, e_end), ascending; row gather/scatter.
+cudaError_t launch_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent, int E, int Ce,
+                           int t_begin, int t_end, int e_begin, int e_end, int32_t* rows,
+                           int32_t* count, cudaStream_t st);
+cudaError_t launch_rows_copy(const void* src, const int32_t* rows, int64_t n, int64_t row_bytes,
+                             void* dst, bool gather, int sm_count, cudaStream_t st);
+
 }  // namespace nmoe

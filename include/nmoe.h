@@ -135,6 +135,18 @@ typedef struct nmoe_options {
    * with gate2 NULL (a gate of 1) or device fp32 [n_segments, d], 16-byte aligned. */
   const void* residual;
   const float* gate2;
+  /* Expert parallelism (no counterpart on the pages; an exact sharding of the layer over
+   * GPUs, one rank per contiguous range of experts). expert_end > expert_begin: the
+   * expert GEMMs run for experts [expert_begin, expert_end) only, W1, W3 and W2 then
+   * holding just those experts ([expert_end - expert_begin, ...]); the router, selection
+   * and token lists still cover all E experts and every token. skip_combine: the call
+   * stops after the down projection and leaves its rows (token-major positions, see
+   * nmoe_workspace_offsets) in the workspace, which the caller must then provide; the
+   * nmoe_ep_rows / nmoe_rows_gather / nmoe_rows_scatter / nmoe_combine_tokens calls
+   * finish the layer. Not combinable with a shared expert or residual. */
+  int64_t expert_begin;
+  int64_t expert_end;
+  int skip_combine;
 } nmoe_options;
 
 /* Fills `o` with the defaults: bf16, softmax, raw combine, route_scale 1, one segment,
@@ -184,6 +196,40 @@ NMOE_API nmoe_status nmoe_forward_ex(const void* x, const void* W_r, const void*
  * sizes). */
 NMOE_API size_t nmoe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C,
                            const nmoe_options* opts);
+
+/* Byte offsets, inside a workspace laid out for these sizes and options, of Y
+ * [E*Ce, d] (fp32 for fp32 layers and SPLIT intermediates, else bf16; row r is the r-th
+ * entry in token-major order), tok_ptr [T + 1] int32 and tok_ent [E*Ce] int32 (entry r
+ * = e*Ce + slot). NMOE_ERR_INVALID_ARG for invalid sizes. Pure host logic. */
+NMOE_API nmoe_status nmoe_workspace_offsets(int64_t T, int64_t d, int64_t E, int64_t F,
+                                            int64_t C, const nmoe_options* opts,
+                                            size_t* y_offset, size_t* tok_ptr_offset,
+                                            size_t* tok_ent_offset);
+
+/* Expert parallelism: the token-major rows of tokens [t_begin, t_end) whose expert lies
+ * in [e_begin, e_end), ascending, into rows (device int32, room for tok_ptr[t_end] -
+ * tok_ptr[t_begin] entries), and their number into *count (device int32). tok_ptr and
+ * tok_ent as left in the workspace (nmoe_workspace_offsets); Ce = n_segments * C. */
+NMOE_API nmoe_status nmoe_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent, int64_t T,
+                                  int64_t E, int64_t Ce, int64_t t_begin, int64_t t_end,
+                                  int64_t e_begin, int64_t e_end, int32_t* rows,
+                                  int32_t* count, nmoe_stream_t stream);
+
+/* dst[i, :] = src[rows[i], :] (gather) / dst[rows[i], :] = src[i, :] (scatter) for
+ * i < n: rows of row_bytes bytes (a positive multiple of 16), 16-byte aligned device
+ * arrays; rows device int32. */
+NMOE_API nmoe_status nmoe_rows_gather(const void* src, const int32_t* rows, int64_t n,
+                                      int64_t row_bytes, void* dst, nmoe_stream_t stream);
+NMOE_API nmoe_status nmoe_rows_scatter(const void* src, const int32_t* rows, int64_t n,
+                                       int64_t row_bytes, void* dst, nmoe_stream_t stream);
+
+/* The combine alone for tokens [t_begin, t_end): out[t - t_begin, :] = sum of Y rows
+ * tok_ptr[t] .. tok_ptr[t+1]-1 in order, fp32, rounded once (0 for a token without
+ * rows). Y in y_dtype (NMOE_F32 or NMOE_BF16), out in out_dtype, d a multiple of 8. */
+NMOE_API nmoe_status nmoe_combine_tokens(const void* Y, const int32_t* tok_ptr, int64_t T,
+                                         int64_t d, int64_t t_begin, int64_t t_end,
+                                         nmoe_dtype y_dtype, nmoe_dtype out_dtype, void* out,
+                                         nmoe_stream_t stream);
 
 /* Number of kernels one nmoe_forward_ex call with these sizes and options launches
  * (0 for invalid sizes): the router, the selection, the token lists (inside the gate/up

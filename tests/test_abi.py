@@ -130,6 +130,35 @@ def test_block_options_are_checked_on_host(kw, expect):
     assert _forward_ex_status(**kw) == expect
 
 
+@pytest.mark.parametrize("kw,expect", [
+    (dict(expert_begin=0, expert_end=2), 1),                    # a rank's range must skip the combine
+    (dict(skip_combine=1), 1),                                  # ... and needs a caller workspace
+    (dict(expert_begin=0, expert_end=2, skip_combine=1, workspace=FAKE + 65536,
+          residual=FAKE + 131072), 1),                          # no residual with expert ranges
+])
+def test_expert_parallel_options_are_checked_on_host(kw, expect):
+    assert _forward_ex_status(**kw) == expect
+
+
+def test_expert_parallel_calls_check_arguments_on_host():
+    lib = nm.lib()
+    # t_end beyond T, an empty expert table, misaligned rows, rows not a multiple of 16 B
+    assert lib.nmoe_ep_rows(FAKE, FAKE, 64, 4, 8, 0, 65, 0, 2, FAKE, FAKE, None) == 1
+    assert lib.nmoe_ep_rows(FAKE, FAKE, 64, 0, 8, 0, 64, 0, 0, FAKE, FAKE, None) == 1
+    assert lib.nmoe_rows_gather(FAKE + 4, FAKE, 4, 64, FAKE, None) == 1
+    assert lib.nmoe_rows_scatter(FAKE, FAKE, 4, 24, FAKE, None) == 1
+    assert lib.nmoe_combine_tokens(FAKE, FAKE, 64, 12, 0, 64, 1, 0, FAKE, None) == 2
+
+
+def test_split_range_covers_every_item_once():
+    from diffusion_transformer_moe_b200 import ep
+    for n, parts in ((64, 3), (7, 7), (128, 8), (10, 4)):
+        got = [ep.split_range(n, parts, i) for i in range(parts)]
+        assert got[0][0] == 0 and got[-1][1] == n
+        assert all(a[1] == b[0] for a, b in zip(got, got[1:]))
+        assert max(e - b for b, e in got) - min(e - b for b, e in got) <= 1
+
+
 def test_missing_gpu_is_reported_not_crashed():
     import torch
     if torch.cuda.is_available():
