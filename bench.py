@@ -285,7 +285,7 @@ def run_reference(args, w, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": _workload_config(w, "fp64 oracle"),
+        "config": dict(_workload_config(w, "fp64 oracle"), l2="n/a (host CPU)"),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _oracle_threads(),
                          "kind": "oracle", "sample": f"each step: {what}"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,

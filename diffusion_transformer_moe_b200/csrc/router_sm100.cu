@@ -259,7 +259,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
     const bool live = t < p.T;
     const float* b = (p.bias != nullptr && live) ? p.bias + (int64_t)(t / p.S) * p.E : nullptr;
     float h[kEpc], l[kEpc], pr[kEpc];
-#pragma unroll 4
+#pragma unroll
     for (int j = 0; j < kEpc; ++j) {
       h[j] = 0.f;
       l[j] = 0.f;
@@ -280,7 +280,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       // h - m + l exactly up to t's rounding (|t| < 1e-6, so the dropped t^2 is far
       // below fp32)
       float m = -INFINITY;
-#pragma unroll 4
+#pragma unroll
       for (int j = 0; j < kEpc; ++j)
         if (eb + j < p.E) m = fmaxf(m, h[j]);
       red_m[grp * 64 + tk] = m;
@@ -288,7 +288,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       for (int k = 0; k < 2 * G; ++k) m = fmaxf(m, red_m[k * 64 + tk]);
       bool deep = false;                     // some argument below -80
       float zs = 0.f, zc = 0.f;              // compensated sum of the exponentials
-#pragma unroll 4
+#pragma unroll
       for (int j = 0; j < kEpc; ++j) {
         float dd, tt;                        // exp argument: dd + tt
         two_sum(h[j], -m, dd, tt);
@@ -306,7 +306,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
           if (eb + j < p.E && dd < -80.f) pr[j] = (float)exp((double)dd + (double)(tt + l[j]));
         }
       }
-#pragma unroll 4
+#pragma unroll
       for (int j = 0; j < kEpc; ++j) {
         float s_, e_;
         two_sum(zs, pr[j], s_, e_);
@@ -325,12 +325,12 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
         zc += e_ + v.y;
       }
       const float rz = 1.f / (zs + zc);      // one division; each score 1 ulp from e / z
-#pragma unroll 4
+#pragma unroll
       for (int j = 0; j < kEpc; ++j) pr[j] *= rz;
     } else {
       // 1 / (1 + exp(-(h + l))), exp(-(h + l)) = exp(-h) (1 - l)
       bool deep = false;
-#pragma unroll 4
+#pragma unroll
       for (int j = 0; j < kEpc; ++j) {
         deep |= fabsf(h[j]) > 80.f;
         pr[j] = 1.f / (1.f + expf(-h[j]) * (1.f - l[j]));
@@ -352,7 +352,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
         for (int j = 0; j < kEpc; ++j)
           if (eb + j < p.E) srow[j] = pr[j];
       }
-#pragma unroll 4
+#pragma unroll
       for (int j = 0; j < kEpc; ++j)
         if (eb + j < p.E) p.scores_t[(int64_t)(eb + j) * p.T + t] = pr[j];
     }
