@@ -383,6 +383,31 @@ def run_ours(args, w, rank, world, local_rank, dist):
     # headline number)
     traced_ms = timed(trace)
     stage_ms, ncalls = trace.read()
+    # the same step replayed from a CUDA graph (one captured layer call; the L2 flush
+    # stays outside the graph and the events)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        gev[i][0].record(stream)
+        graph.replay()
+        gev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    graph_ms = sum(a_.elapsed_time(b_) for a_, b_ in gev)
+    del graph
     if nm.get_last_error() != 0:
         raise RuntimeError("device-side check failed during the timed steps")
 
@@ -422,7 +447,8 @@ def run_ours(args, w, rank, world, local_rank, dist):
         raise RuntimeError("device-side check failed during the end-to-end steps")
     out_host = e2e_out[0]
 
-    ms, e2e_ms, traced_ms = max_over_ranks([ms, e2e_ms, traced_ms], dist, dev)
+    ms, e2e_ms, traced_ms, graph_ms = max_over_ranks([ms, e2e_ms, traced_ms, graph_ms], dist,
+                                                     dev)
     if rank != 0:
         return
 
@@ -473,6 +499,9 @@ def run_ours(args, w, rank, world, local_rank, dist):
         "roofline": roof,
         "stages": stages,
         "traced_ms_per_step": traced_ms / K,
+        "graph_replay": {"ms_per_step": graph_ms / K,
+                         "value": replica_throughput(w.T, world, K, graph_ms),
+                         "how": "one captured layer call, replayed K times"},
         "gpu_launches": K * nm.kernels_per_call(w.T, w.d, w.E, w.F, w.C, intermediate=inter,
                                                 n_segments=w.segments,
                                                 shared_f=args.shared_f or None),

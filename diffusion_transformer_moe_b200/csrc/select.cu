@@ -12,9 +12,10 @@
 // first digit splits fp32 scores into bins an eighth of an octave wide, so the bin
 // holding the threshold is a small share of the row: its keys are copied to a candidate
 // list and the last two digits are counted over that list alone (a list of at most
-// kRankMax keys is instead ranked directly, each key against all). One more sweep of the
-// row records, 32 tokens to a word, which keys lie above the threshold and which equal
-// it; a block-wide scan over the words' popcounts then gives every chosen key (each key
+// kRankMax keys is instead ranked directly, each key against all). The same sweep that
+// lists the candidates records, 32 tokens to a word, which keys lie in a higher bin;
+// once the threshold is known only the candidates' bits are added (above it, or equal
+// to it); a block-wide scan over the words' popcounts then gives every chosen key (each key
 // above the threshold, plus the first C - #above keys equal to it) its position in
 // ascending token order, and, for every block of kBlockTok tokens, how many of the
 // expert's entries come before the block (the boundary table).
@@ -138,12 +139,13 @@ __device__ __forceinline__ void find_digit(const unsigned* hist, unsigned k, uns
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, 1)
 select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int Ce, int E,
               int cached, int32_t* __restrict__ idx, float* __restrict__ gate,
               int32_t* __restrict__ bnd, unsigned* __restrict__ err) {
   pdl_launch_dependents();
   // dynamic: [keys, cached ? S (rounded up to 4) : 0][gt words, nw4][eq words, nw4]
+  //          [the candidates' positions in the row, kCandMax]
   extern __shared__ __align__(16) uint32_t s_dyn[];
   __shared__ __align__(16) unsigned s_hist[kBins];
   __shared__ uint32_t s_cand[kCandMax];
@@ -157,6 +159,7 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
   uint32_t* s_keys = s_dyn;
   uint32_t* s_gtw = s_dyn + (cached ? ((S + 3) & ~3) : 0);
   uint32_t* s_eqw = s_gtw + nw4;
+  int32_t* s_cidx = reinterpret_cast<int32_t*>(s_eqw + nw4);
 
   reinterpret_cast<uint4*>(s_hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
   if (tid == 0) s_ncand = 0;
@@ -200,6 +203,7 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
   uint32_t prefix = 0, pmask = 0;
   int k = C;
   bool ranked = false;
+  bool collected = false;  // candidates listed, and the bitmap words above their bin set
 #pragma unroll 1
   for (int pass = 0; pass < 3 && !ranked; ++pass) {
     const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
@@ -214,36 +218,62 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
     const int nbin = (int)s_res[2];
     reinterpret_cast<uint4*>(s_hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
     if (pass == 0 && nbin <= kCandMax) {
-      // keys of the threshold's bin; their order is irrelevant to the histograms
+      // Keys of the threshold's bin, with their positions (their order is irrelevant
+      // to the histograms), and, 32 keys to a word, which keys lie in a higher bin:
+      // those are above the threshold whatever it is (the equal words start empty).
       for (int i0 = 0; i0 < S; i0 += kSelThreads) {
         const int i = i0 + tid;
         const uint32_t key = i < S ? keys[i] : 0u;
         const bool in = i < S && (key & pmask) == prefix;
+        const unsigned above = __ballot_sync(0xffffffffu, i < S && (key & pmask) > prefix);
+        const int w = (i0 >> 5) + warp;
+        if (lane == 0 && w < nw) {
+          s_gtw[w] = above;
+          s_eqw[w] = 0u;
+        }
         const unsigned b = __ballot_sync(0xffffffffu, in);
         if (b != 0u) {
           unsigned base = 0;
           if (lane == 0) base = atomicAdd(&s_ncand, (unsigned)__popc(b));
           base = __shfl_sync(0xffffffffu, base, 0);
           const unsigned at = base + (unsigned)__popc(b & lanemask_lt());
-          if (in && at < (unsigned)kCandMax) s_cand[at] = key;
+          if (in && at < (unsigned)kCandMax) {
+            s_cand[at] = key;
+            s_cidx[at] = i;
+          }
         }
       }
       src = s_cand;
       n = nbin;
+      collected = true;
       if (nbin <= kRankMax) {
         // Few candidates: rank them directly instead of two more digits. The k-th
-        // largest candidate c has #{> c} < k <= #{>= c}; equal candidates agree.
+        // largest candidate c has #{> c} < k <= #{>= c}; equal candidates agree. Four
+        // threads per candidate each count a quarter of the others.
+        static_assert(kSelThreads == 4 * kRankMax, "four counters per candidate");
         __syncthreads();
-        if (tid < nbin) {
-          const uint32_t c = s_cand[tid];
-          int gt = 0, ge = 0;
-          for (int j = 0; j < nbin; ++j) {
+        const int ci = tid % kRankMax, q = tid / kRankMax;
+        int gt = 0, ge = 0;
+        if (ci < nbin) {
+          const uint32_t c = s_cand[ci];
+          for (int j = q; j < nbin; j += 4) {
             const uint32_t o = s_cand[j];
             gt += o > c;
             ge += o >= c;
           }
+        }
+        int2* part = reinterpret_cast<int2*>(s_hist);  // free: no histogram follows
+        part[q * kRankMax + ci] = make_int2(gt, ge);
+        __syncthreads();
+        if (q == 0 && ci < nbin) {
+#pragma unroll
+          for (int r = 1; r < 4; ++r) {
+            const int2 v = part[r * kRankMax + ci];
+            gt += v.x;
+            ge += v.y;
+          }
           if (gt < k && k <= ge) {
-            s_res[0] = c;
+            s_res[0] = s_cand[ci];
             s_res[1] = (unsigned)gt;
           }
         }
@@ -258,15 +288,25 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
   const uint32_t thr = prefix;  // the C-th largest key; take k keys equal to it
 
   // Word w of the bitmaps covers keys [32w, 32w + 32): bit b set if key 32w + b is
-  // above (gt) or equal to (eq) the threshold.
-  for (int w = warp; w < nw; w += kSelWarps) {
-    const int i = 32 * w + lane;
-    const uint32_t key = i < S ? keys[i] : 0u;
-    const unsigned gw = __ballot_sync(0xffffffffu, i < S && key > thr);
-    const unsigned qw = __ballot_sync(0xffffffffu, i < S && key == thr);
-    if (lane == 0) {
-      s_gtw[w] = gw;
-      s_eqw[w] = qw;
+  // above (gt) or equal to (eq) the threshold. With a candidate list, only the
+  // candidates' bits are left to set; otherwise one sweep of the row sets them all.
+  if (collected) {
+    for (int j = tid; j < n; j += kSelThreads) {
+      const uint32_t key = s_cand[j];
+      const int i = s_cidx[j];
+      if (key > thr) atomicOr(&s_gtw[i >> 5], 1u << (i & 31));
+      else if (key == thr) atomicOr(&s_eqw[i >> 5], 1u << (i & 31));
+    }
+  } else {
+    for (int w = warp; w < nw; w += kSelWarps) {
+      const int i = 32 * w + lane;
+      const uint32_t key = i < S ? keys[i] : 0u;
+      const unsigned gw = __ballot_sync(0xffffffffu, i < S && key > thr);
+      const unsigned qw = __ballot_sync(0xffffffffu, i < S && key == thr);
+      if (lane == 0) {
+        s_gtw[w] = gw;
+        s_eqw[w] = qw;
+      }
     }
   }
   __syncthreads();
@@ -335,7 +375,8 @@ cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, f
   if (s.S > kSelectMaxRow) return cudaErrorInvalidValue;
   const int cached = s.S <= kSelMaxCached;
   const size_t nw4 = (size_t)((ceil_div(s.S, 32) + 3) & ~3);
-  const size_t smem = sizeof(uint32_t) * ((cached ? (size_t)((s.S + 3) & ~3) : 0) + 2 * nw4);
+  const size_t smem = sizeof(uint32_t) * ((cached ? (size_t)((s.S + 3) & ~3) : 0) + 2 * nw4 +
+                                          (size_t)kCandMax);
   dim3 grid((unsigned)s.E, (unsigned)s.n_seg);
   return launch_kernel(select_kernel, grid, dim3(kSelThreads), smem, st, s.pdl, 1, scores_t,
                        (int64_t)s.T, s.S, s.C, s.Ce, s.E, cached, idx, gate, bnd, err);
