@@ -206,7 +206,7 @@ def gated_residual(residual, gate2, ffn_out, n_segments: int = 1) -> np.ndarray:
 def layer(x, W_r, W1, W3, W2, C: int, *, score_fn: str = "softmax",
           combine: str = "raw", route_scale: float = 1.0, n_segments: int = 1,
           router_bias=None, selection=None, shared=None, residual=None,
-          gate2=None) -> dict:
+          gate2=None, router_x=None) -> dict:
     """The whole MoE FFN layer.
 
     ``selection`` injects an expert-choice selection (idx[E, n_segments*C]) instead of
@@ -215,13 +215,15 @@ def layer(x, W_r, W1, W3, W2, C: int, *, score_fn: str = "softmax",
     every token goes through (section 6.2), onto which the routed outputs are added.
     ``residual`` [T,d] (and ``gate2`` [n_segments,d]) add the result to the block's
     residual stream through the gate (section 6.3, :func:`gated_residual`).
+    ``router_x`` [T,d], when given, is what the router scores (section 6.2: the gate
+    reads the unmodulated hidden states, the experts the block's modulated input x).
 
     Returns dict(out [T,d] fp64, p fp64 [T,E], scores32 [T,E], idx, w).
     """
     x = _f64(x)
     T, d = x.shape
     E = np.asarray(W_r).shape[1]
-    logits = router_logits(x, W_r, router_bias, n_segments)
+    logits = router_logits(x if router_x is None else router_x, W_r, router_bias, n_segments)
     p = scores_from_logits(logits, score_fn)
     s32 = round_f32(p)
     idx = select(s32, C, n_segments) if selection is None else np.asarray(selection)
@@ -242,12 +244,12 @@ def layer(x, W_r, W1, W3, W2, C: int, *, score_fn: str = "softmax",
 def layer_rows(x, W_r, W1, W3, W2, C: int, tokens, *, score_fn: str = "softmax",
                combine: str = "raw", route_scale: float = 1.0, n_segments: int = 1,
                router_bias=None, selection=None, shared=None, residual=None,
-               gate2=None) -> dict:
+               gate2=None, router_x=None) -> dict:
     """The layer output for the listed tokens only (for workloads too large to run
     whole). Router, scores and selection still cover every token."""
     x = _f64(x)
     E = np.asarray(W_r).shape[1]
-    logits = router_logits(x, W_r, router_bias, n_segments)
+    logits = router_logits(x if router_x is None else router_x, W_r, router_bias, n_segments)
     p = scores_from_logits(logits, score_fn)
     s32 = round_f32(p)
     idx = select(s32, C, n_segments) if selection is None else np.asarray(selection)

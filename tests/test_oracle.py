@@ -219,6 +219,49 @@ def test_timestep_concat_router_is_a_segment_bias():
                                atol=1e-14)
 
 
+def test_separate_router_input_reproduces_the_pages_concat_gate():
+    # Section 6.2: the gate reads cat([timestep, unmodulated hidden]) while the experts
+    # transform the block's input. Built here from the page's literal gate, softmax,
+    # each expert's top-C by (score, -token) found by sorting, and a per-token sum
+    # of score-weighted dense SwiGLU outputs of the EXPERT input.
+    rng = np.random.default_rng(21)
+    T, d, dt, E, F, C, nseg = 16, 6, 3, 4, 5, 3, 2
+    h = rng.normal(size=(T, d))              # unmodulated hidden states (router input)
+    x = rng.normal(size=(T, d))              # the experts' input
+    temb = rng.normal(size=(nseg, dt))
+    Wg = rng.normal(size=(dt + d, E)) / np.sqrt(dt + d)
+    W1 = rng.normal(size=(E, d, F)); W3 = rng.normal(size=(E, d, F))
+    W2 = rng.normal(size=(E, F, d))
+    lit = np.concatenate([np.repeat(temb, T // nseg, axis=0), h], axis=1) @ Wg
+    z = np.exp(lit - lit.max(axis=1, keepdims=True))
+    p = z / z.sum(axis=1, keepdims=True)
+    p32 = p.astype(np.float32)
+    want = np.zeros((T, d))
+    chosen = np.zeros((E, T), dtype=bool)
+    S = T // nseg
+    for e in range(E):
+        for g in range(nseg):
+            seg = list(range(g * S, (g + 1) * S))
+            for t in sorted(seg, key=lambda t: (-float(p32[t, e]), t))[:C]:
+                chosen[e, t] = True
+                want[t] += p[t, e] * _dense_ffn(x[t:t + 1], W1[e], W3[e], W2[e])[0]
+    r = O.layer(x, Wg[dt:], W1, W3, W2, C, n_segments=nseg, router_bias=temb @ Wg[:dt],
+                router_x=h)
+    for e in range(E):
+        assert sorted(r["idx"][e].tolist()) == np.flatnonzero(chosen[e]).tolist()
+    np.testing.assert_allclose(r["out"], want, rtol=1e-11, atol=1e-12)
+    # the router input decides the selection: scoring x instead changes it here
+    r_x = O.layer(x, Wg[dt:], W1, W3, W2, C, n_segments=nseg, router_bias=temb @ Wg[:dt])
+    assert not np.array_equal(np.sort(r_x["idx"], axis=1), np.sort(r["idx"], axis=1))
+    # and router_x = x is the default layer, value for value
+    r_same = O.layer(x, Wg[dt:], W1, W3, W2, C, n_segments=nseg, router_x=x)
+    r_def = O.layer(x, Wg[dt:], W1, W3, W2, C, n_segments=nseg)
+    assert np.array_equal(r_same["out"], r_def["out"])
+    rows = O.layer_rows(x, Wg[dt:], W1, W3, W2, C, [0, 5, 11], n_segments=nseg,
+                        router_bias=temb @ Wg[:dt], router_x=h)
+    np.testing.assert_allclose(rows["out"], r["out"][[0, 5, 11]], rtol=1e-13, atol=1e-15)
+
+
 def test_sampled_rows_match_full_layer():
     a = _small(40, 8, 5, 6, seed=15)
     r = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=8, combine="normalized",
