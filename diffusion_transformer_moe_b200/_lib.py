@@ -54,7 +54,7 @@ class Options(C.Structure):
         ("tma_gather", C.c_int), ("shared_w1", C.c_void_p), ("shared_w3", C.c_void_p),
         ("shared_w2", C.c_void_p), ("shared_f", C.c_int64), ("residual", C.c_void_p),
         ("gate2", C.c_void_p), ("expert_begin", C.c_int64), ("expert_end", C.c_int64),
-        ("skip_combine", C.c_int),
+        ("skip_combine", C.c_int), ("router_x", C.c_void_p),
     ]
 
 
@@ -167,11 +167,13 @@ def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
             n_segments=1, router_bias=None, workspace=None, scores_out=None, idx_out=None,
             host_io=False, trace=None, intermediate="split", out_f32=False,
             tma_gather=False, shared=None, shared_f=None, residual=None,
-            gate2=None, expert_begin=0, expert_end=0, skip_combine=False) -> Options:
+            gate2=None, expert_begin=0, expert_end=0, skip_combine=False,
+            router_x=None) -> Options:
     """nmoe_options from keyword arguments. ``shared`` = (Ws1 [d,Fs], Ws3 [d,Fs],
     Ws2 [Fs,d]) device tensors adds the shared expert; ``shared_f`` alone (no tensors)
     only sizes a workspace for one. ``residual`` [T,d] and ``gate2`` fp32
-    [n_segments,d] add the block's gated residual."""
+    [n_segments,d] add the block's gated residual. ``router_x`` [T,d] is what the
+    router scores instead of x (on the host with ``host_io``)."""
     o = Options()
     lib().nmoe_options_init(C.byref(o))
     o.dtype = dtype
@@ -205,6 +207,7 @@ def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
     o.expert_begin = int(expert_begin)
     o.expert_end = int(expert_end)
     o.skip_combine = 1 if skip_combine else 0
+    o.router_x = _ptr(router_x)
     return o
 
 
@@ -240,13 +243,19 @@ def select(scores_t, C_: int, n_segments=1, csr=True, stream=None):
 def forward(x, W_r, W1, W3, W2, C_: int, out=None, stream=None, **opts):
     """The whole layer. ``opts`` are the nmoe_options fields (score_fn, combine,
     route_scale, n_segments, router_bias, workspace, scores_out, idx_out, trace,
-    intermediate, out_f32, tma_gather, shared=(Ws1, Ws3, Ws2), residual, gate2). With
-    ``host_io=True`` x and out are pinned CPU tensors."""
+    intermediate, out_f32, tma_gather, shared=(Ws1, Ws3, Ws2), residual, gate2, router_x).
+    With ``host_io=True`` x, router_x and out are pinned CPU tensors."""
     host_io = bool(opts.get("host_io", False))
     for n, t in (("W_r", W_r), ("W1", W1), ("W3", W3), ("W2", W2)):
         _dev(t, n)
+    rx = opts.get("router_x")
+    if rx is not None and (rx.shape != x.shape or rx.dtype != x.dtype
+                           or not rx.is_contiguous()):
+        raise ValueError("router_x must be a contiguous tensor of x's shape and dtype")
     if not host_io:
         _dev(x, "x")
+        if rx is not None:
+            _dev(rx, "router_x")
     T, d = x.shape
     E, _, F = W1.shape
     if out is None:

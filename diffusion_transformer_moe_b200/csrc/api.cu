@@ -113,7 +113,7 @@ size_t out_size(nmoe_dtype dt, const nmoe_options& o) {
 }
 
 struct Layout {
-  size_t scores, scores_t, idx, gate, bnd, tok_ptr, tok_ent, ent_pos, H, Hs, Y, xin, xout,
+  size_t scores, scores_t, idx, gate, bnd, tok_ptr, tok_ent, ent_pos, H, Hs, Y, xin, xr, xout,
       total;
 };
 
@@ -137,6 +137,7 @@ Layout make_layout(const Shape& s, nmoe_dtype dt, const nmoe_options& o) {
   L.Hs = o.shared_w1 ? take(is * (size_t)s.T * (size_t)o.shared_f) : none;
   L.Y = take(is * ((size_t)s.E * s.Ce + shared_rows) * s.d);
   L.xin = o.host_io ? take(esize(dt) * (size_t)s.T * s.d) : none;
+  L.xr = o.host_io && o.router_x ? take(esize(dt) * (size_t)s.T * s.d) : none;
   L.xout = o.host_io ? take(out_size(dt, o) * (size_t)s.T * s.d) : none;
   L.total = off;
   return L;
@@ -174,6 +175,7 @@ nmoe_status options_ok(const nmoe_options& o) {
   if (o.expert_end > o.expert_begin && !o.skip_combine) return NMOE_ERR_INVALID_ARG;
   if (o.residual && !aligned16(o.residual)) return NMOE_ERR_INVALID_ARG;
   if (o.gate2 && !aligned16(o.gate2)) return NMOE_ERR_INVALID_ARG;
+  if (o.router_x && !o.host_io && !aligned16(o.router_x)) return NMOE_ERR_INVALID_ARG;
   return NMOE_OK;
 }
 
@@ -206,6 +208,7 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   if (!o.host_io && (!aligned16(x) || (out && !aligned16(out)))) return NMOE_ERR_INVALID_ARG;
   if (x == out) return NMOE_ERR_INVALID_ARG;
   if (o.residual != nullptr && o.residual == out) return NMOE_ERR_INVALID_ARG;
+  if (o.router_x != nullptr && o.router_x == out) return NMOE_ERR_INVALID_ARG;
 
   DevState* ds = nullptr;
   if ((v = dev_state(&ds)) != NMOE_OK) return v;
@@ -259,12 +262,18 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   const bool out_f32 = f32 || o.out_f32;
 
   const void* xd = x;
+  const void* xrd = o.router_x ? o.router_x : x;  // what the router scores
   void* outd = out;
   cudaError_t e = cudaSuccess;
   if (o.host_io) {
     xd = ws + L.xin;
     outd = ws + L.xout;
     e = cudaMemcpyAsync(ws + L.xin, x, xbytes, cudaMemcpyHostToDevice, st);
+    xrd = xd;
+    if (o.router_x && e == cudaSuccess) {
+      xrd = ws + L.xr;
+      e = cudaMemcpyAsync(ws + L.xr, o.router_x, xbytes, cudaMemcpyHostToDevice, st);
+    }
   }
   cudaEvent_t* ev = trace_slot(o.trace);
   auto mark = [&](int i) {
@@ -273,10 +282,10 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   mark(0);
   if (e == cudaSuccess) {
     if (o.dtype == NMOE_BF16 && nmoe::router_sm100_supported(s))
-      e = nmoe::launch_router_sm100(xd, W_r, s, o.score_fn, o.router_bias, scores, scores_t,
+      e = nmoe::launch_router_sm100(xrd, W_r, s, o.score_fn, o.router_bias, scores, scores_t,
                                     ds->err, st);
     else
-      e = nmoe::launch_router_simt(xd, W_r, s, o.dtype, o.score_fn, o.router_bias, scores,
+      e = nmoe::launch_router_simt(xrd, W_r, s, o.dtype, o.score_fn, o.router_bias, scores,
                                    scores_t, st);
   }
   mark(1);
@@ -370,6 +379,7 @@ void nmoe_options_init(nmoe_options* o) {
   o->expert_begin = 0;
   o->expert_end = 0;
   o->skip_combine = 0;
+  o->router_x = nullptr;
 }
 
 nmoe_status nmoe_router(const void* x, const void* W_r, int64_t T, int64_t d, int64_t E,

@@ -147,11 +147,19 @@ typedef struct nmoe_options {
   int64_t expert_begin;
   int64_t expert_end;
   int skip_combine;
+  /* Separate router input (section 6.2: the gate reads the unmodulated hidden states,
+   * concatenated with the timestep, while the experts transform the block's modulated
+   * input). NULL: the router scores x. Else [T, d] in `dtype`, 16-byte aligned, not
+   * overlapping out: the router scores router_x and the experts still gather their rows
+   * from x (with router_bias carrying the timestep half, this is the page's gate
+   * exactly). With host_io it is a HOST pointer, copied in like x. */
+  const void* router_x;
 } nmoe_options;
 
 /* Fills `o` with the defaults: bf16, softmax, raw combine, route_scale 1, one segment,
  * no bias, internal workspace, no extra outputs, device I/O, no trace, SPLIT
- * intermediates, out in the input dtype. */
+ * intermediates, out in the input dtype, no shared expert or residual, all experts, the
+ * router scoring x. */
 NMOE_API void nmoe_options_init(nmoe_options* o);
 
 /* Router (section 6.2 "gate = Linear(..., num_experts, bias=False)", then softmax over

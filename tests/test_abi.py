@@ -36,6 +36,7 @@ def test_options_struct_matches_defaults():
     nm.lib().nmoe_options_init(C.byref(o))
     assert (o.dtype, o.score_fn, o.combine, o.n_segments, o.host_io) == (0, 0, 0, 1, 0)
     assert o.route_scale == 1.0 and not o.workspace and not o.trace
+    assert not o.router_x and not o.residual and o.expert_end == 0
 
 
 def test_status_strings_and_build_info():
@@ -96,6 +97,21 @@ def test_workspace_size_accounts_for_every_buffer():
     assert host32 >= n + 2 * T * d + 4 * T * d
 
 
+def test_workspace_holds_a_host_router_input():
+    T, d, E, F, C_ = 2048, 1024, 16, 2048, 256
+    host = nm.workspace_size(T, d, E, F, C_, host_io=True)
+    # a separate router input in host memory is copied into one more [T, d] buffer; on
+    # the device it needs none
+    o = L.options(host_io=True)
+    o.router_x = FAKE
+    with_rx = int(nm.lib().nmoe_workspace_size(T, d, E, F, C_, C.byref(o)))
+    assert 2 * T * d <= with_rx - host <= 2 * T * d + 256
+    o = L.options()
+    o.router_x = FAKE
+    assert int(nm.lib().nmoe_workspace_size(T, d, E, F, C_, C.byref(o))) == \
+        nm.workspace_size(T, d, E, F, C_)
+
+
 def test_workspace_grows_by_the_shared_expert():
     T, d, E, F, C_, Fs = 8192, 2048, 64, 1024, 128, 1024
     n = nm.workspace_size(T, d, E, F, C_)
@@ -125,6 +141,8 @@ def _forward_ex_status(**kw):
     (dict(gate2=FAKE + 65536), 1),                                       # gate without residual
     (dict(residual=FAKE + 65544), 1),                                    # misaligned
     (dict(residual=FAKE + 32768), 1),                                    # residual is out
+    (dict(router_x=FAKE + 65544), 1),                                    # misaligned
+    (dict(router_x=FAKE + 32768), 1),                                    # router input is out
 ])
 def test_block_options_are_checked_on_host(kw, expect):
     assert _forward_ex_status(**kw) == expect

@@ -42,8 +42,9 @@ def _run(a, C_, **opts):
     nseg = opts.get("n_segments", 1)
     scores = torch.empty(T, E, device="cuda", dtype=torch.float32)
     idx = torch.empty(E, nseg * C_, device="cuda", dtype=torch.int32)
-    if "router_bias" in opts and opts["router_bias"] is not None:
-        opts["router_bias"] = opts["router_bias"].cuda()
+    for k in ("router_bias", "router_x"):
+        if opts.get(k) is not None:
+            opts[k] = opts[k].cuda()
     out = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], C_,
                      scores_out=scores, idx_out=idx, **opts)
     torch.cuda.synchronize()
@@ -376,6 +377,51 @@ def test_host_io_matches_device_io():
     x_host = a["x"].pin_memory()
     y_host = nm.forward(x_host, dev["W_r"], dev["W1"], dev["W3"], dev["W2"], 64, host_io=True)
     torch.cuda.synchronize()
+    assert torch.equal(y_host, y_dev.cpu())
+
+
+# -- a separate router input (walkthrough section 6.2: the gate reads the timestep and the
+#    unmodulated hidden states, the experts transform the block's input) -----------------
+
+def _router_input_case(T, d, E, F, dtype, nseg, seed):
+    a = I.make_small(T, d, E, F, dtype, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    h = (1.5 * torch.randn(T, d, generator=g)).to(a["x"].dtype)
+    bias = torch.randn(nseg, E, generator=g)
+    return a, h, bias
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T,d,E,F,C_,nseg", [
+    (300, 136, 5, 200, 20, 3),     # ragged everywhere
+    (520, 264, 12, 328, 65, 2),    # C spans a 128-row tile boundary per segment pair
+])
+def test_separate_router_input_matches_oracle(dtype, T, d, E, F, C_, nseg):
+    a, h, bias = _router_input_case(T, d, E, F, dtype, nseg, seed=T + E)
+    out, scores, idx = _run(a, C_, n_segments=nseg, router_bias=bias, router_x=h)
+    sel = O.select(scores.cpu().numpy(), C_, nseg)
+    assert np.array_equal(sel, idx.cpu().numpy())
+    r = O.layer(I.to_numpy_f64(a["x"]), I.to_numpy_f64(a["W_r"]), I.to_numpy_f64(a["W1"]),
+                I.to_numpy_f64(a["W3"]), I.to_numpy_f64(a["W2"]), C_, selection=sel,
+                n_segments=nseg, router_bias=bias.double().numpy(),
+                router_x=I.to_numpy_f64(h))
+    _check_scores(scores, r["p"])
+    _check_out(out, r["out"], dtype)
+    # the selection follows the router input: scoring x instead picks other tokens here
+    _, _, idx_x = _run(a, C_, n_segments=nseg, router_bias=bias)
+    assert not torch.equal(idx_x, idx)
+
+
+def test_separate_router_input_through_host_buffers():
+    a, h, bias = _router_input_case(512, 256, 8, 128, "bf16", 2, seed=43)
+    dev = {k: v.cuda() for k, v in a.items()}
+    kw = dict(n_segments=2, router_bias=bias.cuda())
+    y_dev = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], 32,
+                       router_x=h.cuda(), **kw)
+    y_host = nm.forward(a["x"].pin_memory(), dev["W_r"], dev["W1"], dev["W3"], dev["W2"], 32,
+                        host_io=True, router_x=h.pin_memory(), **kw)
+    torch.cuda.synchronize()
+    assert nm.get_last_error() == 0
     assert torch.equal(y_host, y_dev.cpu())
 
 
