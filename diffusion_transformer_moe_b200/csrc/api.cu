@@ -655,8 +655,10 @@ const char* nmoe_stage_name(int stage) {
 }
 
 const char* nmoe_build_info(void) {
-  return "nmoe sm_100a: router tcgen05(bf16)/simt(fp32); select radix; csr lower-bound; "
-         "experts tcgen05+TMA gather4(bf16)/simt(fp32); combine fixed-order";
+  return "nmoe sm_100a: router tcgen05(bf16)/simt(fp32); select radix; token lists in the "
+         "gate/up GEMM's epilogue warps (own kernel beyond 128 experts); experts tcgen05 with "
+         "cp.async row gather (TMA gather4 option) and TMA weights (bf16)/simt(fp32); "
+         "combine fixed-order";
 }
 
 }  // extern "C"
