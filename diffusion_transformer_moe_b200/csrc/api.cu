@@ -656,7 +656,7 @@ const char* nmoe_stage_name(int stage) {
 
 const char* nmoe_build_info(void) {
   return "nmoe sm_100a: router tcgen05(bf16)/simt(fp32); select radix; token lists in the "
-         "gate/up GEMM's epilogue warps (own kernel beyond 128 experts); experts tcgen05 with "
+         "gate/up GEMM's epilogue warps (own kernel when too many experts); experts tcgen05 with "
          "cp.async row gather (TMA gather4 option) and TMA weights (bf16)/simt(fp32); "
          "combine fixed-order";
 }
