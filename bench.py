@@ -51,6 +51,9 @@ def _args():
                          "with +read, then read a second one, so that the written lines "
                          "are written back to HBM before the step's first event instead "
                          "of inside the step")
+    ap.add_argument("--e2e-streams", type=int, default=3,
+                    help="streams the end-to-end steps rotate over (each with its own "
+                         "workspace and pinned output)")
     ap.add_argument("--shared-f", type=int, default=0,
                     help="add a shared SwiGLU expert of this width and the block's gated "
                          "residual (out = x + tanh(clamp(gate2)) * ffn_out)")
@@ -435,21 +438,24 @@ def run_ours(args, w, rank, world, local_rank, dist):
 
     # End to end through the C ABI with host buffers: every step copies its x in from
     # pinned host memory and its out back to pinned host memory inside the call. Steps
-    # alternate between two streams (each with its own workspace and host output), so
-    # one step's copy back overlaps the next step's copy in and layer: PCIe carries both
-    # directions at once. The weights (read every step) are larger than L2, so no flush.
+    # rotate over --e2e-streams streams (each with its own workspace and host output). With
+    # three, a step's copy in never waits behind an earlier step's copy back on its own
+    # stream, so the copies in run back to back while the layer and the copies back of
+    # earlier steps overlap them: PCIe carries both directions at once. The weights
+    # (read every step) are larger than L2, so no flush.
+    n_streams = max(1, args.e2e_streams)
     x_host = a["x"].pin_memory()
-    e2e_streams = [stream, torch.cuda.Stream(device=dev)]
-    e2e_ws = [ws, torch.empty_like(ws)]
-    e2e_out = [torch.empty_like(x_host).pin_memory() for _ in range(2)]
+    e2e_streams = [stream] + [torch.cuda.Stream(device=dev) for _ in range(n_streams - 1)]
+    e2e_ws = [ws] + [torch.empty_like(ws) for _ in range(n_streams - 1)]
+    e2e_out = [torch.empty_like(x_host).pin_memory() for _ in range(n_streams)]
 
     def e2e_step(i):
-        j = i % 2
+        j = i % n_streams
         nm.forward(x_host, W_r, W1, W3, W2, w.C, out=e2e_out[j], workspace=e2e_ws[j],
                    n_segments=w.segments, intermediate=inter, host_io=True,
                    tma_gather=args.tma_gather, stream=e2e_streams[j], **block)
 
-    for i in range(max(2, args.warmup // 2)):
+    for i in range(max(n_streams, args.warmup // 2)):
         e2e_step(i)
     torch.cuda.synchronize()
     e2e_t0 = torch.cuda.Event(enable_timing=True)
@@ -457,10 +463,12 @@ def run_ours(args, w, rank, world, local_rank, dist):
     barrier()
     torch.cuda.synchronize()
     e2e_t0.record(e2e_streams[0])
-    e2e_streams[1].wait_event(e2e_t0)
+    for s_ in e2e_streams[1:]:
+        s_.wait_event(e2e_t0)
     for i in range(K):
         e2e_step(i)
-    e2e_streams[0].wait_stream(e2e_streams[1])
+    for s_ in e2e_streams[1:]:
+        e2e_streams[0].wait_stream(s_)
     e2e_t1.record(e2e_streams[0])
     torch.cuda.synchronize()
     barrier()
@@ -532,7 +540,8 @@ def run_ours(args, w, rank, world, local_rank, dist):
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
                 "ms_per_step": e2e_ms / K,
                 "how": "nmoe_forward_ex with host_io (x copied in, out copied back to pinned "
-                       "host memory inside each call), steps alternating over 2 streams"},
+                       "host memory inside each call), steps rotating over "
+                       f"{n_streams} streams"},
         "clocks": clk,
     }
     if world == 1:
