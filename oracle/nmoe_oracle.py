@@ -21,7 +21,7 @@ expert", and section 6 (packed SwiGLU experts, ``gate_up_proj`` of shape
     weights them by the token's score, optionally normalised by the total score of the
     token's selections and multiplied by ``route_scale``.
 
-Readings taken where the page is silent (each is listed in the design doc as well):
+Readings taken where the page is silent:
   * softmax runs over the experts of one token;
   * selection runs over a flat token axis, or per segment when ``n_segments > 1``
     (the page's per-sample selection); C is the per-segment capacity;
@@ -37,6 +37,8 @@ Readings taken where the page is silent (each is listed in the design doc as well):
   * the page's router input cat([timestep, hidden]) is exactly a per-segment additive
     logit bias ``router_bias[s, e] = temb_s . W_gate[:d_t, e]``
     (see :func:`router_logits_concat` for the literal form);
+  * the gate reads the unmodulated hidden states while the experts transform the
+    block's input: ``router_x`` gives the router its own input; by default both are x;
   * the shared expert (section 6.2: one SwiGLU feed-forward over every token, the
     routed outputs added onto its output) has its own width F_shared, which the page
     does not give;
