@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
   NMOE_OK = 0,
   NMOE_ERR_INVALID_ARG = 1,   /* a size, pointer or alignment the ABI forbids */
-  NMOE_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+  NMOE_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement */
   NMOE_ERR_WORKSPACE = 3,     /* caller workspace too small, or allocation failed */
   NMOE_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
   NMOE_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out */
