@@ -52,7 +52,7 @@ class Rank:
                                                 C.byref(tp), C.byref(te)),
                  "nmoe_workspace_offsets")
         rows = E * self.Ce
-        self.y_f32 = True  # fp32 layers and the default split intermediates keep Y in fp32
+        # Y is fp32: fp32 layers and the default split intermediates keep it so
         self.Y = workspace[y.value: y.value + rows * d * 4].view(torch.float32).view(rows, d)
         self.tok_ptr = workspace[tp.value: tp.value + (T + 1) * 4].view(torch.int32)
         self.tok_ent = workspace[te.value: te.value + rows * 4].view(torch.int32)
