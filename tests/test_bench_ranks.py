@@ -91,3 +91,19 @@ def test_reference_arm_prints_one_contract_line_on_rank_zero():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_algorithmic_bytes_and_flops_of_the_1024px_layer():
+    # the per-kernel minimum traffic the roofline divides by (x, W_r, scores; W1|W3,
+    # gathered rows, H hi+lo; W2, H, Y fp32; Y, out) and the contractions' FLOPs
+    from diffusion_transformer_moe_b200 import inputs as I
+    w = I.WORKLOADS["1024px_cfg"]
+    mb = {k: round(v / 1e6, 1) for k, v in bench.stage_bytes(w).items()}
+    assert (mb["router"], mb["gemm1_swiglu"], mb["gemm2_scale"], mb["combine"]) == \
+        (38.0, 604.0, 369.1, 100.7)
+    gf = {k: round(v / 1e9, 2) for k, v in bench.stage_flops(w).items()}
+    assert gf == {"router": 2.15, "gemm1_swiglu": 68.72, "gemm2_scale": 34.36}
+    # bf16 intermediates move H and Y at two bytes each
+    small = bench.stage_bytes(w, "bf16")
+    assert bench.stage_bytes(w)["gemm2_scale"] - small["gemm2_scale"] == \
+        2 * w.E * w.Ce * w.F + 2 * w.E * w.Ce * w.d
