@@ -262,6 +262,20 @@ def test_separate_router_input_reproduces_the_pages_concat_gate():
     np.testing.assert_allclose(rows["out"], r["out"][[0, 5, 11]], rtol=1e-13, atol=1e-15)
 
 
+def test_segments_are_independent_layers():
+    # section 6.2 selects per sample: a layer over n_segments samples is n_segments
+    # independent layers, one per sample, each with that sample's bias row
+    a = _small(36, 6, 5, 4, seed=23)
+    bias = np.random.default_rng(4).normal(size=(3, 5))
+    whole = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=4, n_segments=3,
+                    router_bias=bias, combine="normalized", route_scale=2.5)
+    for g in range(3):
+        part = O.layer(a["x"][12 * g:12 * (g + 1)], a["W_r"], a["W1"], a["W3"], a["W2"], C=4,
+                       router_bias=bias[g:g + 1], combine="normalized", route_scale=2.5)
+        np.testing.assert_array_equal(whole["out"][12 * g:12 * (g + 1)], part["out"])
+        assert np.array_equal(whole["idx"][:, 4 * g:4 * (g + 1)], part["idx"] + 12 * g)
+
+
 def test_sampled_rows_match_full_layer():
     a = _small(40, 8, 5, 6, seed=15)
     r = O.layer(a["x"], a["W_r"], a["W1"], a["W3"], a["W2"], C=8, combine="normalized",

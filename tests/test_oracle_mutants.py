@@ -35,6 +35,9 @@ MUTANTS = {
                              "order = np.lexsort((tok, col))"),
     "chosen tokens unsorted": ("chosen.append(np.sort(tok[order[:C]]))",
                                "chosen.append(tok[order[:C]])"),
+    "selection over all tokens, not per segment": (
+        "col = s[g * S:(g + 1) * S, e].astype(F64)\n            tok = np.arange(g * S, (g + 1) * S)",
+        "col = s[:, e].astype(F64)\n            tok = np.arange(T)"),
     "scores not rounded to fp32": ("return _f64(p).astype(np.float32)", "return _f64(p)"),
     "router bias subtracted": ("l = l + np.repeat(b, S, axis=0)",
                                "l = l - np.repeat(b, S, axis=0)"),
