@@ -54,6 +54,9 @@ def _args():
     ap.add_argument("--e2e-streams", type=int, default=3,
                     help="streams the end-to-end steps rotate over (each with its own "
                          "workspace and pinned output)")
+    ap.add_argument("--tensor-workload", default="batch4_1024px_cfg",
+                    help="a tensor-bound workload timed in the same run (its own key of "
+                         "the JSON line); empty to skip")
     ap.add_argument("--shared-f", type=int, default=0,
                     help="add a shared SwiGLU expert of this width and the block's gated "
                          "residual (out = x + tanh(clamp(gate2)) * ffn_out)")
@@ -70,51 +73,72 @@ def _peaks():
     return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, source="fallback")
 
 
-def _l2_note(mode):
-    if mode == "write":
-        return "flushed before every timed step (256 MiB write, outside the step's events)"
-    return ("flushed before every timed step (256 MiB write, then a 256 MiB read that "
-            "evicts the written lines; both outside the step's events)")
+L2_NOTE = {
+    "write+read": ("GPU arm: L2 flushed before every timed step (a 256 MiB write, then a "
+                   "256 MiB read that evicts the written lines; both outside the step's "
+                   "events); the CPU reference arm has no L2 flush"),
+    "write": ("GPU arm: L2 flushed before every timed step (a 256 MiB write, outside the "
+              "step's events); the CPU reference arm has no L2 flush"),
+}
 
 
-def _workload_config(w, intermediate, l2_flush="write+read"):
+def _workload_config(w, l2_flush="write+read"):
+    """The `config` object of the JSON line: the same for both arms on one workload."""
     return {
         "workload": f"{w.name}: T={w.T} tokens, d={w.d}, E={w.E} experts, SwiGLU F={w.F}, "
                     f"capacity_factor={w.capacity_factor:g} (C={w.C}"
                     + (f" per segment of {w.T // w.segments} tokens)" if w.segments > 1 else ")"),
         "T": w.T, "d": w.d, "E": w.E, "F": w.F, "C": w.C, "segments": w.segments,
-        "intermediates": intermediate,
-        "l2": _l2_note(l2_flush),
+        "l2": L2_NOTE[l2_flush],
     }
 
 
-# ---- algorithmic bytes / flops of each stage (minimum traffic the method must move) ----
+# ---- algorithmic bytes / flops of each stage ----------------------------------------------
+#
+# Algorithmic bytes are the minimum each stage must move with every intermediate in the
+# layer's own type (bf16 H and Y for bf16 layers): router x + W_r in, scores + scores_t
+# out; gate/up GEMM W1|W3, the gathered rows and H; down GEMM W2, H and Y; combine Y and
+# out. These are the roofline numerators. Design bytes are what this implementation
+# moves on purpose beyond them: with split intermediates H is a bf16 hi/lo pair and Y is
+# fp32 (4 bytes each), plus the small index arrays the kernels read.
 
-def stage_bytes(w, intermediate="split", shared_f=0):
-    """Bytes each stage must read + write at least, per layer call (with a shared expert
-    of width shared_f: its weights, its H and Y rows, and the residual read)."""
-    T, d, E, F, Ce = w.T, w.d, w.E, w.F, w.Ce
-    hb = 4 if intermediate == "split" else 2   # H: bf16 hi+lo pair, or bf16
-    yb = 4 if intermediate == "split" else 2   # Y: fp32, or bf16
-    Fs = shared_f
-    sh = {"gemm1_swiglu": 2 * 2 * d * Fs + 2 * T * d + hb * T * Fs,
-          "gemm2_scale": 2 * Fs * d + hb * T * Fs + yb * T * d,
-          "combine": yb * T * d + 2 * T * d} if Fs else {}
-    return {k: v + sh.get(k, 0) for k, v in _routed_bytes(T, d, E, F, Ce, hb, yb).items()}
-
-
-def _routed_bytes(T, d, E, F, Ce, hb, yb):
-    return {
-        "router": 2 * T * d + 2 * d * E + 2 * 4 * T * E,          # x, W_r in; scores, scores_t out
-        "select": 4 * T * E + 8 * E * Ce,                          # scores_t in; idx, gate out
-        "csr": 4 * E * Ce + 4 * (T + 1) + 4 * E * Ce,              # idx in; tok_ptr, tok_ent out
-        "gemm1_swiglu": 2 * 2 * E * d * F + 2 * E * Ce * d + hb * E * Ce * F,
-        "gemm2_scale": 2 * E * F * d + hb * E * Ce * F + 4 * E * Ce + yb * E * Ce * d,
-        "combine": yb * E * Ce * d + 4 * (T + 1) + 4 * E * Ce + 2 * T * d,
+def stage_bytes(w, shared_f=0):
+    """Algorithmic bytes per stage and layer call (with a shared expert of width
+    shared_f: its weights, its gathered rows, H and Y, and the residual read)."""
+    T, d, E, F, Ce, Fs = w.T, w.d, w.E, w.F, w.Ce, shared_f
+    b = {
+        "router": 2 * T * d + 2 * d * E + 2 * 4 * T * E,
+        "select": 4 * T * E + 8 * E * Ce,
+        "csr": 4 * E * Ce + 4 * (T + 1) + 4 * E * Ce,
+        "gemm1_swiglu": 2 * 2 * E * d * F + 2 * E * Ce * d + 2 * E * Ce * F,
+        "gemm2_scale": 2 * E * F * d + 2 * E * Ce * F + 2 * E * Ce * d,
+        "combine": 2 * E * Ce * d + 2 * T * d,
     }
+    if Fs:
+        b["gemm1_swiglu"] += 2 * 2 * d * Fs + 2 * T * d + 2 * T * Fs
+        b["gemm2_scale"] += 2 * Fs * d + 2 * T * Fs + 2 * T * d
+        b["combine"] += 2 * T * d + 2 * T * d
+    return b
 
 
-def stage_flops(w, intermediate="split", shared_f=0):
+def stage_design_bytes(w, intermediate="split", shared_f=0):
+    """Bytes each stage moves as built: split intermediates keep H as a bf16 hi/lo pair
+    and Y in fp32; the down GEMM also reads the combine weights and the rows' token-major
+    positions, the combine the token lists."""
+    T, d, E, F, Ce, Fs = w.T, w.d, w.E, w.F, w.Ce, shared_f
+    hb = yb = 4 if intermediate == "split" else 2
+    b = dict(stage_bytes(w, shared_f))
+    b["gemm1_swiglu"] += (hb - 2) * E * Ce * F + 4 * E * Ce
+    b["gemm2_scale"] += (hb - 2) * E * Ce * F + (yb - 2) * E * Ce * d + 8 * E * Ce
+    b["combine"] += (yb - 2) * E * Ce * d + 4 * (T + 1)
+    if Fs:
+        b["gemm1_swiglu"] += (hb - 2) * T * Fs
+        b["gemm2_scale"] += (hb - 2) * T * Fs + (yb - 2) * T * d
+        b["combine"] += (yb - 2) * T * d
+    return b
+
+
+def stage_flops(w, shared_f=0):
     """Algorithmic FLOPs of the contractions (the split intermediates' second set of
     down-projection MMAs is executed work, not counted here)."""
     T, d, E, F, Ce, Fs = w.T, w.d, w.E, w.F, w.Ce, shared_f
@@ -149,7 +173,8 @@ STAGE_SOURCE = {"router": "router_sm100.cu", "select": "select.cu", "csr": "sele
 # ---- clocks during the timed region ----------------------------------------------------
 
 class ClockSampler:
-    """Samples SM clocks and clock-event reasons every 10 ms through NVML (read only)."""
+    """Samples SM clocks and clock-event reasons every millisecond through NVML (read
+    only), so that even a timed region of a few milliseconds holds several samples."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
@@ -198,7 +223,7 @@ class ClockSampler:
             except Exception as e:
                 self.err = f"nvml sample failed: {type(e).__name__}"
                 return
-            self._stop.wait(0.01)
+            self._stop.wait(0.001)
 
     def stop(self):
         if self.err and not self.samples:
@@ -300,7 +325,9 @@ def run_reference(args, w, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(_workload_config(w, "fp64 oracle"), l2="n/a (host CPU)"),
+        "config": _workload_config(w, args.l2_flush),
+        "impl_options": {"arithmetic": "fp64 numpy oracle on the host cores"},
+        "parallelism": "one host process (rank 0)",
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _oracle_threads(),
                          "kind": "oracle", "sample": f"each step: {what}"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -329,221 +356,292 @@ def replica_throughput(T, world, K, ms):
 
 # ---- our CUDA path ---------------------------------------------------------------------
 
-def run_ours(args, w, rank, world, local_rank, dist):
+def _device_inputs(w, seed, dev, shared_f):
+    import torch
+    from diffusion_transformer_moe_b200 import inputs as I
+    a = I.make_inputs(w, seed=seed)
+    d = {k: v.to(dev) for k, v in a.items()}
+    block = {}
+    if shared_f:
+        g = torch.Generator().manual_seed(1000 + seed)
+        block = dict(shared=tuple((torch.randn(*sh, generator=g) / sh[0] ** 0.5)
+                                  .to(d["x"].dtype).to(dev)
+                                  for sh in ((w.d, shared_f), (w.d, shared_f),
+                                             (shared_f, w.d))),
+                     residual=d["x"],
+                     gate2=torch.randn(w.segments, w.d, generator=g).to(dev))
+    return a, d, block
+
+
+class Flush:
+    """Before every timed step: write a buffer twice the size of L2; with "write+read",
+    then read a second one, so that the written lines are written back here and the step
+    starts from an L2 that holds nothing of its own and owes no write-back (the state
+    ncu's cache control gives each kernel)."""
+
+    def __init__(self, mode, dev):
+        import torch
+        self.buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.clean = (torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+                      if mode == "write+read" else None)
+
+    def __call__(self):
+        self.buf.zero_()
+        if self.clean is not None:
+            self.clean.amax()
+
+
+def _timed_steps(step, K, flush, stream, barrier, per_step_events=True):
+    """Exactly K steps between a barrier + synchronize on both sides; the L2 flush runs
+    before each step, outside its CUDA events (recorded on the launching stream).
+    Returns the summed milliseconds of the K steps."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return sum(s_.elapsed_time(e_) for s_, e_ in ev)
+
+
+def measure(args, w, seed, dev, dist, K, W, inter, shared_f=0, extras=True):
+    """Times the layer on workload w: K steps back to back (the headline), K traced steps
+    (per-stage events), and with `extras` a replayed CUDA graph and the end-to-end
+    steps through host buffers. Returns the per-rank measurements."""
     import torch
     import diffusion_transformer_moe_b200 as nm
-    from diffusion_transformer_moe_b200 import inputs as I
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    a = I.make_inputs(w, seed=rank)
-    x = a["x"].to(dev)
-    W_r, W1, W3, W2 = (a[k].to(dev) for k in ("W_r", "W1", "W3", "W2"))
-    inter = args.intermediate
+    a, d, block = _device_inputs(w, seed, dev, shared_f)
+    x, W_r, W1, W3, W2 = d["x"], d["W_r"], d["W1"], d["W3"], d["W2"]
     ws = torch.empty(nm.workspace_size(w.T, w.d, w.E, w.F, w.C, intermediate=inter,
                                        n_segments=w.segments, host_io=True,
-                                       shared_f=args.shared_f or None),
+                                       shared_f=shared_f or None),
                      dtype=torch.uint8, device=dev)
     out = torch.empty_like(x)
-    block = {}
-    if args.shared_f:
-        g = torch.Generator().manual_seed(1000 + rank)
-        Fs = args.shared_f
-        block = dict(shared=tuple((torch.randn(*sh, generator=g) / sh[0] ** 0.5)
-                                  .to(x.dtype).to(dev)
-                                  for sh in ((w.d, Fs), (w.d, Fs), (Fs, w.d))),
-                     residual=x, gate2=torch.randn(w.segments, w.d, generator=g).to(dev))
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    clean = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev) \
-        if args.l2_flush == "write+read" else None
-
-    def l2_flush():
-        # the write leaves L2 full of dirty lines; reading another buffer of twice its
-        # size writes them back here, so the step starts from an L2 that holds nothing
-        # of its own and owes no write-back (the state ncu's cache control gives)
-        flush.zero_()
-        if clean is not None:
-            clean.amax()
+    flush = Flush(args.l2_flush, dev)
     stream = torch.cuda.current_stream()
-    K = args.steps
     trace = nm.Trace(K)
 
     def step(tr=None):
         nm.forward(x, W_r, W1, W3, W2, w.C, out=out, workspace=ws, intermediate=inter,
-                   n_segments=w.segments,
-                   trace=tr, tma_gather=args.tma_gather, **block)
+                   n_segments=w.segments, trace=tr, tma_gather=args.tma_gather, **block)
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        l2_flush()
+    for _ in range(W):
+        flush()
         step()
     torch.cuda.synchronize()
     if nm.get_last_error() != 0:
         raise RuntimeError("device-side check failed during warm-up")
 
-    def timed(tr):
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(K)]
-        barrier()
-        torch.cuda.synchronize()
-        for i in range(K):
-            l2_flush()
-            ev[i][0].record(stream)
-            step(tr)
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        return sum(s.elapsed_time(e) for s, e in ev)
-
-    # the timed region: K whole-layer steps, launched back to back as a user would
-    clocks = ClockSampler(local_rank)
+    # the timed region: K whole-layer steps, launched back to back as a user would,
+    # with the SM clocks sampled throughout
+    clocks = ClockSampler(dev.index)
     clocks.start()
-    ms = timed(None)
+    ms = _timed_steps(step, K, flush, stream, barrier)
     clk = clocks.stop()
-    # per-stage times: K more steps with CUDA events recorded between the stages (the
-    # events keep the stages from overlapping their launches, so this pass is not the
-    # headline number)
-    traced_ms = timed(trace)
+    # per-stage times: K more steps with CUDA events between the stages (the events keep
+    # the stages from overlapping their launches, so this pass is not the headline)
+    traced_ms = _timed_steps(lambda: step(trace), K, flush, stream, barrier)
     stage_ms, ncalls = trace.read()
-    # the same step replayed from a CUDA graph (one captured layer call; the L2 flush
-    # stays outside the graph and the events)
-    graph = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream(device=dev)
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        step()
-    stream.wait_stream(side)
-    torch.cuda.synchronize()
-    with torch.cuda.graph(graph):
-        step()
-    torch.cuda.synchronize()
-    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(K):
-        l2_flush()
-        gev[i][0].record(stream)
-        graph.replay()
-        gev[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    graph_ms = sum(a_.elapsed_time(b_) for a_, b_ in gev)
-    del graph
+    trace.close()
+    r = dict(ms=ms, traced_ms=traced_ms, clocks=clk,
+             stage_ms={k: v / max(ncalls, 1) for k, v in stage_ms.items()},
+             launches=nm.kernels_per_call(w.T, w.d, w.E, w.F, w.C, intermediate=inter,
+                                          n_segments=w.segments, shared_f=shared_f or None))
+    if extras:
+        # the same step replayed from a CUDA graph (one captured layer call; the flush
+        # stays outside the graph and the events)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize()
+        r["graph_ms"] = _timed_steps(graph.replay, K, flush, stream, barrier)
+        del graph
+        r.update(_e2e(args, w, a, d, block, ws, inter, K, W, dev, barrier))
     if nm.get_last_error() != 0:
         raise RuntimeError("device-side check failed during the timed steps")
+    return r
 
-    # End to end through the C ABI with host buffers: every step copies its x in from
-    # pinned host memory and its out back to pinned host memory inside the call. Steps
-    # rotate over --e2e-streams streams (each with its own workspace and host output). With
-    # three, a step's copy in never waits behind an earlier step's copy back on its own
-    # stream, so the copies in run back to back while the layer and the copies back of
-    # earlier steps overlap them: PCIe carries both directions at once. The weights
-    # (read every step) are larger than L2, so no flush.
+
+def _e2e(args, w, a, d, block, ws, inter, K, W, dev, barrier):
+    """End to end through the C ABI with host buffers: every step copies its x in from
+    pinned host memory and its out back to pinned host memory inside the call. Steps
+    rotate over --e2e-streams streams (each with its own workspace and host output);
+    with three, a step's copy in never waits behind an earlier step's copy back on its
+    own stream, so the copies in run back to back while the layer and the copies back of
+    earlier steps overlap them (PCIe carries both directions at once). The weights, read
+    every step, are larger than L2, so no flush."""
+    import torch
+    import diffusion_transformer_moe_b200 as nm
     n_streams = max(1, args.e2e_streams)
+    stream = torch.cuda.current_stream()
     x_host = a["x"].pin_memory()
-    e2e_streams = [stream] + [torch.cuda.Stream(device=dev) for _ in range(n_streams - 1)]
-    e2e_ws = [ws] + [torch.empty_like(ws) for _ in range(n_streams - 1)]
-    e2e_out = [torch.empty_like(x_host).pin_memory() for _ in range(n_streams)]
+    streams = [stream] + [torch.cuda.Stream(device=dev) for _ in range(n_streams - 1)]
+    wss = [ws] + [torch.empty_like(ws) for _ in range(n_streams - 1)]
+    outs = [torch.empty_like(x_host).pin_memory() for _ in range(n_streams)]
 
     def e2e_step(i):
         j = i % n_streams
-        nm.forward(x_host, W_r, W1, W3, W2, w.C, out=e2e_out[j], workspace=e2e_ws[j],
-                   n_segments=w.segments, intermediate=inter, host_io=True,
-                   tma_gather=args.tma_gather, stream=e2e_streams[j], **block)
+        nm.forward(x_host, d["W_r"], d["W1"], d["W3"], d["W2"], w.C, out=outs[j],
+                   workspace=wss[j], n_segments=w.segments, intermediate=inter,
+                   host_io=True, tma_gather=args.tma_gather, stream=streams[j], **block)
 
-    for i in range(max(n_streams, args.warmup // 2)):
+    for i in range(max(n_streams, W // 2)):
         e2e_step(i)
     torch.cuda.synchronize()
-    e2e_t0 = torch.cuda.Event(enable_timing=True)
-    e2e_t1 = torch.cuda.Event(enable_timing=True)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    e2e_t0.record(e2e_streams[0])
-    for s_ in e2e_streams[1:]:
-        s_.wait_event(e2e_t0)
+    t0.record(streams[0])
+    for s_ in streams[1:]:
+        s_.wait_event(t0)
     for i in range(K):
         e2e_step(i)
-    for s_ in e2e_streams[1:]:
-        e2e_streams[0].wait_stream(s_)
-    e2e_t1.record(e2e_streams[0])
+    for s_ in streams[1:]:
+        streams[0].wait_stream(s_)
+    t1.record(streams[0])
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e2e_t0.elapsed_time(e2e_t1)
-    if nm.get_last_error() != 0:
-        raise RuntimeError("device-side check failed during the end-to-end steps")
-    out_host = e2e_out[0]
+    return dict(e2e_ms=t0.elapsed_time(t1), e2e_streams=n_streams,
+                h2d=x_host.numel() * x_host.element_size(),
+                d2h=outs[0].numel() * outs[0].element_size())
 
-    ms, e2e_ms, traced_ms, graph_ms = max_over_ranks([ms, e2e_ms, traced_ms, graph_ms], dist,
-                                                     dev)
+
+def _stage_report(w, stage_ms, peaks, inter, shared_f):
+    """Per-stage µs, algorithmic GB/s and fraction of HBM, FLOP rate and fraction of the
+    sustained bf16 peak, and the bytes as built."""
+    sb = stage_bytes(w, shared_f)
+    db = stage_design_bytes(w, inter, shared_f)
+    sf = stage_flops(w, shared_f)
+    out = {}
+    for name, ms_ in stage_ms.items():
+        s_ = ms_ / 1e3
+        st = {"us": s_ * 1e6, "GB/s": sb[name] / s_ / 1e9,
+              "hbm_frac": sb[name] / s_ / 1e9 / peaks["hbm"],
+              "design_GB/s": db[name] / s_ / 1e9}
+        if name in sf:
+            st["TFLOP/s"] = sf[name] / s_ / 1e12
+            st["tensor_frac"] = st["TFLOP/s"] / peaks["tensor_sustained"]
+            if name == "gemm2_scale" and inter == "split":
+                # the hi and lo halves of H each run their own MMAs into one accumulator
+                st["executed_TFLOP/s"] = 2 * st["TFLOP/s"]
+        out[name] = st
+    return out
+
+
+def _roofline(w, stage_ms, peaks, inter, shared_f):
+    """The dominant kernel's roofline: the larger of its algorithmic byte time and its
+    FLOP time at the measured peaks (the sustained tensor figure: the kernel runs inside
+    a long step)."""
+    sb = stage_bytes(w, shared_f)
+    db = stage_design_bytes(w, inter, shared_f)
+    sf = stage_flops(w, shared_f)
+    dom = max(stage_ms, key=lambda k: stage_ms[k])
+    dom_s = stage_ms[dom] / 1e3
+    src = "MEASURED_PEAKS.json" if peaks["source"] == "measured" else "fallback"
+    if sf.get(dom, 0) / (peaks["tensor_sustained"] * 1e12) > sb[dom] / (peaks["hbm"] * 1e9):
+        achieved = sf[dom] / dom_s / 1e12
+        return {"kernel": dom, "bound": "tensor", "achieved": achieved,
+                "peak": peaks["tensor_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["tensor_sustained"],
+                "algorithmic_flops_per_launch": sf[dom],
+                "peak_source": f"{src} bf16_tflops_sustained", "traffic": None}
+    achieved = sb[dom] / dom_s / 1e9
+    return {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm"],
+            "unit": "GB/s", "frac": achieved / peaks["hbm"],
+            "algorithmic_bytes_per_launch": sb[dom],
+            "design_bytes_per_launch": db[dom],
+            "design_frac": db[dom] / dom_s / 1e9 / peaks["hbm"],
+            "peak_source": f"{src} hbm_gbs", "traffic": _traffic(dom, w.name)}
+
+
+def run_ours(args, w, rank, world, local_rank, dist):
+    import torch
+    from diffusion_transformer_moe_b200 import inputs as I
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inter = args.intermediate
+    K, W = args.steps, args.warmup
+    m = measure(args, w, rank, dev, dist, K, W, inter, args.shared_f)
+    tb = None
+    if args.tensor_workload and args.tensor_workload != w.name:
+        torch.cuda.empty_cache()
+        wt = I.WORKLOADS[args.tensor_workload]
+        tb = measure(args, wt, rank, dev, dist, K, W, inter, 0, extras=False)
+    keys = ["ms", "traced_ms", "graph_ms", "e2e_ms"] + (["tb_ms"] if tb else [])
+    vals = [m["ms"], m["traced_ms"], m["graph_ms"], m["e2e_ms"]] + ([tb["ms"]] if tb else [])
+    mx = dict(zip(keys, max_over_ranks(vals, dist, dev)))
     if rank != 0:
         return
 
     peaks = _peaks()
-    per_step_s = ms / 1e3 / K
-    value = replica_throughput(w.T, world, K, ms)
-    sb = stage_bytes(w, inter, args.shared_f)
-    sf = stage_flops(w, inter, args.shared_f)
-    stages = {}
-    for name, tot in stage_ms.items():
-        avg_s = tot / 1e3 / max(ncalls, 1)
-        st = {"us": avg_s * 1e6, "GB/s": sb[name] / avg_s / 1e9,
-              "hbm_frac": sb[name] / avg_s / 1e9 / peaks["hbm"]}
-        if name in sf:
-            st["TFLOP/s"] = sf[name] / avg_s / 1e12
-        stages[name] = st
-    dom = max(stage_ms, key=lambda k: stage_ms[k])
-    dom_s = stage_ms[dom] / 1e3 / max(ncalls, 1)
-    # the dominant kernel's bound: the larger of its byte time and its FLOP time at the
-    # measured peaks (the sustained tensor figure: the kernel runs inside a long step)
-    src = "MEASURED_PEAKS.json" if peaks["source"] == "measured" else "fallback"
-    if sf.get(dom, 0) / (peaks["tensor_sustained"] * 1e12) > sb[dom] / (peaks["hbm"] * 1e9):
-        achieved = sf[dom] / dom_s / 1e12
-        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved,
-                "peak": peaks["tensor_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["tensor_sustained"],
-                "algorithmic_flops_per_launch": sf[dom],
-                "peak_source": f"{src} bf16_tflops_sustained"}
-    else:
-        achieved = sb[dom] / dom_s / 1e9
-        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm"],
-                "unit": "GB/s", "frac": achieved / peaks["hbm"],
-                "algorithmic_bytes_per_launch": sb[dom],
-                "peak_source": f"{src} hbm_gbs"}
-    roof["traffic"] = _traffic(dom, w.name)
+    per_step_s = mx["ms"] / 1e3 / K
     flops = w.expert_flops() + w.router_flops() + 6.0 * w.T * w.d * args.shared_f
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(_workload_config(w, inter, args.l2_flush), parallelism=f"replicas x{world}",
-                       gather="tma gather4" if args.tma_gather else "cp.async",
-                       **({"shared_f": args.shared_f,
-                           "block": "x + tanh(clamp(gate2, -2, 2)) * (shared + routed)"}
-                          if args.shared_f else {})),
+        "metric": METRIC, "value": replica_throughput(w.T, world, K, mx["ms"]),
+        "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": mx["ms"] / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _workload_config(w, args.l2_flush),
+        "parallelism": f"replicas x{world} (one independent layer per GPU, no exchange)",
+        "impl_options": {"intermediates": inter,
+                         "gather": "tma gather4" if args.tma_gather else "cp.async",
+                         **({"shared_f": args.shared_f,
+                             "block": "x + tanh(clamp(gate2, -2, 2)) * (shared + routed)"}
+                            if args.shared_f else {})},
         "tflops": flops / per_step_s / 1e12,
         "tensor_frac_of_layer": flops / per_step_s / 1e12 / peaks["tensor_sustained"],
-        "roofline": roof,
-        "stages": stages,
-        "traced_ms_per_step": traced_ms / K,
-        "graph_replay": {"ms_per_step": graph_ms / K,
-                         "value": replica_throughput(w.T, world, K, graph_ms),
+        "roofline": _roofline(w, m["stage_ms"], peaks, inter, args.shared_f),
+        "stages": _stage_report(w, m["stage_ms"], peaks, inter, args.shared_f),
+        "traced_ms_per_step": mx["traced_ms"] / K,
+        "graph_replay": {"ms_per_step": mx["graph_ms"] / K,
+                         "value": replica_throughput(w.T, world, K, mx["graph_ms"]),
                          "how": "one captured layer call, replayed K times"},
-        "gpu_launches": K * nm.kernels_per_call(w.T, w.d, w.E, w.F, w.C, intermediate=inter,
-                                                n_segments=w.segments,
-                                                shared_f=args.shared_f or None),
-        "e2e": {"value": replica_throughput(w.T, world, K, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
-                "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
-                "ms_per_step": e2e_ms / K,
+        "gpu_launches": K * m["launches"],
+        "e2e": {"value": replica_throughput(w.T, world, K, mx["e2e_ms"]), "unit": "tokens/s",
+                "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"],
+                "ms_per_step": mx["e2e_ms"] / K,
                 "how": "nmoe_forward_ex with host_io (x copied in, out copied back to pinned "
                        "host memory inside each call), steps rotating over "
-                       f"{n_streams} streams"},
-        "clocks": clk,
+                       f"{m['e2e_streams']} streams"},
+        "clocks": m["clocks"],
     }
+    if tb is not None:
+        wt = I.WORKLOADS[args.tensor_workload]
+        t_s = mx["tb_ms"] / 1e3 / K
+        tflops = wt.expert_flops() + wt.router_flops()
+        st = _stage_report(wt, tb["stage_ms"], peaks, inter, 0)
+        line["tensor_bound"] = {
+            "config": _workload_config(wt, args.l2_flush), "intermediates": inter,
+            "steps": K, "warmup": W, "ms_per_step": mx["tb_ms"] / K,
+            "value": replica_throughput(wt.T, world, K, mx["tb_ms"]), "unit": "tokens/s",
+            "tflops": tflops / t_s / 1e12,
+            "tensor_frac_of_layer": tflops / t_s / 1e12 / peaks["tensor_sustained"],
+            "peak": peaks["tensor_sustained"],
+            "peak_source": ("MEASURED_PEAKS.json" if peaks["source"] == "measured"
+                            else "fallback") + " bf16_tflops_sustained",
+            "gemms": {k: st[k] for k in ("gemm1_swiglu", "gemm2_scale")},
+            "stages": st, "gpu_launches": K * tb["launches"],
+            "clocks": tb["clocks"],
+        }
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
