@@ -14,7 +14,10 @@ import threading
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libnmoe.so")
+# NMOE_DEBUG=1 loads the debug build (index and span checks in the kernels, reported
+# through the error word); both are this package's own CUDA library.
+DEBUG = os.environ.get("NMOE_DEBUG", "0") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libnmoe_debug.so" if DEBUG else "libnmoe.so")
 
 NMOE_BF16, NMOE_F32 = 0, 1
 SCORE = {"softmax": 0, "sigmoid": 1}
@@ -55,6 +58,7 @@ class Options(C.Structure):
         ("shared_w2", C.c_void_p), ("shared_f", C.c_int64), ("residual", C.c_void_p),
         ("gate2", C.c_void_p), ("expert_begin", C.c_int64), ("expert_end", C.c_int64),
         ("skip_combine", C.c_int), ("router_x", C.c_void_p),
+        ("wait_budget_ns", C.c_uint64),
     ]
 
 
@@ -113,7 +117,7 @@ def lib() -> C.CDLL:
             L.nmoe_workspace_offsets.argtypes = [_i64] * 5 + [C.POINTER(Options)] + [
                 C.POINTER(C.c_size_t)] * 3
             L.nmoe_workspace_offsets.restype = C.c_int
-            L.nmoe_ep_rows.argtypes = [_vp, _vp] + [_i64] * 7 + [_vp, _vp, _vp]
+            L.nmoe_ep_rows.argtypes = [_vp, _vp] + [_i64] * 7 + [_vp, _i64, _vp, _vp]
             L.nmoe_ep_rows.restype = C.c_int
             L.nmoe_rows_gather.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp]
             L.nmoe_rows_gather.restype = C.c_int
@@ -168,12 +172,13 @@ def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
             host_io=False, trace=None, intermediate="split", out_f32=False,
             tma_gather=False, shared=None, shared_f=None, residual=None,
             gate2=None, expert_begin=0, expert_end=0, skip_combine=False,
-            router_x=None) -> Options:
+            router_x=None, wait_budget_ns=0) -> Options:
     """nmoe_options from keyword arguments. ``shared`` = (Ws1 [d,Fs], Ws3 [d,Fs],
     Ws2 [Fs,d]) device tensors adds the shared expert; ``shared_f`` alone (no tensors)
     only sizes a workspace for one. ``residual`` [T,d] and ``gate2`` fp32
     [n_segments,d] add the block's gated residual. ``router_x`` [T,d] is what the
-    router scores instead of x (on the host with ``host_io``)."""
+    router scores instead of x (on the host with ``host_io``). ``wait_budget_ns`` bounds
+    every device-side pipeline wait (0: the library's default)."""
     o = Options()
     lib().nmoe_options_init(C.byref(o))
     o.dtype = dtype
@@ -208,6 +213,7 @@ def options(dtype=NMOE_BF16, score_fn="softmax", combine="raw", route_scale=1.0,
     o.expert_end = int(expert_end)
     o.skip_combine = 1 if skip_combine else 0
     o.router_x = _ptr(router_x)
+    o.wait_budget_ns = int(wait_budget_ns)
     return o
 
 

@@ -100,6 +100,8 @@ Shape make_shape(int64_t T, int64_t d, int64_t E, int64_t F, int64_t C, int64_t 
   s.T = (int)T; s.d = (int)d; s.E = (int)E; s.F = (int)F; s.C = (int)C;
   s.n_seg = (int)n_seg; s.S = (int)(T / n_seg); s.Ce = (int)(n_seg * C);
   s.pdl = true;
+  s.wait_ns = nmoe::kDefaultWaitNs;
+  s.y_rows = (int64_t)s.E * s.Ce;
   return s;
 }
 
@@ -222,6 +224,8 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   if (has_shared && (int64_t)s.E * s.Ce + s.T >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
   // per-stage events sit between the launches, so traced calls run without overlap
   s.pdl = o.trace == nullptr;
+  if (o.wait_budget_ns != 0) s.wait_ns = o.wait_budget_ns;
+  if (has_shared) s.y_rows += s.T;
   const Layout L = make_layout(s, o.dtype, o);
 
   char* ws = static_cast<char*>(o.workspace);
@@ -380,6 +384,7 @@ void nmoe_options_init(nmoe_options* o) {
   o->expert_end = 0;
   o->skip_combine = 0;
   o->router_x = nullptr;
+  o->wait_budget_ns = 0;
 }
 
 nmoe_status nmoe_router(const void* x, const void* W_r, int64_t T, int64_t d, int64_t E,
@@ -463,16 +468,19 @@ nmoe_status nmoe_workspace_offsets(int64_t T, int64_t d, int64_t E, int64_t F, i
 
 nmoe_status nmoe_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent, int64_t T, int64_t E,
                          int64_t Ce, int64_t t_begin, int64_t t_end, int64_t e_begin,
-                         int64_t e_end, int32_t* rows, int32_t* count, nmoe_stream_t stream) {
-  if (!tok_ptr || !tok_ent || !rows || !count) return NMOE_ERR_INVALID_ARG;
+                         int64_t e_end, int32_t* rows, int64_t capacity, int32_t* count,
+                         nmoe_stream_t stream) {
+  if (!tok_ptr || !tok_ent || !count) return NMOE_ERR_INVALID_ARG;
   if (T < 1 || E < 1 || Ce < 1 || E * Ce >= (int64_t(1) << 31)) return NMOE_ERR_INVALID_ARG;
   if (t_begin < 0 || t_end < t_begin || t_end > T) return NMOE_ERR_INVALID_ARG;
   if (e_begin < 0 || e_end < e_begin || e_end > E) return NMOE_ERR_INVALID_ARG;
+  if (capacity < 0 || capacity >= (int64_t(1) << 31) || (capacity > 0 && !rows))
+    return NMOE_ERR_INVALID_ARG;
   DevState* ds = nullptr;
   nmoe_status v = dev_state(&ds);
   if (v != NMOE_OK) return v;
   if (nmoe::launch_ep_rows(tok_ptr, tok_ent, (int)E, (int)Ce, (int)t_begin, (int)t_end,
-                           (int)e_begin, (int)e_end, rows, count,
+                           (int)e_begin, (int)e_end, rows, (int)capacity, count, ds->err,
                            static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return NMOE_ERR_CUDA;
@@ -527,6 +535,7 @@ nmoe_status nmoe_combine_tokens(const void* Y, const int32_t* tok_ptr, int64_t T
   // the token range as a layer of its own: its tok_ptr entries, its output rows
   Shape s = make_shape(t_end - t_begin, d, 1, 8, 1, 1);
   s.pdl = false;
+  s.y_rows = int64_t(1) << 40;  // Y's row count is not passed: only the order is checked
   if (nmoe::launch_combine(Y, tok_ptr + t_begin, s, y_dtype == NMOE_F32,
                            out_dtype == NMOE_F32, out, nullptr, false, nullptr, ds->err,
                            ds->sm_count, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
@@ -658,7 +667,11 @@ const char* nmoe_build_info(void) {
   return "nmoe sm_100a: router tcgen05(bf16)/simt(fp32); select radix; token lists in the "
          "gate/up GEMM's epilogue warps (own kernel when too many experts); experts tcgen05 with "
          "cp.async row gather (TMA gather4 option) and TMA weights (bf16)/simt(fp32); "
-         "combine fixed-order";
+         "combine fixed-order"
+#ifdef NMOE_DEBUG
+         "; debug checks (gathered indices, row positions, token-list spans)"
+#endif
+      ;
 }
 
 }  // extern "C"

@@ -117,7 +117,8 @@ template <typename TY, typename TO>
 __global__ void __launch_bounds__(512)
 combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, int Tn, int d,
                int tok_per_cta, TO* __restrict__ out, const void* __restrict__ residual,
-               int res_bf16, const float* __restrict__ gate2, int S) {
+               int res_bf16, const float* __restrict__ gate2, int S, int64_t y_rows,
+               unsigned* __restrict__ err) {
   constexpr int N = Vec<TY>::N;          // columns per 16-byte group
   pdl_launch_dependents();
   __shared__ int s_ptr[kMaxTokPerCta + 1];
@@ -126,6 +127,16 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
   for (int i = threadIdx.x; i <= t1 - t0; i += blockDim.x) s_ptr[i] = tok_ptr[t0 + i];
   __syncthreads();
   if (t0 >= t1) return;
+  if (kDebugChecks) {
+    // debug build: every span must run forwards and inside Y, else nothing is read
+    bool bad = false;
+    for (int i = threadIdx.x; i <= t1 - t0; i += blockDim.x)
+      bad |= s_ptr[i] < 0 || s_ptr[i] > y_rows || (i > 0 && s_ptr[i] < s_ptr[i - 1]);
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0) atomicOr(err, kErrDeviceCheck);
+      return;
+    }
+  }
   const int r0 = s_ptr[0], r1 = s_ptr[t1 - t0];
   const int ngroups = d / N;
   const int64_t stride = d / N;          // 16-byte groups per row
@@ -170,7 +181,7 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
 template <typename TY, typename TO>
 cudaError_t launch_typed(const void* Y, const int32_t* tok_ptr, const Shape& s, void* out,
                          const void* residual, bool res_bf16, const float* gate2,
-                         int sm_count, cudaStream_t st) {
+                         unsigned* err, int sm_count, cudaStream_t st) {
   constexpr int N = Vec<TY>::N;
   const int ngroups = s.d / N;
   int threads = ((ngroups + 31) / 32) * 32;
@@ -185,7 +196,7 @@ cudaError_t launch_typed(const void* Y, const int32_t* tok_ptr, const Shape& s, 
   }
   return launch_kernel(combine_kernel<TY, TO>, dim3(grid), dim3(threads), 0, st, s.pdl, 1,
                        (const TY*)Y, tok_ptr, s.T, s.d, per, (TO*)out, residual,
-                       (int)res_bf16, gate2, s.S);
+                       (int)res_bf16, gate2, s.S, s.y_rows, err);
 }
 
 }  // namespace
@@ -193,17 +204,19 @@ cudaError_t launch_typed(const void* Y, const int32_t* tok_ptr, const Shape& s, 
 cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const Shape& s, bool y_f32,
                            bool out_f32, void* out, const void* residual, bool res_bf16,
                            const float* gate2, unsigned* err, int sm_count, cudaStream_t st) {
-  (void)err;
   using bf = __nv_bfloat16;
   if (s.d % 8 != 0) return cudaErrorInvalidValue;
   if (y_f32 && out_f32)
-    return launch_typed<float, float>(Y, tok_ptr, s, out, residual, res_bf16, gate2, sm_count,
-                                      st);
+    return launch_typed<float, float>(Y, tok_ptr, s, out, residual, res_bf16, gate2, err,
+                                      sm_count, st);
   if (y_f32)
-    return launch_typed<float, bf>(Y, tok_ptr, s, out, residual, res_bf16, gate2, sm_count, st);
+    return launch_typed<float, bf>(Y, tok_ptr, s, out, residual, res_bf16, gate2, err, sm_count,
+                                   st);
   if (out_f32)
-    return launch_typed<bf, float>(Y, tok_ptr, s, out, residual, res_bf16, gate2, sm_count, st);
-  return launch_typed<bf, bf>(Y, tok_ptr, s, out, residual, res_bf16, gate2, sm_count, st);
+    return launch_typed<bf, float>(Y, tok_ptr, s, out, residual, res_bf16, gate2, err, sm_count,
+                                   st);
+  return launch_typed<bf, bf>(Y, tok_ptr, s, out, residual, res_bf16, gate2, err, sm_count,
+                                   st);
 }
 
 }  // namespace nmoe

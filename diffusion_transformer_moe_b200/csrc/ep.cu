@@ -1,6 +1,11 @@
 // Expert-parallel pieces: the row lists one rank owes another, row gather/scatter, and
 // the combine of a token range.
 //
+// Every list is padded to a capacity the host knows in advance (a rank's experts own
+// (e_end - e_begin) * Ce entries, so no list can be longer), with -1 rows that the copies
+// skip: the exchange moves fixed-size buffers, and no count has to come back to the host
+// before the next launch.
+//
 // With experts split into contiguous ranges, one per rank, every rank computes the same
 // routing and token lists, runs the expert GEMMs for its own range (each row landing at
 // its token-major position in Y), and the owner of a token range needs exactly the rows
@@ -16,15 +21,23 @@ namespace {
 constexpr int kRowsThreads = 1024;
 
 // One CTA: ordered compaction of the rows [tok_ptr[t_begin], tok_ptr[t_end]) whose entry
-// e*Ce + slot has e in [e_begin, e_end).
+// e*Ce + slot has e in [e_begin, e_end), into rows[0 .. count); rows[count .. capacity)
+// are set to -1 (padding the copies below skip). A list longer than `capacity` keeps its
+// first `capacity` rows and sets the error word; *count is the full length either way.
 __global__ void __launch_bounds__(kRowsThreads)
 ep_rows_kernel(const int32_t* __restrict__ tok_ptr, const int32_t* __restrict__ tok_ent,
                int E, int Ce, int t_begin, int t_end, int e_begin, int e_end,
-               int32_t* __restrict__ rows, int32_t* __restrict__ count) {
+               int32_t* __restrict__ rows, int capacity, int32_t* __restrict__ count,
+               unsigned* __restrict__ err) {
   __shared__ int s_warp[kRowsThreads / 32];
   __shared__ int s_base;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int r0 = tok_ptr[t_begin], r1 = tok_ptr[t_end];
+  int r0 = tok_ptr[t_begin], r1 = tok_ptr[t_end];
+  if (kDebugChecks && (r0 < 0 || r1 < r0 || r1 > E * Ce)) {
+    // debug build: a span outside the token lists is reported and nothing is listed
+    if (tid == 0) atomicOr(err, kErrDeviceCheck);
+    r0 = r1 = 0;
+  }
   if (tid == 0) s_base = 0;
   __syncthreads();
   for (int c0 = r0; c0 < r1; c0 += kRowsThreads) {
@@ -42,15 +55,22 @@ ep_rows_kernel(const int32_t* __restrict__ tok_ptr, const int32_t* __restrict__ 
       if (w < warp) before += s_warp[w];
       total += s_warp[w];
     }
-    if (keep) rows[before + __popc(b & ((1u << lane) - 1u))] = r;
+    const int at = before + __popc(b & ((1u << lane) - 1u));
+    if (keep && at < capacity) rows[at] = r;
     __syncthreads();
     if (tid == 0) s_base += total;
     __syncthreads();
   }
-  if (tid == 0) *count = s_base;
+  const int n = s_base;
+  for (int i = n + tid; i < capacity; i += kRowsThreads) rows[i] = -1;
+  if (tid == 0) {
+    *count = n;
+    if (n > capacity) atomicOr(err, kErrDeviceCheck);
+  }
 }
 
-// dst[i] = src[rows[i]] (GATHER) or dst[rows[i]] = src[i], rows of `chunks` 16-byte units
+// dst[i] = src[rows[i]] (GATHER; a zero row where rows[i] < 0) or dst[rows[i]] = src[i]
+// (nothing where rows[i] < 0), rows of `chunks` 16-byte units
 template <bool GATHER>
 __global__ void rows_copy_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ rows,
                                  int64_t n, int chunks, uint4* __restrict__ dst) {
@@ -60,8 +80,8 @@ __global__ void rows_copy_kernel(const uint4* __restrict__ src, const int32_t* _
     const int64_t i = k / chunks, c = k % chunks;
     const int64_t r = rows[i];
     if (GATHER)
-      dst[i * chunks + c] = src[r * chunks + c];
-    else
+      dst[i * chunks + c] = r >= 0 ? src[r * chunks + c] : make_uint4(0, 0, 0, 0);
+    else if (r >= 0)
       dst[r * chunks + c] = src[i * chunks + c];
   }
 }
@@ -70,9 +90,9 @@ __global__ void rows_copy_kernel(const uint4* __restrict__ src, const int32_t* _
 
 cudaError_t launch_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent, int E, int Ce,
                            int t_begin, int t_end, int e_begin, int e_end, int32_t* rows,
-                           int32_t* count, cudaStream_t st) {
+                           int capacity, int32_t* count, unsigned* err, cudaStream_t st) {
   ep_rows_kernel<<<1, kRowsThreads, 0, st>>>(tok_ptr, tok_ent, E, Ce, t_begin, t_end, e_begin,
-                                              e_end, rows, count);
+                                              e_end, rows, capacity, count, err);
   return cudaGetLastError();
 }
 

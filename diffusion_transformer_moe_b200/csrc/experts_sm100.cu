@@ -54,28 +54,42 @@ constexpr int kBBoxBytes = 64 * kBK * 2;        // 8 KB: 64 N x 64 K
 constexpr int kBBytes = 4 * kBBoxBytes;         // 32 KB: N = 256
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 2 * kAccCols;
-constexpr uint64_t kWaitNs = 2000000000ull;     // 2 s per wait
-constexpr uint64_t kDrainNs = 20000000ull;      // 20 ms per drain wait
+constexpr uint64_t kDrainNs = 20000000ull;      // 20 ms per drain wait after an abort
 
 enum { kGemm1 = 0, kGemm2 = 1 };
 enum { kGatherLsu = 0, kGatherTma4 = 1 };       // how gemm1 fetches its token rows
 
+// Operand rings. gemm1 keeps one ring whose stages hold an A tile (gathered token rows)
+// and a B tile (W1|W3) under one pair of barriers. gemm2 splits them: its A tiles (H hi
+// and lo) are re-read by every N block of an expert and mostly come from L2, while its
+// B tiles (W2) stream from HBM once, so the B ring is deeper than the A ring and each
+// has its own barriers and producer warp. With 4 B stages (instead of 3 shared ones)
+// more of the weight stream is in flight per SM for the same shared memory.
 template <int MODE, bool SPLIT, int GATHER>
 struct Cfg {
   static constexpr bool kLsuA = MODE == kGemm1 && GATHER == kGatherLsu;
+  static constexpr bool kSplitRing = MODE == kGemm2;
   static constexpr int kATiles = (MODE == kGemm2 && SPLIT) ? 2 : 1;
-  static constexpr int kStageBytes = kATiles * kABytes + kBBytes;
-  static constexpr int kStages = (MODE == kGemm2 && SPLIT) ? 3 : 4;
+  static constexpr int kAStageBytes = kATiles * kABytes;
+  static constexpr int kStageBytes = kAStageBytes + kBBytes;   // unified stage
+  static constexpr int kStages = 4;                            // unified ring depth
+  static constexpr int kStagesA = kSplitRing ? (SPLIT ? 2 : 3) : kStages;
+  static constexpr int kStagesB = kSplitRing ? (SPLIT ? 4 : 5) : kStages;
+  static constexpr size_t kRingBytes =
+      kSplitRing ? (size_t)kStagesA * kAStageBytes + (size_t)kStagesB * kBBytes
+                 : (size_t)kStages * kStageBytes;
   static constexpr int kAWarps = kLsuA ? 4 : 0;          // cp.async gather warps
+  static constexpr int kAProdWarps = kSplitRing ? 1 : 0; // TMA producer of the A ring
   static constexpr int kEpiWarps = 8;                    // two per TMEM lane quarter
-  static constexpr int kEpiWarp0 = 2 + kAWarps;
-  static constexpr int kThreads = 32 * (2 + kAWarps + kEpiWarps);
+  static constexpr int kEpiWarp0 = 2 + kAWarps + kAProdWarps;
+  static constexpr int kThreads = 32 * (2 + kAWarps + kAProdWarps + kEpiWarps);
   static constexpr int kFullCount = 1 + 32 * kAWarps;    // TMA arrive + one per gather thread
   // staging block per epilogue warp: gemm2 with fp32 Y, 32 rows x 32 fp32; gemm1, 32
   // rows x 32 bf16 of H (and as much again for H lo)
   static constexpr int kEpiStage =
       MODE == kGemm2 ? (SPLIT ? 32 * 32 * 4 : 0) : (SPLIT ? 2 * 32 * 64 : 32 * 64);
-  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + kEpiWarps * kEpiStage + 1024;
+  static constexpr size_t kSmem = kRingBytes + kEpiWarps * kEpiStage + 1024;
+  static_assert(kSmem <= 232448, "dynamic shared memory beyond the 227 KB a CTA may use");
 };
 
 struct Params {
@@ -96,7 +110,20 @@ struct Params {
   CsrArgs csr;
   int csr_blocks;
   unsigned* err;
+  uint64_t wait_ns;      // budget of each pipeline wait
+  int rows_x;            // gemm1: rows of x (debug checks of the gathered indices)
+  int64_t rows_y;        // gemm2: rows of Y (debug checks of ent_pos)
 };
+
+// Debug build: a gathered token index must lie in x; otherwise the error word is set and
+// row 0 is read instead (nothing outside x is touched).
+__device__ __forceinline__ int checked_row(int t, const Params& p) {
+  if (kDebugChecks && (t < 0 || t >= p.rows_x)) {
+    atomicOr(p.err, kErrDeviceCheck);
+    return 0;
+  }
+  return t;
+}
 
 // silu(g) = g * sigmoid(g) = g / (1 + e^-g) with the fast exp and the fast divide
 // (each within a few ulp of fp32, far below the hi/lo split's 16 bits). g is a finite
@@ -148,12 +175,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                     const __grid_constant__ CUtensorMap map_b1, const __nv_bfloat16* x,
                     const Params p) {
   using C = Cfg<MODE, SPLIT, GATHER>;
-  constexpr int kStages = C::kStages;
+  constexpr int kStages = C::kStagesB;   // the B ring (or the unified ring)
+  constexpr int kStagesA = C::kStagesA;
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // full/empty: the B ring (unified ring: both operands); fullA/emptyA: the A ring
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t fullA_bar[kStagesA], emptyA_bar[kStagesA];
   __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -161,14 +191,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = (p.K + kBK - 1) / kBK;
   constexpr int n_per_tile = MODE == kGemm1 ? 128 : 256;
-  // stage s: A tile(s) at s * kStageBytes, B boxes after them
-  auto a_tile = [&](int s, int which) { return smem + s * C::kStageBytes + which * kABytes; };
-  auto b_tile = [&](int s) { return smem + s * C::kStageBytes + C::kATiles * kABytes; };
+  // unified ring: stage s holds A tile(s) at s * kStageBytes and the B boxes after them;
+  // split rings: A stage s at s * kAStageBytes, B stage s after the whole A ring
+  auto a_tile = [&](int s, int which) {
+    return smem + s * (C::kSplitRing ? C::kAStageBytes : C::kStageBytes) + which * kABytes;
+  };
+  auto b_tile = [&](int s) {
+    return C::kSplitRing ? smem + kStagesA * C::kAStageBytes + s * kBBytes
+                         : smem + s * C::kStageBytes + C::kAStageBytes;
+  };
+  uint8_t* const epi_smem = smem + C::kRingBytes;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full_bar[i], C::kFullCount);
       mbar_init(&empty_bar[i], 1);
+    }
+    if (C::kSplitRing) {
+      for (int i = 0; i < kStagesA; ++i) {
+        mbar_init(&fullA_bar[i], 1);
+        mbar_init(&emptyA_bar[i], 1);
+      }
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
@@ -203,20 +246,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       if (MODE == kGemm1 && !C::kLsuA) {
         const int32_t* ir = p.idx + (int64_t)e * p.Ce;  // NULL idx: identity (shared)
         const int s = m0 + 4 * lane;
-        r0 = s + 0 < p.Ce ? (p.idx ? ir[s + 0] : s + 0) : 0;
-        r1 = s + 1 < p.Ce ? (p.idx ? ir[s + 1] : s + 1) : 0;
-        r2 = s + 2 < p.Ce ? (p.idx ? ir[s + 2] : s + 2) : 0;
-        r3 = s + 3 < p.Ce ? (p.idx ? ir[s + 3] : s + 3) : 0;
+        r0 = checked_row(s + 0 < p.Ce ? (p.idx ? ir[s + 0] : s + 0) : 0, p);
+        r1 = checked_row(s + 1 < p.Ce ? (p.idx ? ir[s + 1] : s + 1) : 0, p);
+        r2 = checked_row(s + 2 < p.Ce ? (p.idx ? ir[s + 2] : s + 2) : 0, p);
+        r3 = checked_row(s + 3 < p.Ce ? (p.idx ? ir[s + 3] : s + 3) : 0, p);
       }
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
         int w = 1;
-        if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, kWaitNs);
+        if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, p.wait_ns);
         ok = __shfl_sync(0xffffffffu, w, 0) != 0;
         if (!ok) break;
         if (lane == 0)
-          mbar_arrive_expect_tx(&full_bar[stage],
-                                C::kLsuA ? b_bytes : C::kATiles * kABytes + b_bytes);
+          mbar_arrive_expect_tx(&full_bar[stage], (C::kLsuA || C::kSplitRing)
+                                                      ? b_bytes
+                                                      : C::kAStageBytes + b_bytes);
         __syncwarp();
         const int k0 = kb * kBK;
         uint8_t* b_dst = b_tile(stage);
@@ -232,10 +276,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                         k0, e);
           }
         } else {
-          if (lane == 0)
-            tma_load_2d(a_tile(stage, 0), &map_a, &full_bar[stage], k0, e * p.Ce + m0);
-          if (C::kATiles == 2 && lane == 1)
-            tma_load_2d(a_tile(stage, 1), &map_a2, &full_bar[stage], k0, e * p.Ce + m0);
+          // gemm2: the weights only; the A ring has its own producer warp
           if (lane < nbox)
             tma_load_3d(b_dst + lane * kBBoxBytes, &map_b0, &full_bar[stage], n0 + 64 * lane,
                         k0, e);
@@ -252,6 +293,38 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       for (int s = 0; s < kStages; ++s)
         if (issued_mask & (1u << s))
           mbar_wait(&full_bar[s], (issued_par >> s) & 1u, &dummy, kDrainNs);
+    }
+    __syncwarp();
+  } else if (C::kSplitRing && warp == 2 + C::kAWarps) {
+    // ---------------- TMA producer of the A ring (gemm2: H hi, H lo) ----------------
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, issued_par = 0;
+    for (int item = blockIdx.x; item < p.num_items; item += gridDim.x) {
+      const Tile tl = tile_of(item, p, n_per_tile);
+      const int row0 = tl.e * p.Ce + tl.m0;
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&emptyA_bar[stage], phase ^ 1, abort_v, p.wait_ns);
+        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(&fullA_bar[stage], C::kAStageBytes);
+        __syncwarp();
+        if (lane == 0) tma_load_2d(a_tile(stage, 0), &map_a, &fullA_bar[stage], kb * kBK, row0);
+        if (C::kATiles == 2 && lane == 1)
+          tma_load_2d(a_tile(stage, 1), &map_a2, &fullA_bar[stage], kb * kBK, row0);
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStagesA) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    if (*abort_v && lane == 0) {
+      int dummy = 0;
+      for (int s2 = 0; s2 < kStagesA; ++s2)
+        if (issued_mask & (1u << s2))
+          mbar_wait(&fullA_bar[s2], (issued_par >> s2) & 1u, &dummy, kDrainNs);
     }
     __syncwarp();
   } else if (C::kLsuA && warp >= 2 && warp < 2 + C::kAWarps) {
@@ -275,13 +348,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       for (int i = 0; i < 8; ++i) {
         const int r = pw * 32 + i * 4 + sub;
         const int s = m0 + r;
-        const int t = s < p.Ce ? (p.idx ? p.idx[(int64_t)e * p.Ce + s] : s) : 0;
+        const int t = checked_row(s < p.Ce ? (p.idx ? p.idx[(int64_t)e * p.Ce + s] : s) : 0, p);
         src[i] = x + (int64_t)t * p.K + c * 8;
         dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
       }
       for (int kb = 0; kb < nk; ++kb) {
         int w = 1;
-        if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, kWaitNs);
+        if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, p.wait_ns);
         if (__shfl_sync(0xffffffffu, w, 0) == 0) { ok = false; break; }
         uint8_t* dst = a_tile(stage, 0);
         const int k0 = kb * kBK;
@@ -305,30 +378,39 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     if (lane == 0) {
       constexpr uint32_t idesc_full = idesc_bf16(kBM, 256, 1);
       constexpr uint32_t idesc_half = idesc_bf16(kBM, 128, 1);
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int stage = 0, acc = 0, stage_a = 0;
+      uint32_t phase = 0, acc_phase = 0, phase_a = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
         const uint32_t idesc = tile_of(item, p, n_per_tile).half ? idesc_half : idesc_full;
-        if (!(ok = mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_v, kWaitNs))) break;
+        if (!(ok = mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_v, p.wait_ns))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!(ok = mbar_wait(&full_bar[stage], phase, abort_v, kWaitNs))) break;
+          // split rings: the A stage first (it comes from L2), then the weights
+          if (C::kSplitRing &&
+              !(ok = mbar_wait(&fullA_bar[stage_a], phase_a, abort_v, p.wait_ns)))
+            break;
+          if (!(ok = mbar_wait(&full_bar[stage], phase, abort_v, p.wait_ns))) break;
           tc_fence_after();
           if (C::kLsuA) fence_proxy_async_smem();  // cp.async writes -> tensor-core reads
           const uint32_t b_addr = smem_u32(b_tile(stage));
+          const int sa = C::kSplitRing ? stage_a : stage;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, kBBoxBytes, 1024);
 #pragma unroll
             for (int h = 0; h < C::kATiles; ++h) {
-              const uint64_t ad = sdesc_sw128(smem_u32(a_tile(stage, h)) + kk * 32, 16, 1024);
+              const uint64_t ad = sdesc_sw128(smem_u32(a_tile(sa, h)) + kk * 32, 16, 1024);
               mma_bf16(d_tmem, ad, bd, idesc, (kb | kk | h) != 0);
             }
           }
           mma_commit(&empty_bar[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
+          if (C::kSplitRing) {
+            mma_commit(&emptyA_bar[stage_a]);
+            if (++stage_a == kStagesA) { stage_a = 0; phase_a ^= 1; }
+          }
         }
         if (!ok) break;
         mma_commit(&tfull_bar[acc]);
@@ -344,7 +426,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     // ---------------- epilogue: eight warps, two per TMEM lane quarter ----------------
     if (MODE == kGemm1 && p.csr_blocks > 0) {
       static_assert(C::kEpiWarps * 32 == kCsrThreads, "one CSR block per epilogue");
-      uint8_t* cs = smem + kStages * C::kStageBytes;
+      uint8_t* cs = epi_smem;
       const int et = threadIdx.x - 32 * C::kEpiWarp0;
       for (int blk = blockIdx.x; blk < p.csr_blocks; blk += gridDim.x)
         csr_block(blk, p.csr, cs, et, []() { asm volatile("bar.sync 1, 256;" ::: "memory"); });
@@ -364,18 +446,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       const int c_n = MODE == kGemm1 ? acc_n / 4 : acc_n / 2;
       const int c_lo = half * c_n;
       int w = 1;
-      if (lane == 0) w = mbar_wait(&tfull_bar[acc], acc_phase, abort_v, kWaitNs);
+      if (lane == 0) w = mbar_wait(&tfull_bar[acc], acc_phase, abort_v, p.wait_ns);
       if (__shfl_sync(0xffffffffu, w, 0) == 0) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * kAccCols;
       const int s = m0 + row;
-      const bool valid = s < p.Ce;
+      bool valid = s < p.Ce;
       const int64_t ent = (int64_t)e * p.Ce + (valid ? s : 0);
-      const int64_t orow = (MODE == kGemm2 ? (int64_t)p.ent_pos[ent] : ent) * p.N;
+      int64_t pos = MODE == kGemm2 ? (int64_t)p.ent_pos[ent] : ent;
+      if (kDebugChecks && MODE == kGemm2 && valid && (pos < 0 || pos >= p.rows_y)) {
+        // debug build: a row position outside Y is reported and its store skipped
+        atomicOr(p.err, kErrDeviceCheck);
+        valid = false;
+        pos = 0;
+      }
+      const int64_t orow = pos * p.N;
       if (MODE == kGemm1) {
         // staging blocks of this warp, 32 rows x 64 bytes each (H, then H lo): 16-byte
         // chunk c of row r at r * 64 + (c ^ ((r / 2) % 4)) * 16
-        uint8_t* sh = smem + kStages * C::kStageBytes + (warp - C::kEpiWarp0) * C::kEpiStage;
+        uint8_t* sh = epi_smem + (warp - C::kEpiWarp0) * C::kEpiStage;
         uint8_t* sl = sh + 32 * 64;
         const int sw = (lane >> 1) & 3;
 #pragma unroll 1
@@ -429,7 +518,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       } else {
         const float gw = valid ? (p.gate ? p.gate[(int64_t)e * p.Ce + s] : 1.f) : 0.f;
         // staging block of this warp: 16-byte chunk c of row r at r * 128 + (c ^ (r % 8)) * 16
-        float* sb = reinterpret_cast<float*>(smem + kStages * C::kStageBytes +
+        float* sb = reinterpret_cast<float*>(epi_smem +
                                              (warp - C::kEpiWarp0) * C::kEpiStage);
 #pragma unroll 1
         for (int j0 = c_lo; j0 < c_lo + c_n; j0 += 32) {
@@ -595,6 +684,9 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
     p.csr_blocks = (int)ceil_div(s.T, kCsrBlockTok);
   }
   p.err = err;
+  p.wait_ns = s.wait_ns;
+  p.rows_x = s.T;
+  p.rows_y = s.y_rows;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (tma_gather)
     return split ? launch<kGemm1, true, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl)
@@ -621,6 +713,9 @@ cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* 
   p.idx = nullptr; p.gate = gate; p.ent_pos = ent_pos; p.out = Y; p.out_lo = nullptr;
   p.csr_blocks = 0;
   p.err = err;
+  p.wait_ns = s.wait_ns;
+  p.rows_x = s.T;
+  p.rows_y = s.y_rows;
   return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl)
                : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl);
 }

@@ -15,6 +15,17 @@ namespace nmoe {
 constexpr unsigned kErrDeviceCheck = 1u;
 constexpr unsigned kErrTimeout = 2u;
 
+// The debug build (-DNMOE_DEBUG, libnmoe_debug.so) adds index and span checks to the
+// kernels: a gathered token index outside x, a down-projection row position outside Y,
+// a token-list span that runs backwards or outside Y. A failed check sets
+// kErrDeviceCheck and skips the access it guards (no trap); the release build compiles
+// the checks out.
+#ifdef NMOE_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
@@ -84,7 +95,13 @@ struct Shape {
   int S;         // tokens per segment = T / n_seg
   int Ce;        // entries per expert = n_seg * C
   bool pdl;      // launch with programmatic dependent launch
+  uint64_t wait_ns;  // budget of each bounded device-side wait (nmoe_options)
+  int64_t y_rows;    // rows of the layer's Y (all experts' entries, plus the shared rows)
 };
+
+// Budget of a device-side wait when the caller sets none: far beyond any wait of a
+// healthy call (the longest are a few microseconds).
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 
 // Launchers. Each returns the launch status (cudaGetLastError after the launch).
 cudaError_t launch_router_simt(const void* x, const void* W_r, const Shape& s, nmoe_dtype dt,
@@ -140,10 +157,11 @@ cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const Shape& s
                            const float* gate2, unsigned* err, int sm_count, cudaStream_t st);
 
 // Expert parallelism (ep.cu): rows[0 .. *count) = the token-major rows of tokens
-// [t_begin, t_end) whose expert is in [e_begin, e_end), ascending; row gather/scatter.
+// [t_begin, t_end) whose expert is in [e_begin, e_end), ascending, then -1 up to
+// `capacity`; row gather/scatter (rows < 0 are skipped).
 cudaError_t launch_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent, int E, int Ce,
                            int t_begin, int t_end, int e_begin, int e_end, int32_t* rows,
-                           int32_t* count, cudaStream_t st);
+                           int capacity, int32_t* count, unsigned* err, cudaStream_t st);
 cudaError_t launch_rows_copy(const void* src, const int32_t* rows, int64_t n, int64_t row_bytes,
                              void* dst, bool gather, int sm_count, cudaStream_t st);
 

@@ -45,8 +45,7 @@ constexpr int kBBoxBytes = 64 * kBK * 2;   // 8 KB: 64 experts x 64 k
 constexpr int kMaxE = 128;
 constexpr int kSplit = 2;   // CTAs per token tile (one cluster), each owning half of d
 constexpr int kChunkKB = 2; // k-blocks accumulated per TMEM chunk slice (128-long chunks)
-constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr uint64_t kDrainNs = 20000000ull;
+constexpr uint64_t kDrainNs = 20000000ull;  // 20 ms per drain wait after an abort
 
 struct Params {
   int T, d, E, S;
@@ -58,6 +57,7 @@ struct Params {
   float* scores;
   float* scores_t;
   unsigned* err;
+  uint64_t wait_ns;  // budget of each pipeline wait
 };
 
 // a + b = s + e exactly (Knuth's two-sum; no operation here may be contracted or
@@ -118,7 +118,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       int stage = 0;
       uint32_t phase = 0, issued_mask = 0, issued_par = 0;
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, kWaitNs)) break;
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, p.wait_ns)) break;
         mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
         const int k0 = (kb0 + kb) * kBK;
         tma_load_2d(sA + stage * kABytes, &map_x, &full_bar[stage], k0, t0);
@@ -145,8 +145,8 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       for (int kb = 0; kb < nk; ++kb) {
         const bool first = kb % kChunkKB == 0;
         const bool last = kb % kChunkKB == kChunkKB - 1 || kb == nk - 1;
-        if (first && !mbar_wait(&tempty_bar[buf], buf_phase ^ 1, abort_v, kWaitNs)) break;
-        if (!mbar_wait(&full_bar[stage], phase, abort_v, kWaitNs)) break;
+        if (first && !mbar_wait(&tempty_bar[buf], buf_phase ^ 1, abort_v, p.wait_ns)) break;
+        if (!mbar_wait(&full_bar[stage], phase, abort_v, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sA + stage * kABytes);
         const uint32_t b_addr = smem_u32(sB + stage * b_bytes);
@@ -189,8 +189,8 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       const bool two = ch + 1 < nch;
       int w = 1;
       if (lane == 0) {
-        w = mbar_wait(&tfull_bar[buf], buf_phase, abort_v, kWaitNs);
-        if (w && two) w = mbar_wait(&tfull_bar[buf + 1], buf_phase, abort_v, kWaitNs);
+        w = mbar_wait(&tfull_bar[buf], buf_phase, abort_v, p.wait_ns);
+        if (w && two) w = mbar_wait(&tfull_bar[buf + 1], buf_phase, abort_v, p.wait_ns);
       }
       if (__shfl_sync(0xffffffffu, w, 0) == 0) { ok = false; break; }
       tc_fence_after();
@@ -417,6 +417,7 @@ cudaError_t launch_router_sm100(const void* x, const void* W_r, const Shape& s,
   if (p.nbuf > 8) p.nbuf = 8;
   p.score_fn = (int)fn;
   p.bias = bias; p.scores = scores; p.scores_t = scores_t; p.err = err;
+  p.wait_ns = s.wait_ns;
   CUtensorMap mx, mw;
   if (!map_2d(&mx, x, (uint64_t)s.d, (uint64_t)s.T, 64, kBM) ||
       !map_2d(&mw, W_r, (uint64_t)s.E, (uint64_t)s.d, 64, 64))

@@ -57,8 +57,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Gives up after `budget_ns`
-// (or at once if *abort is set by another thread), records kErrTimeout-style failure
-// through the caller, and returns false.
+// (or at once if *abort is set by another thread), sets *abort so that the CTA's other
+// waits give up too, and returns false; the kernel then records kErrTimeout. The
+// elapsed time is taken as a signed difference, so a timer read that steps backwards
+// (another SM's clock domain, a coarse update) never looks like a wait of 2^64 ns.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag, uint64_t budget_ns) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -66,7 +68,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > budget_ns) {
+    if ((int64_t)(globaltimer_ns() - t0) > (int64_t)budget_ns) {
       *abort_flag = 1;
       return false;
     }

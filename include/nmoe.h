@@ -154,12 +154,20 @@ typedef struct nmoe_options {
    * from x (with router_bias carrying the timestep half, this is the page's gate
    * exactly). With host_io it is a HOST pointer, copied in like x. */
   const void* router_x;
+  /* Longest time, in nanoseconds, that any single device-side wait of the tensor-core
+   * kernels (a pipeline barrier between their copy, MMA and epilogue roles) may take
+   * before the kernel gives up: it then stops issuing work, lets its copies and MMAs in
+   * flight finish, frees its tensor memory, returns, and sets the error word that
+   * nmoe_get_last_error() reports as NMOE_ERR_TIMEOUT; the call's outputs are then
+   * undefined. 0 = the default of 2 s, far beyond any wait of a healthy call. A tiny
+   * value makes a wait give up on purpose (the failure path is tested that way). */
+  uint64_t wait_budget_ns;
 } nmoe_options;
 
 /* Fills `o` with the defaults: bf16, softmax, raw combine, route_scale 1, one segment,
  * no bias, internal workspace, no extra outputs, device I/O, no trace, SPLIT
  * intermediates, out in the input dtype, no shared expert or residual, all experts, the
- * router scoring x. */
+ * router scoring x, the default wait budget. */
 NMOE_API void nmoe_options_init(nmoe_options* o);
 
 /* Router (section 6.2 "gate = Linear(..., num_experts, bias=False)", then softmax over
@@ -215,17 +223,21 @@ NMOE_API nmoe_status nmoe_workspace_offsets(int64_t T, int64_t d, int64_t E, int
                                             size_t* tok_ent_offset);
 
 /* Expert parallelism: the token-major rows of tokens [t_begin, t_end) whose expert lies
- * in [e_begin, e_end), ascending, into rows (device int32, room for tok_ptr[t_end] -
- * tok_ptr[t_begin] entries), and their number into *count (device int32). tok_ptr and
- * tok_ent as left in the workspace (nmoe_workspace_offsets); Ce = n_segments * C. */
+ * in [e_begin, e_end), ascending, into rows[0 .. n) (device int32), and -1 into
+ * rows[n .. capacity), with n written to *count (device int32). The capacity is known
+ * on the host in advance: (e_end - e_begin) * Ce can never be exceeded, so buffers of
+ * that many rows let ranks exchange fixed-size buffers without reading any count back
+ * to the host. A list longer than `capacity` keeps its first `capacity` rows and sets
+ * the error word (NMOE_ERR_DEVICE_CHECK). tok_ptr and tok_ent as left in the workspace
+ * (nmoe_workspace_offsets); Ce = n_segments * C. */
 NMOE_API nmoe_status nmoe_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent, int64_t T,
                                   int64_t E, int64_t Ce, int64_t t_begin, int64_t t_end,
                                   int64_t e_begin, int64_t e_end, int32_t* rows,
-                                  int32_t* count, nmoe_stream_t stream);
+                                  int64_t capacity, int32_t* count, nmoe_stream_t stream);
 
-/* dst[i, :] = src[rows[i], :] (gather) / dst[rows[i], :] = src[i, :] (scatter) for
- * i < n: rows of row_bytes bytes (a positive multiple of 16), 16-byte aligned device
- * arrays; rows device int32. */
+/* dst[i, :] = src[rows[i], :] (gather; a zero row where rows[i] < 0) / dst[rows[i], :] =
+ * src[i, :] (scatter; nothing where rows[i] < 0) for i < n: rows of row_bytes bytes (a
+ * positive multiple of 16), 16-byte aligned device arrays; rows device int32. */
 NMOE_API nmoe_status nmoe_rows_gather(const void* src, const int32_t* rows, int64_t n,
                                       int64_t row_bytes, void* dst, nmoe_stream_t stream);
 NMOE_API nmoe_status nmoe_rows_scatter(const void* src, const int32_t* rows, int64_t n,

@@ -33,7 +33,9 @@ def test_library_exports_every_declared_symbol():
 
 def test_options_struct_matches_defaults():
     o = L.Options()
+    o.wait_budget_ns = 12345  # the last field: init must reach it at the same offset
     nm.lib().nmoe_options_init(C.byref(o))
+    assert o.wait_budget_ns == 0
     assert (o.dtype, o.score_fn, o.combine, o.n_segments, o.host_io) == (0, 0, 0, 1, 0)
     assert o.route_scale == 1.0 and not o.workspace and not o.trace
     assert not o.router_x and not o.residual and o.expert_end == 0
@@ -160,12 +162,30 @@ def test_expert_parallel_options_are_checked_on_host(kw, expect):
 
 def test_expert_parallel_calls_check_arguments_on_host():
     lib = nm.lib()
-    # t_end beyond T, an empty expert table, misaligned rows, rows not a multiple of 16 B
-    assert lib.nmoe_ep_rows(FAKE, FAKE, 64, 4, 8, 0, 65, 0, 2, FAKE, FAKE, None) == 1
-    assert lib.nmoe_ep_rows(FAKE, FAKE, 64, 0, 8, 0, 64, 0, 0, FAKE, FAKE, None) == 1
+    # t_end beyond T, an empty expert table, a negative capacity, a capacity without a
+    # row buffer, misaligned rows, rows not a multiple of 16 B
+    assert lib.nmoe_ep_rows(FAKE, FAKE, 64, 4, 8, 0, 65, 0, 2, FAKE, 16, FAKE, None) == 1
+    assert lib.nmoe_ep_rows(FAKE, FAKE, 64, 0, 8, 0, 64, 0, 0, FAKE, 16, FAKE, None) == 1
+    assert lib.nmoe_ep_rows(FAKE, FAKE, 64, 4, 8, 0, 64, 0, 2, FAKE, -1, FAKE, None) == 1
+    assert lib.nmoe_ep_rows(FAKE, FAKE, 64, 4, 8, 0, 64, 0, 2, None, 16, FAKE, None) == 1
     assert lib.nmoe_rows_gather(FAKE + 4, FAKE, 4, 64, FAKE, None) == 1
     assert lib.nmoe_rows_scatter(FAKE, FAKE, 4, 24, FAKE, None) == 1
     assert lib.nmoe_combine_tokens(FAKE, FAKE, 64, 12, 0, 64, 1, 0, FAKE, None) == 2
+
+
+def test_exchange_plan_is_static_and_symmetric():
+    # what rank a sends rank b is what b expects from a; nobody sends itself anything;
+    # every buffer holds the sender's whole entry count (an upper bound on any list)
+    from diffusion_transformer_moe_b200 import ep
+    for E, Ce, world in ((64, 128, 2), (6, 100, 4), (7, 5, 3), (8, 16, 1)):
+        plans = [ep.exchange_plan(E, Ce, world, r) for r in range(world)]
+        for a in range(world):
+            lo, hi = ep.split_range(E, world, a)
+            assert plans[a][0][a] == 0 and plans[a][1][a] == 0
+            for b in range(world):
+                assert plans[a][0][b] == plans[b][1][a]
+                if a != b:
+                    assert plans[a][0][b] == (hi - lo) * Ce
 
 
 def test_split_range_covers_every_item_once():
@@ -184,3 +204,11 @@ def test_missing_gpu_is_reported_not_crashed():
     # valid arguments on a machine without a device: NMOE_ERR_NO_DEVICE
     st = nm.lib().nmoe_forward(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 16, 4, 16, 8, FAKE + 64, None)
     assert st == 7
+
+
+def test_the_1024px_workload_fits_the_allocation_free_scratch():
+    # nmoe_forward_noalloc promises to run the 1024 px CFG layer in its fixed 128 MiB
+    # array: its scratch with default options must stay within that
+    from diffusion_transformer_moe_b200 import inputs as I
+    w = I.WORKLOADS["1024px_cfg"]
+    assert nm.workspace_size(w.T, w.d, w.E, w.F, w.C) <= (128 << 20)

@@ -11,8 +11,8 @@ at the layer's stated tolerances:
                    final rounding to bf16 (|y| reaches ~90 on the LogNormal workload,
                    where that half-ulp alone is 0.25)
   fp32 layers:     ||y - y_ref|| / ||y_ref|| <= 1e-4
-Small shapes run whole; the full workloads compare every score and selection, and the
-outputs of a seeded sample of tokens that the oracle computes one by one.
+Small shapes and the full workloads alike compare every score, every selection and every
+element of every output row with the oracle.
 """
 
 import numpy as np
@@ -244,7 +244,7 @@ def test_residual_may_be_x_and_a_zero_gate_returns_it():
     assert torch.equal(out, x)
 
 
-def test_shared_expert_full_1024px_rows_match_oracle():
+def test_shared_expert_full_1024px_matches_oracle():
     w = I.WORKLOADS["1024px_cfg"]
     a = I.make_inputs(w)
     g = torch.Generator().manual_seed(11)
@@ -260,13 +260,14 @@ def test_shared_expert_full_1024px_rows_match_oracle():
     torch.cuda.synchronize()
     assert nm.get_last_error() == 0
     sel = idx.cpu().numpy()
+    out = out.cpu()
+    del dev
     x = I.to_numpy_f64(a["x"])
-    toks = np.random.default_rng(2).choice(w.T, 96, replace=False)
-    r = O.layer_rows(x, I.to_numpy_f64(a["W_r"]), a["W1"].float().numpy(),
-                     a["W3"].float().numpy(), a["W2"].float().numpy(), w.C, toks,
-                     selection=sel, shared=tuple(I.to_numpy_f64(t) for t in sh),
-                     residual=x, gate2=gate2.double().numpy())
-    _check_out(out[torch.as_tensor(toks, device="cuda")], r["out"], "bf16")
+    r = O.layer(x, I.to_numpy_f64(a["W_r"]), a["W1"].float().numpy(),
+                a["W3"].float().numpy(), a["W2"].float().numpy(), w.C, selection=sel,
+                shared=tuple(I.to_numpy_f64(t) for t in sh), residual=x,
+                gate2=gate2.double().numpy())
+    _check_out(out, r["out"], "bf16")
 
 
 # -- invariants on the GPU path --------------------------------------------------------------
@@ -362,6 +363,27 @@ def test_first_large_row_select_in_a_fresh_process():
     assert r.returncode == 0, r.stderr[-2000:]
 
 
+def test_a_wait_that_runs_out_reports_timeout_and_the_next_call_is_clean():
+    """Failure detection without a fault: a wait budget of one nanosecond makes the
+    tensor-core kernels' first pipeline wait that is not already satisfied give up. The
+    kernels then stop issuing work, let their copies and MMAs in flight land, free their
+    tensor memory and return; the call reports NMOE_ERR_TIMEOUT through the error word.
+    The workspace starts zeroed, so the selection reads zero scores where the aborted
+    router wrote none (every index it derives stays in range). The next call with the
+    default budget must match the oracle and leave the word clean."""
+    T, d, E, F, C_ = 512, 256, 8, 256, 64
+    a = I.make_small(T, d, E, F, "bf16", seed=51)
+    dev = {k: v.cuda() for k, v in a.items()}
+    ws = torch.zeros(nm.workspace_size(T, d, E, F, C_), dtype=torch.uint8, device="cuda")
+    nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], C_, workspace=ws,
+               wait_budget_ns=1)
+    torch.cuda.synchronize()
+    assert nm.get_last_error() == 5  # NMOE_ERR_TIMEOUT
+    assert nm.get_last_error() == 0  # read and cleared
+    _full_parity(a, C_, "bf16")
+    assert nm.get_last_error() == 0
+
+
 def test_nan_scores_raise_the_device_check():
     scores_t = torch.rand(4, 256, device="cuda")
     scores_t[2, 17] = float("nan")
@@ -440,77 +462,91 @@ def test_caller_workspace_matches_internal():
 
 
 # -- the full workloads ------------------------------------------------------------------------
+#
+# Every element of every output row is compared with the oracle's whole layer (given the
+# GPU's selection, which is itself checked bit-exactly against the oracle's selection on
+# the GPU's scores). Unchosen tokens must be exact zeros.
 
-N_SAMPLE = 192
+FULL = ["512px_cfg", "1024px_cfg", "skewed_2048px", "model_default_1024px_cfg",
+        "batch4_1024px_cfg"]
 
 
-@pytest.mark.parametrize("name", ["512px_cfg", "1024px_cfg", "skewed_2048px",
-                                  "batch4_1024px_cfg", "model_default_1024px_cfg"])
-def test_full_workload_matches_oracle(name):
-    w = I.WORKLOADS[name]
-    nseg = w.segments
+def _full_run(w, **opts):
+    """The full workload on the GPU: bf16 and fp32 outputs, the scores and the chosen
+    tokens (host copies), with the device memory released before the oracle runs."""
     a = I.make_inputs(w)
+    nseg = w.segments
     dev = {k: v.cuda() for k, v in a.items()}
     ws = torch.empty(nm.workspace_size(w.T, w.d, w.E, w.F, w.C, out_f32=True,
-                                       n_segments=nseg),
+                                       n_segments=nseg, **opts),
                      dtype=torch.uint8, device="cuda")
     scores = torch.empty(w.T, w.E, device="cuda", dtype=torch.float32)
     idx = torch.empty(w.E, w.Ce, device="cuda", dtype=torch.int32)
     out = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C,
-                     workspace=ws, scores_out=scores, idx_out=idx, n_segments=nseg)
+                     workspace=ws, scores_out=scores, idx_out=idx, n_segments=nseg, **opts)
     out32 = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C,
-                       workspace=ws, out_f32=True, n_segments=nseg)
+                       workspace=ws, out_f32=True, n_segments=nseg, **opts)
     torch.cuda.synchronize()
     assert nm.get_last_error() == 0
     # the bf16 output is the fp32 result rounded once
     assert torch.equal(out, out32.to(torch.bfloat16))
+    res = (a, out.cpu(), out32.cpu(), scores.cpu(), idx.cpu().numpy())
     del dev, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def _oracle_full(w, a, sel):
     x = I.to_numpy_f64(a["x"])
-    W_r = I.to_numpy_f64(a["W_r"])
-    s_gpu = scores.cpu().numpy()
-    sel = O.select(s_gpu, w.C, nseg)
-    assert np.array_equal(sel, idx.cpu().numpy())
-    p = O.scores_from_logits(O.router_logits(x, W_r))
+    return O.layer(x, I.to_numpy_f64(a["W_r"]), a["W1"].float().numpy(),
+                   a["W3"].float().numpy(), a["W2"].float().numpy(), w.C, selection=sel,
+                   n_segments=w.segments)
+
+
+def _errors(y, y_ref):
+    y = _np(y)
+    d = np.abs(y - y_ref)
+    return np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref), d.max(), np.abs(y_ref).max()
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_workload_matches_oracle(name):
+    w = I.WORKLOADS[name]
+    a, out, out32, scores, idx = _full_run(w)
+    sel = O.select(scores.numpy(), w.C, w.segments)
+    assert np.array_equal(sel, idx)
+    x = I.to_numpy_f64(a["x"])
+    p = O.scores_from_logits(O.router_logits(x, I.to_numpy_f64(a["W_r"])))
     _check_scores(scores, p)
     # the oracle's own selection may differ only where scores are within tolerance
-    own = O.select(O.round_f32(p), w.C, nseg)
+    own = O.select(O.round_f32(p), w.C, w.segments)
     n_diff = sum(len(set(own[e]) ^ set(sel[e])) for e in range(w.E))
     assert n_diff <= 2 * w.E
-    rng = np.random.default_rng(0)
-    chosen = np.unique(sel.ravel())
-    # random tokens, random chosen tokens, and the chosen tokens of largest norm (the
-    # largest outputs)
-    norms = np.linalg.norm(x[chosen], axis=1)
-    toks = np.unique(np.concatenate([rng.choice(w.T, N_SAMPLE // 3, replace=False),
-                                     rng.choice(chosen, N_SAMPLE // 3, replace=False),
-                                     chosen[np.argsort(-norms)[:N_SAMPLE // 3]]]))
-    W1 = a["W1"].float().numpy(); W3 = a["W3"].float().numpy(); W2 = a["W2"].float().numpy()
-    r = O.layer_rows(x, W_r, W1, W3, W2, w.C, toks, selection=sel, n_segments=nseg)
-    tk = torch.as_tensor(toks, device="cuda")
-    _check_out(out[tk], r["out"], w.dtype)
-    _check_out(out32[tk], r["out"], "bf16f32" if w.dtype == "bf16" else "f32")
-    unchosen = np.setdiff1d(np.arange(w.T), chosen)
+    r = _oracle_full(w, a, sel)
+    # every element of every row, both output types
+    _check_out(out, r["out"], "bf16")
+    _check_out(out32, r["out"], "bf16")
+    unchosen = np.setdiff1d(np.arange(w.T), np.unique(sel.ravel()))
     if len(unchosen):
-        assert torch.all(out[torch.as_tensor(unchosen, device="cuda")] == 0)
+        assert torch.all(out[torch.as_tensor(unchosen)] == 0)
+    rel, mx, ymax = _errors(out32, r["out"])
+    print(f"{name}: all {w.T} rows, fp32 out rel {rel:.2e} max-abs {mx:.2e} "
+          f"(max |y| {ymax:.1f}); selection differences from the oracle's own scores {n_diff}")
 
 
-def test_bf16_intermediates_stay_within_relative_tolerance():
-    """The opt-in bf16 storage of H and Y (the usual bf16 numerics) still meets the
-    relative-norm tolerance on the LogNormal workload; its larger per-element drift is
-    the documented price of its smaller traffic."""
-    w = I.WORKLOADS["1024px_cfg"]
-    a = I.make_inputs(w)
-    dev = {k: v.cuda() for k, v in a.items()}
-    idx = torch.empty(w.E, w.C, device="cuda", dtype=torch.int32)
-    out = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C,
-                     idx_out=idx, intermediate="bf16", out_f32=True)
-    torch.cuda.synchronize()
-    sel = idx.cpu().numpy()
-    x = I.to_numpy_f64(a["x"])
-    toks = np.random.default_rng(1).choice(np.unique(sel.ravel()), 96, replace=False)
-    r = O.layer_rows(x, I.to_numpy_f64(a["W_r"]), a["W1"].float().numpy(),
-                     a["W3"].float().numpy(), a["W2"].float().numpy(), w.C, toks,
-                     selection=sel)
-    y = _np(out[torch.as_tensor(toks, device="cuda")])
-    rel = np.linalg.norm(y - r["out"]) / np.linalg.norm(r["out"])
+@pytest.mark.parametrize("name", ["1024px_cfg", "batch4_1024px_cfg"])
+def test_bf16_intermediates_full_workload(name):
+    """The opt-in bf16 storage of H and Y (the usual bf16 numerics), every row against
+    the oracle. The relative-norm tolerance holds on both workloads. On the LogNormal
+    workload the largest outputs (|y| ~ 90) drift beyond the 5e-2 absolute bar, which is
+    why split intermediates are the default; on the batch-4 workload (x ~ N(0, 1))
+    the absolute bar holds too."""
+    w = I.WORKLOADS[name]
+    a, out, out32, scores, idx = _full_run(w, intermediate="bf16")
+    r = _oracle_full(w, a, idx)
+    rel, mx, ymax = _errors(out32, r["out"])
+    print(f"{name} bf16 intermediates: all {w.T} rows, fp32 out rel {rel:.2e} "
+          f"max-abs {mx:.2e} (max |y| {ymax:.1f})")
     assert rel <= BF16_REL
+    if not w.lognormal_scale:
+        assert mx <= BF16_ABS

@@ -51,6 +51,21 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
         _close(out, ref)
 
 
+def test_noalloc_matches_forward_on_the_1024px_workload():
+    w = I.WORKLOADS["1024px_cfg"]
+    a = I.make_inputs(w)
+    dev = {k: v.cuda() for k, v in a.items()}
+    ref = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C)
+    for _ in range(2):  # the second call sees the first call's scratch
+        out = torch.full_like(dev["x"], float("nan"))
+        st = _noalloc(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], w.C, out)
+        assert st == 0, nm.lib().nmoe_status_str(st)
+        torch.cuda.synchronize()
+        assert nm.get_last_error() == 0
+        # the same kernels on the same inputs: the same bits
+        assert torch.equal(out, ref)
+
+
 def test_noalloc_rejects_sizes_beyond_its_capacity():
     # the batch-4 workload needs far more than 128 MiB of scratch: rejected, nothing runs
     w = I.WORKLOADS["batch4_1024px_cfg"]
