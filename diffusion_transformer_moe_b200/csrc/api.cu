@@ -304,11 +304,17 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   // On the tensor-core path the gate/up GEMM's epilogue warps build the token lists
   // while their first accumulators fill (no CSR launch); otherwise the CSR kernel does.
   const bool fuse_csr = tc && nmoe::gemm1_sm100_fuses_csr(s, split);
+  // A token that a single expert chose: its output is that expert's weighted row rounded
+  // once, so the tensor-core down projection writes it straight to out and the combine
+  // skips it (its row of Y is never written or read). Only for the plain layer output:
+  // no shared expert, no residual, all experts on this GPU, combined here.
+  const bool direct = tc && !has_shared && o.residual == nullptr && !o.skip_combine &&
+                      e_lo == 0 && e_hi == (int)E;
   const nmoe::CsrArgs csr = nmoe::csr_args(idx, bnd, s, has_shared, tok_ptr, tok_ent, ent_pos,
-                                           gate, o.combine, o.route_scale, ds->err);
+                                           gate, o.combine, o.route_scale, direct, ds->err);
   if (e == cudaSuccess && !fuse_csr)
     e = nmoe::launch_csr(idx, bnd, s, has_shared, tok_ptr, tok_ent, ent_pos, gate, o.combine,
-                         o.route_scale, ds->err, st);
+                         o.route_scale, direct, ds->err, st);
   mark(3);
   const bool tc_sh = has_shared && !f32 && nmoe::experts_sm100_supported(sh);
   if (has_shared && e == cudaSuccess)
@@ -327,18 +333,19 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
   mark(4);
   if (has_shared && e == cudaSuccess)
     e = tc_sh ? nmoe::launch_gemm2_sm100(Hs, Hs_lo, nullptr, tok_ptr, o.shared_w2, sh, split,
-                                         Y, ds->err, ds->sm_count, st)
+                                         Y, nullptr, false, ds->err, ds->sm_count, st)
               : nmoe::launch_gemm2_simt(Hs, nullptr, o.shared_w2, tok_ptr, sh, o.dtype, split,
                                         y_f32, Y, st);
   if (e == cudaSuccess && run_experts)
     e = tc ? nmoe::launch_gemm2_sm100(H, H_lo, gate + eoff, ent_pos + eoff, W2, sl, split, Y,
-                                      ds->err, ds->sm_count, st)
+                                      direct ? outd : nullptr, out_f32, ds->err, ds->sm_count,
+                                      st)
            : nmoe::launch_gemm2_simt(H, gate + eoff, W2, ent_pos + eoff, sl, o.dtype, split,
                                      y_f32, Y, st);
   mark(5);
   if (e == cudaSuccess && !o.skip_combine)
     e = nmoe::launch_combine(Y, tok_ptr, s, y_f32, out_f32, outd, o.residual, !f32, o.gate2,
-                             ds->err, ds->sm_count, st);
+                             direct, ds->err, ds->sm_count, st);
   mark(6);
   if (o.host_io && e == cudaSuccess)
     e = cudaMemcpyAsync(out, outd, obytes, cudaMemcpyDeviceToHost, st);
@@ -433,7 +440,7 @@ nmoe_status nmoe_select(const float* scores_t, int64_t T, int64_t E, int64_t C,
   cudaError_t e = nmoe::launch_select(scores_t, s, idx, gate, nullptr, ds->err, st);
   if (e == cudaSuccess && tok_ptr)
     e = nmoe::launch_csr(idx, nullptr, s, false, tok_ptr, tok_ent, nullptr, gate,
-                         NMOE_COMBINE_RAW, 1.f, ds->err, st);
+                         NMOE_COMBINE_RAW, 1.f, false, ds->err, st);
   if (e != cudaSuccess) { cudaGetLastError(); return NMOE_ERR_CUDA; }
   return NMOE_OK;
 }
@@ -537,7 +544,7 @@ nmoe_status nmoe_combine_tokens(const void* Y, const int32_t* tok_ptr, int64_t T
   s.pdl = false;
   s.y_rows = int64_t(1) << 40;  // Y's row count is not passed: only the order is checked
   if (nmoe::launch_combine(Y, tok_ptr + t_begin, s, y_dtype == NMOE_F32,
-                           out_dtype == NMOE_F32, out, nullptr, false, nullptr, ds->err,
+                           out_dtype == NMOE_F32, out, nullptr, false, nullptr, false, ds->err,
                            ds->sm_count, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return NMOE_ERR_CUDA;

@@ -14,18 +14,26 @@
 //   out[t, :] = residual[t, :] + tanh(clamp(gate2[t / S, :], -2, 2)) * sum,
 // in fp32 before the one rounding.
 //
-// Each CTA owns a contiguous token range, whose rows of Y form one contiguous span.
-// Every thread owns one 16-byte column group and walks the span row by row with eight
-// independent loads in flight, adding into the current token's sum and storing it when
-// the row index crosses the token's end: the memory access pattern of a plain copy, with
-// no synchronisation between warps.
+// Each CTA owns a contiguous token range and a slice of at most kMaxGroups 16-byte
+// column groups; every thread owns one column group. The CTA lists, in shared memory, the
+// rows of Y it has to read, in order (each token's rows are contiguous in Y); every thread
+// then walks the list with eight independent loads in flight, adding into the current
+// token's sum and storing it when the list crosses the token's end: the memory access
+// pattern of a plain copy, with no synchronisation between warps inside a round.
+//
+// When the down projection has already written the output row of every token that a
+// single expert chose (its sum is that one term, rounded once), those tokens' rows of Y
+// were never written: they are left out of the list, and such a token costs neither a
+// load nor a store here.
 #include "nmoe_internal.cuh"
 
 namespace nmoe {
 namespace {
 
 constexpr int kAhead = 8;                 // rows loaded per round
-constexpr int kMaxTokPerCta = 4096;
+constexpr int kMaxTokPerCta = 1024;       // tokens per CTA
+constexpr int kRowChunk = 2048;           // rows listed per pass over the list
+constexpr int kMaxGroups = 512;           // column groups (threads) per CTA
 
 template <typename T> struct Vec;        // 16 bytes of T, unpacked to fp32
 template <> struct Vec<float> {
@@ -113,15 +121,20 @@ struct Gated {
   }
 };
 
-template <typename TY, typename TO>
-__global__ void __launch_bounds__(512)
+// One CTA: tokens [t0, t1) (blockIdx.x), column groups of blockIdx.y. RES: the block's
+// gated residual is applied to each stored sum (its gate and residual registers make that
+// variant one CTA per SM; the plain sum fits two).
+template <typename TY, typename TO, bool RES>
+__global__ void __launch_bounds__(kMaxGroups, RES ? 1 : 2)
 combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, int Tn, int d,
                int tok_per_cta, TO* __restrict__ out, const void* __restrict__ residual,
                int res_bf16, const float* __restrict__ gate2, int S, int64_t y_rows,
-               unsigned* __restrict__ err) {
+               int skip_single, unsigned* __restrict__ err) {
   constexpr int N = Vec<TY>::N;          // columns per 16-byte group
   pdl_launch_dependents();
-  __shared__ int s_ptr[kMaxTokPerCta + 1];
+  __shared__ int s_ptr[kMaxTokPerCta + 1];   // Y row of each token's first entry
+  __shared__ int s_cpt[kMaxTokPerCta + 1];   // each token's first position in the list
+  __shared__ int s_rows[kRowChunk];          // the list, one chunk at a time
   const int t0 = min(Tn, (int)blockIdx.x * tok_per_cta), t1 = min(Tn, t0 + tok_per_cta);
   pdl_wait();
   for (int i = threadIdx.x; i <= t1 - t0; i += blockDim.x) s_ptr[i] = tok_ptr[t0 + i];
@@ -137,86 +150,127 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
       return;
     }
   }
-  const int r0 = s_ptr[0], r1 = s_ptr[t1 - t0];
-  const int ngroups = d / N;
+  // Positions in the list: token i keeps its s_ptr[i+1] - s_ptr[i] rows, or none when it
+  // has exactly one and the down projection wrote its output.
+  const int n = t1 - t0;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int run = 0;
+    for (int base = 0; base <= n; base += 32) {
+      const int i = base + lane;
+      int c = 0;
+      if (i < n) {
+        const int cnt = s_ptr[i + 1] - s_ptr[i];
+        c = (skip_single && cnt == 1) ? 0 : cnt;
+      }
+      int inc = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (i <= n) s_cpt[i] = run + inc - c;
+      run += __shfl_sync(0xffffffffu, inc, 31);
+    }
+  }
+  __syncthreads();
+  const int m = s_cpt[n];
+  const int grp = blockIdx.y * blockDim.x + threadIdx.x;
+  const bool active = grp < d / N;
+  const int col = grp * N;
   const int64_t stride = d / N;          // 16-byte groups per row
-  for (int grp = threadIdx.x; grp < ngroups; grp += blockDim.x) {
-    const int col = grp * N;
-    Gated<N> gt{residual, res_bf16 != 0, gate2, d, S, col};
-    const uint4* src = reinterpret_cast<const uint4*>(Y) + grp;
-    float acc[N];
+  const uint4* src = reinterpret_cast<const uint4*>(Y) + grp;
+  float acc[N];
 #pragma unroll
-    for (int i = 0; i < N; ++i) acc[i] = 0.f;
-    int t = t0;                           // token whose sum is being built
-    int tend = s_ptr[1];                  // its rows end here
-    for (int r = r0; r < r1; r += kAhead) {
-      uint4 v[kAhead];
+  for (int i = 0; i < N; ++i) acc[i] = 0.f;
+  [[maybe_unused]] Gated<N> gt{residual, res_bf16 != 0, gate2, d, S, col};
+  // the sum of token t is complete: store it, unless the down projection already did
+  auto finish = [&](int t) {
+    const int i = t - t0;
+    if (!(skip_single && s_ptr[i + 1] - s_ptr[i] == 1)) {
+      if (RES) gt.apply(t, acc);
+      store_out<N>(out + (int64_t)t * d + col, acc);
+    }
 #pragma unroll
-      for (int k = 0; k < kAhead; ++k)
-        v[k] = r + k < r1 ? __ldg(src + (int64_t)(r + k) * stride) : make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < N; ++k) acc[k] = 0.f;
+  };
+  int t = t0;                            // token whose sum is being built
+  int tend = s_cpt[1];                   // its rows end here in the list
+  for (int c0 = 0; c0 < m; c0 += kRowChunk) {
+    const int c1 = min(m, c0 + kRowChunk);
+    // the chunk's rows: token i's positions [s_cpt[i], s_cpt[i+1]) cut to [c0, c1)
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const int lo = max(s_cpt[i], c0), hi = min(s_cpt[i + 1], c1);
+      for (int j = lo; j < hi; ++j) s_rows[j - c0] = s_ptr[i] + (j - s_cpt[i]);
+    }
+    __syncthreads();
+    if (active) {
+      for (int j = c0; j < c1; j += kAhead) {
+        uint4 v[kAhead];
 #pragma unroll
-      for (int k = 0; k < kAhead; ++k) {
-        if (r + k < r1) {
-          while (r + k >= tend) {         // token t is complete (or had no rows)
-            gt.apply(t, acc);
-            store_out<N>(out + (int64_t)t * d + col, acc);
+        for (int k = 0; k < kAhead; ++k)
+          v[k] = j + k < c1 ? __ldg(src + (int64_t)s_rows[j + k - c0] * stride)
+                            : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int i = 0; i < N; ++i) acc[i] = 0.f;
-            ++t;
-            tend = s_ptr[t - t0 + 1];
+        for (int k = 0; k < kAhead; ++k) {
+          if (j + k < c1) {
+            while (j + k >= tend) {      // token t is complete (or had no rows to read)
+              finish(t);
+              ++t;
+              tend = s_cpt[t - t0 + 1];
+            }
+            Vec<TY>::add(acc, v[k]);
           }
-          Vec<TY>::add(acc, v[k]);
         }
       }
     }
-    for (; t < t1; ++t) {                  // the last token and any empty ones after it
-      gt.apply(t, acc);
-      store_out<N>(out + (int64_t)t * d + col, acc);
-#pragma unroll
-      for (int i = 0; i < N; ++i) acc[i] = 0.f;
-    }
+    __syncthreads();                     // the chunk's list is read before the next one
   }
+  if (active)
+    for (; t < t1; ++t) finish(t);       // the last token and any after it without rows
 }
 
 template <typename TY, typename TO>
 cudaError_t launch_typed(const void* Y, const int32_t* tok_ptr, const Shape& s, void* out,
                          const void* residual, bool res_bf16, const float* gate2,
-                         unsigned* err, int sm_count, cudaStream_t st) {
+                         bool skip_single, unsigned* err, int sm_count, cudaStream_t st) {
   constexpr int N = Vec<TY>::N;
   const int ngroups = s.d / N;
-  int threads = ((ngroups + 31) / 32) * 32;
-  if (threads > 512) threads = 512;
+  // column slices of at most kMaxGroups groups, as even as possible
+  const int slices = (int)ceil_div(ngroups, kMaxGroups);
+  int threads = (int)ceil_div(ceil_div(ngroups, slices), 32) * 32;
   // two CTAs per SM, each a contiguous token range
-  int grid = 2 * sm_count;
-  if (grid > s.T) grid = s.T;
-  int per = (int)ceil_div(s.T, grid);
-  if (per > kMaxTokPerCta) {
-    per = kMaxTokPerCta;
-    grid = (int)ceil_div(s.T, per);
-  }
-  return launch_kernel(combine_kernel<TY, TO>, dim3(grid), dim3(threads), 0, st, s.pdl, 1,
+  int ranges = (2 * sm_count + slices - 1) / slices;
+  if (ranges > s.T) ranges = s.T;
+  int per = (int)ceil_div(s.T, ranges);
+  if (per > kMaxTokPerCta) per = kMaxTokPerCta;
+  ranges = (int)ceil_div(s.T, per);
+  const dim3 grid((unsigned)ranges, (unsigned)slices);
+  if (residual != nullptr)
+    return launch_kernel(combine_kernel<TY, TO, true>, grid, dim3(threads), 0, st, s.pdl, 1,
+                         (const TY*)Y, tok_ptr, s.T, s.d, per, (TO*)out, residual,
+                         (int)res_bf16, gate2, s.S, s.y_rows, (int)skip_single, err);
+  return launch_kernel(combine_kernel<TY, TO, false>, grid, dim3(threads), 0, st, s.pdl, 1,
                        (const TY*)Y, tok_ptr, s.T, s.d, per, (TO*)out, residual,
-                       (int)res_bf16, gate2, s.S, s.y_rows, err);
+                       (int)res_bf16, gate2, s.S, s.y_rows, (int)skip_single, err);
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const Shape& s, bool y_f32,
                            bool out_f32, void* out, const void* residual, bool res_bf16,
-                           const float* gate2, unsigned* err, int sm_count, cudaStream_t st) {
+                           const float* gate2, bool skip_single, unsigned* err, int sm_count,
+                           cudaStream_t st) {
   using bf = __nv_bfloat16;
   if (s.d % 8 != 0) return cudaErrorInvalidValue;
-  if (y_f32 && out_f32)
-    return launch_typed<float, float>(Y, tok_ptr, s, out, residual, res_bf16, gate2, err,
-                                      sm_count, st);
-  if (y_f32)
-    return launch_typed<float, bf>(Y, tok_ptr, s, out, residual, res_bf16, gate2, err, sm_count,
-                                   st);
-  if (out_f32)
-    return launch_typed<bf, float>(Y, tok_ptr, s, out, residual, res_bf16, gate2, err, sm_count,
-                                   st);
-  return launch_typed<bf, bf>(Y, tok_ptr, s, out, residual, res_bf16, gate2, err, sm_count,
-                                   st);
+  auto go = [&](auto launch) {
+    return launch(Y, tok_ptr, s, out, residual, res_bf16, gate2, skip_single, err, sm_count,
+                  st);
+  };
+  if (y_f32 && out_f32) return go(launch_typed<float, float>);
+  if (y_f32) return go(launch_typed<float, bf>);
+  if (out_f32) return go(launch_typed<bf, float>);
+  return go(launch_typed<bf, bf>);
 }
 
 }  // namespace nmoe

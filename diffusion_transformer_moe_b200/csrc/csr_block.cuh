@@ -11,7 +11,9 @@
 // entry's token-major position (ent_pos), where the down projection writes its row.
 // With a shared expert every token's span starts with one more entry, its shared row.
 // NORMALIZED combine weights are rewritten in place from the fp32 sum of the token's
-// gates in ascending expert order.
+// gates in ascending expert order. With `direct`, the one entry of a token that a single
+// expert chose gets ent_pos = -(t + 1): the down projection writes that row straight to
+// the output (a sum of one term is that term, rounded once), and the combine skips it.
 #pragma once
 
 #include "nmoe_internal.cuh"
@@ -33,6 +35,7 @@ struct CsrArgs {
   float* gate;          // [E, Ce]
   int normalize;
   float route_scale;
+  int direct;           // single-entry tokens: ent_pos = -(t + 1), written by gemm2
   unsigned* err;
 };
 
@@ -172,7 +175,8 @@ __device__ __forceinline__ void csr_block(int blk, const CsrArgs& a, uint8_t* sm
       if (sl >= 0) {
         const int at = out + __popc(m & lt);
         a.tok_ent[at] = e * Ce + sl;
-        if (a.ent_pos != nullptr) a.ent_pos[e * Ce + sl] = at;
+        if (a.ent_pos != nullptr)
+          a.ent_pos[e * Ce + sl] = (a.direct && sh.cnt[r] == 1) ? -(t0 + r + 1) : at;
       }
       if (a.normalize) {
         const float v = sl >= 0 ? a.gate[(int64_t)e * Ce + sl] : 0.f;

@@ -57,32 +57,22 @@ constexpr int kTmemCols = 2 * kAccCols;
 constexpr uint64_t kDrainNs = 20000000ull;      // 20 ms per drain wait after an abort
 
 enum { kGemm1 = 0, kGemm2 = 1 };
-enum { kGatherLsu = 0, kGatherTma4 = 1 };       // how gemm1 fetches its token rows
+// How the A tiles are fetched: gemm1's token rows by 16-byte cp.async copies (LSU) or TMA
+// tile::gather4; gemm2's H rows by cp.async (LSU) or plain TMA tiles (kGatherTma4).
+enum { kGatherLsu = 0, kGatherTma4 = 1 };
 
-// Operand rings. gemm1 keeps one ring whose stages hold an A tile (gathered token rows)
-// and a B tile (W1|W3) under one pair of barriers. gemm2 splits them: its A tiles (H hi
-// and lo) are re-read by every N block of an expert and mostly come from L2, while its
-// B tiles (W2) stream from HBM once, so the B ring is deeper than the A ring and each
-// has its own barriers and producer warp. With 4 B stages (instead of 3 shared ones)
-// more of the weight stream is in flight per SM for the same shared memory.
 template <int MODE, bool SPLIT, int GATHER>
 struct Cfg {
-  static constexpr bool kLsuA = MODE == kGemm1 && GATHER == kGatherLsu;
-  static constexpr bool kSplitRing = MODE == kGemm2;
+  static constexpr bool kLsuA = GATHER == kGatherLsu;
   static constexpr int kATiles = (MODE == kGemm2 && SPLIT) ? 2 : 1;
   static constexpr int kAStageBytes = kATiles * kABytes;
-  static constexpr int kStageBytes = kAStageBytes + kBBytes;   // unified stage
-  static constexpr int kStages = 4;                            // unified ring depth
-  static constexpr int kStagesA = kSplitRing ? (SPLIT ? 2 : 3) : kStages;
-  static constexpr int kStagesB = kSplitRing ? (SPLIT ? 4 : 5) : kStages;
-  static constexpr size_t kRingBytes =
-      kSplitRing ? (size_t)kStagesA * kAStageBytes + (size_t)kStagesB * kBBytes
-                 : (size_t)kStages * kStageBytes;
+  static constexpr int kStageBytes = kAStageBytes + kBBytes;
+  static constexpr int kStages = (MODE == kGemm2 && SPLIT) ? 3 : 4;
+  static constexpr size_t kRingBytes = (size_t)kStages * kStageBytes;
   static constexpr int kAWarps = kLsuA ? 4 : 0;          // cp.async gather warps
-  static constexpr int kAProdWarps = kSplitRing ? 1 : 0; // TMA producer of the A ring
   static constexpr int kEpiWarps = 8;                    // two per TMEM lane quarter
-  static constexpr int kEpiWarp0 = 2 + kAWarps + kAProdWarps;
-  static constexpr int kThreads = 32 * (2 + kAWarps + kAProdWarps + kEpiWarps);
+  static constexpr int kEpiWarp0 = 2 + kAWarps;
+  static constexpr int kThreads = 32 * (2 + kAWarps + kEpiWarps);
   static constexpr int kFullCount = 1 + 32 * kAWarps;    // TMA arrive + one per gather thread
   // staging block per epilogue warp: gemm2 with fp32 Y, 32 rows x 32 fp32; gemm1, 32
   // rows x 32 bf16 of H (and as much again for H lo)
@@ -113,6 +103,11 @@ struct Params {
   uint64_t wait_ns;      // budget of each pipeline wait
   int rows_x;            // gemm1: rows of x (debug checks of the gathered indices)
   int64_t rows_y;        // gemm2: rows of Y (debug checks of ent_pos)
+  // gemm2: a row whose position is -(t + 1) is token t's only entry; it goes straight to
+  // row t of out_direct (the layer output, fp32 if out_direct_f32, else bf16), rounded
+  // once, instead of to Y
+  void* out_direct;
+  int out_direct_f32;
 };
 
 // Debug build: a gathered token index must lie in x; otherwise the error word is set and
@@ -173,17 +168,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                     const __grid_constant__ CUtensorMap map_a2,
                     const __grid_constant__ CUtensorMap map_b0,
                     const __grid_constant__ CUtensorMap map_b1, const __nv_bfloat16* x,
-                    const Params p) {
+                    const __nv_bfloat16* x2, const Params p) {
   using C = Cfg<MODE, SPLIT, GATHER>;
-  constexpr int kStages = C::kStagesB;   // the B ring (or the unified ring)
-  constexpr int kStagesA = C::kStagesA;
+  constexpr int kStages = C::kStages;
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // full/empty: the B ring (unified ring: both operands); fullA/emptyA: the A ring
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
-  __shared__ __align__(8) uint64_t fullA_bar[kStagesA], emptyA_bar[kStagesA];
   __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -191,27 +183,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = (p.K + kBK - 1) / kBK;
   constexpr int n_per_tile = MODE == kGemm1 ? 128 : 256;
-  // unified ring: stage s holds A tile(s) at s * kStageBytes and the B boxes after them;
-  // split rings: A stage s at s * kAStageBytes, B stage s after the whole A ring
-  auto a_tile = [&](int s, int which) {
-    return smem + s * (C::kSplitRing ? C::kAStageBytes : C::kStageBytes) + which * kABytes;
-  };
-  auto b_tile = [&](int s) {
-    return C::kSplitRing ? smem + kStagesA * C::kAStageBytes + s * kBBytes
-                         : smem + s * C::kStageBytes + C::kAStageBytes;
-  };
+  // stage s: A tile(s) at s * kStageBytes, B boxes after them
+  auto a_tile = [&](int s, int which) { return smem + s * C::kStageBytes + which * kABytes; };
+  auto b_tile = [&](int s) { return smem + s * C::kStageBytes + C::kAStageBytes; };
   uint8_t* const epi_smem = smem + C::kRingBytes;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full_bar[i], C::kFullCount);
       mbar_init(&empty_bar[i], 1);
-    }
-    if (C::kSplitRing) {
-      for (int i = 0; i < kStagesA; ++i) {
-        mbar_init(&fullA_bar[i], 1);
-        mbar_init(&emptyA_bar[i], 1);
-      }
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
@@ -221,7 +201,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     abort_flag = 0;
     fence_mbar_init();
     if (!C::kLsuA) prefetch_tensormap(&map_a);
-    if (C::kATiles == 2) prefetch_tensormap(&map_a2);
+    if (!C::kLsuA && C::kATiles == 2) prefetch_tensormap(&map_a2);
     prefetch_tensormap(&map_b0);
     if (MODE == kGemm1) prefetch_tensormap(&map_b1);
   }
@@ -258,9 +238,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         ok = __shfl_sync(0xffffffffu, w, 0) != 0;
         if (!ok) break;
         if (lane == 0)
-          mbar_arrive_expect_tx(&full_bar[stage], (C::kLsuA || C::kSplitRing)
-                                                      ? b_bytes
-                                                      : C::kAStageBytes + b_bytes);
+          mbar_arrive_expect_tx(&full_bar[stage],
+                                C::kLsuA ? b_bytes : C::kAStageBytes + b_bytes);
         __syncwarp();
         const int k0 = kb * kBK;
         uint8_t* b_dst = b_tile(stage);
@@ -276,7 +255,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                         k0, e);
           }
         } else {
-          // gemm2: the weights only; the A ring has its own producer warp
+          if (!C::kLsuA && lane == 0)
+            tma_load_2d(a_tile(stage, 0), &map_a, &full_bar[stage], k0, e * p.Ce + m0);
+          if (!C::kLsuA && C::kATiles == 2 && lane == 1)
+            tma_load_2d(a_tile(stage, 1), &map_a2, &full_bar[stage], k0, e * p.Ce + m0);
           if (lane < nbox)
             tma_load_3d(b_dst + lane * kBBoxBytes, &map_b0, &full_bar[stage], n0 + 64 * lane,
                         k0, e);
@@ -295,40 +277,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
           mbar_wait(&full_bar[s], (issued_par >> s) & 1u, &dummy, kDrainNs);
     }
     __syncwarp();
-  } else if (C::kSplitRing && warp == 2 + C::kAWarps) {
-    // ---------------- TMA producer of the A ring (gemm2: H hi, H lo) ----------------
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t issued_mask = 0, issued_par = 0;
-    for (int item = blockIdx.x; item < p.num_items; item += gridDim.x) {
-      const Tile tl = tile_of(item, p, n_per_tile);
-      const int row0 = tl.e * p.Ce + tl.m0;
-      bool ok = true;
-      for (int kb = 0; kb < nk; ++kb) {
-        int w = 1;
-        if (lane == 0) w = mbar_wait(&emptyA_bar[stage], phase ^ 1, abort_v, p.wait_ns);
-        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
-        if (!ok) break;
-        if (lane == 0) mbar_arrive_expect_tx(&fullA_bar[stage], C::kAStageBytes);
-        __syncwarp();
-        if (lane == 0) tma_load_2d(a_tile(stage, 0), &map_a, &fullA_bar[stage], kb * kBK, row0);
-        if (C::kATiles == 2 && lane == 1)
-          tma_load_2d(a_tile(stage, 1), &map_a2, &fullA_bar[stage], kb * kBK, row0);
-        issued_mask |= 1u << stage;
-        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == kStagesA) { stage = 0; phase ^= 1; }
-      }
-      if (!ok) break;
-    }
-    if (*abort_v && lane == 0) {
-      int dummy = 0;
-      for (int s2 = 0; s2 < kStagesA; ++s2)
-        if (issued_mask & (1u << s2))
-          mbar_wait(&fullA_bar[s2], (issued_par >> s2) & 1u, &dummy, kDrainNs);
-    }
-    __syncwarp();
   } else if (C::kLsuA && warp >= 2 && warp < 2 + C::kAWarps) {
-    // ---------------- cp.async gather of the token rows (gemm1) ----------------
+    // ---------------- cp.async loads of the A rows ----------------
+    // gemm1: the chosen token rows of x; gemm2: the expert's rows of H (hi, and lo with
+    // SPLIT). These copies go through the load/store units, beside the weight tiles that
+    // the TMA unit brings in, so the two paths fill shared memory together (a kernel
+    // whose every tile comes by TMA is held to the TMA unit's rate).
     // Warp pw owns tile rows [32 pw, 32 pw + 32); per instruction each group of eight
     // lanes copies one row's 128-byte k-slice (eight 16-byte pieces), and the piece c of
     // row r lands at r * 128 + ((c ^ (r % 8)) * 16): the 128-byte swizzle TMA would apply.
@@ -348,24 +302,40 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       for (int i = 0; i < 8; ++i) {
         const int r = pw * 32 + i * 4 + sub;
         const int s = m0 + r;
-        const int t = checked_row(s < p.Ce ? (p.idx ? p.idx[(int64_t)e * p.Ce + s] : s) : 0, p);
-        src[i] = x + (int64_t)t * p.K + c * 8;
+        // gemm1: the chosen token (idx NULL: row s); gemm2: the expert's row of H. Rows
+        // past the expert's Ce are read from a valid row and never stored.
+        int64_t t;
+        if (MODE == kGemm1)
+          t = checked_row(s < p.Ce ? (p.idx ? p.idx[(int64_t)e * p.Ce + s] : s) : 0, p);
+        else
+          t = (int64_t)e * p.Ce + (s < p.Ce ? s : 0);
+        src[i] = x + t * p.K + c * 8;
         dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
       }
+      // gemm2 with SPLIT: the lo rows sit at the same offsets of x2
+      const int64_t lo_off = (MODE == kGemm2 && C::kATiles == 2) ? (x2 - x) : 0;
       for (int kb = 0; kb < nk; ++kb) {
         int w = 1;
         if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, p.wait_ns);
         if (__shfl_sync(0xffffffffu, w, 0) == 0) { ok = false; break; }
         uint8_t* dst = a_tile(stage, 0);
+        uint8_t* dst2 = a_tile(stage, 1);
         const int k0 = kb * kBK;
         if (k0 + c * 8 < p.K) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) cp_async16(dst + dst_off[i], src[i] + k0);
-          cp_async_arrive_noinc(&full_bar[stage]);
-        } else {  // beyond d: zeros, as the TMA path's out-of-bounds fill
+          if (C::kATiles == 2) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 8; ++i) cp_async16(dst2 + dst_off[i], src[i] + lo_off + k0);
+          }
+          cp_async_arrive_noinc(&full_bar[stage]);
+        } else {  // beyond the row: zeros, as the TMA path's out-of-bounds fill
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
             *reinterpret_cast<uint4*>(dst + dst_off[i]) = make_uint4(0, 0, 0, 0);
+            if (C::kATiles == 2)
+              *reinterpret_cast<uint4*>(dst2 + dst_off[i]) = make_uint4(0, 0, 0, 0);
+          }
           fence_proxy_async_smem();
           mbar_arrive(&full_bar[stage]);
         }
@@ -378,8 +348,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     if (lane == 0) {
       constexpr uint32_t idesc_full = idesc_bf16(kBM, 256, 1);
       constexpr uint32_t idesc_half = idesc_bf16(kBM, 128, 1);
-      int stage = 0, acc = 0, stage_a = 0;
-      uint32_t phase = 0, acc_phase = 0, phase_a = 0;
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
         const uint32_t idesc = tile_of(item, p, n_per_tile).half ? idesc_half : idesc_full;
@@ -387,30 +357,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
         for (int kb = 0; kb < nk; ++kb) {
-          // split rings: the A stage first (it comes from L2), then the weights
-          if (C::kSplitRing &&
-              !(ok = mbar_wait(&fullA_bar[stage_a], phase_a, abort_v, p.wait_ns)))
-            break;
           if (!(ok = mbar_wait(&full_bar[stage], phase, abort_v, p.wait_ns))) break;
           tc_fence_after();
           if (C::kLsuA) fence_proxy_async_smem();  // cp.async writes -> tensor-core reads
           const uint32_t b_addr = smem_u32(b_tile(stage));
-          const int sa = C::kSplitRing ? stage_a : stage;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, kBBoxBytes, 1024);
 #pragma unroll
             for (int h = 0; h < C::kATiles; ++h) {
-              const uint64_t ad = sdesc_sw128(smem_u32(a_tile(sa, h)) + kk * 32, 16, 1024);
+              const uint64_t ad = sdesc_sw128(smem_u32(a_tile(stage, h)) + kk * 32, 16, 1024);
               mma_bf16(d_tmem, ad, bd, idesc, (kb | kk | h) != 0);
             }
           }
           mma_commit(&empty_bar[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
-          if (C::kSplitRing) {
-            mma_commit(&emptyA_bar[stage_a]);
-            if (++stage_a == kStagesA) { stage_a = 0; phase_a ^= 1; }
-          }
         }
         if (!ok) break;
         mma_commit(&tfull_bar[acc]);
@@ -454,13 +415,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       bool valid = s < p.Ce;
       const int64_t ent = (int64_t)e * p.Ce + (valid ? s : 0);
       int64_t pos = MODE == kGemm2 ? (int64_t)p.ent_pos[ent] : ent;
-      if (kDebugChecks && MODE == kGemm2 && valid && (pos < 0 || pos >= p.rows_y)) {
-        // debug build: a row position outside Y is reported and its store skipped
+      if (kDebugChecks && MODE == kGemm2 && valid &&
+          (pos >= p.rows_y ||
+           (pos < 0 && (p.out_direct == nullptr || -pos - 1 >= (int64_t)p.rows_x)))) {
+        // debug build: a row position outside Y (or the output) is reported and its
+        // store skipped
         atomicOr(p.err, kErrDeviceCheck);
         valid = false;
         pos = 0;
       }
-      const int64_t orow = pos * p.N;
+      const bool direct = MODE == kGemm2 && pos < 0;   // the token's only entry
+      const int64_t orow = (direct ? -pos - 1 : pos) * p.N;
       if (MODE == kGemm1) {
         // staging blocks of this warp, 32 rows x 64 bytes each (H, then H lo): 16-byte
         // chunk c of row r at r * 64 + (c ^ ((r / 2) % 4)) * 16
@@ -542,26 +507,63 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
               const int r = 4 * i + (lane >> 3);
               const int64_t ro = __shfl_sync(0xffffffffu, orow, r);
               const int rv = __shfl_sync(0xffffffffu, (int)valid, r);
-              const float4 v =
-                  *reinterpret_cast<const float4*>(sb + r * 32 + ((c ^ (r & 7)) << 2));
-              if (rv && col < p.N)
-                *reinterpret_cast<float4*>(static_cast<float*>(p.out) + ro + col) = v;
+              const int rd = __shfl_sync(0xffffffffu, (int)direct, r);
+              float4 v = *reinterpret_cast<const float4*>(sb + r * 32 + ((c ^ (r & 7)) << 2));
+              if (rv && col < p.N) {
+                if (!rd) {
+                  *reinterpret_cast<float4*>(static_cast<float*>(p.out) + ro + col) = v;
+                } else {
+                  // the combine's sum of one term: 0 + y (a -0 becomes +0), rounded once
+                  v = make_float4(v.x + 0.f, v.y + 0.f, v.z + 0.f, v.w + 0.f);
+                  if (p.out_direct_f32)
+                    *reinterpret_cast<float4*>(static_cast<float*>(p.out_direct) + ro + col) = v;
+                  else
+                    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out_direct) + ro +
+                                              col) =
+                        make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+                }
+              }
             }
             __syncwarp();  // the block is read before the next chunk overwrites it
           } else {
-            __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.out) + orow;
             uint32_t h[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               h[i] = pack_bf16x2(gw * __uint_as_float(y[2 * i]),
                                  gw * __uint_as_float(y[2 * i + 1]));
-            if (valid) {
+            if (valid && !direct) {
+              __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.out) + orow;
 #pragma unroll
               for (int v = 0; v < 4; ++v) {
                 const int c = n0 + j0 + 8 * v;
                 if (c < p.N)
                   *reinterpret_cast<uint4*>(yr + c) =
                       make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+              }
+            } else if (valid) {
+              // the combine's sum of one bf16 term: 0 + float(bf16(y)), rounded once
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const int c = n0 + j0 + 8 * v;
+                if (c >= p.N) continue;
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float2 t = __bfloat1622float2(
+                      *reinterpret_cast<const __nv_bfloat162*>(&h[4 * v + i]));
+                  f[2 * i] = t.x + 0.f;
+                  f[2 * i + 1] = t.y + 0.f;
+                }
+                if (p.out_direct_f32) {
+                  float* o = static_cast<float*>(p.out_direct) + orow + c;
+                  *reinterpret_cast<float4*>(o) = make_float4(f[0], f[1], f[2], f[3]);
+                  *reinterpret_cast<float4*>(o + 4) = make_float4(f[4], f[5], f[6], f[7]);
+                } else {
+                  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out_direct) + orow +
+                                            c) =
+                      make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                }
               }
             }
           }
@@ -639,12 +641,12 @@ void split_tail(Params& p, int sm_count) {
 
 template <int MODE, bool SPLIT, int GATHER>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b0,
-                   const CUtensorMap& b1, const __nv_bfloat16* x, const Params& p,
-                   int sm_count, cudaStream_t st, bool pdl) {
+                   const CUtensorMap& b1, const __nv_bfloat16* x, const __nv_bfloat16* x2,
+                   const Params& p, int sm_count, cudaStream_t st, bool pdl) {
   using C = Cfg<MODE, SPLIT, GATHER>;
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   return launch_kernel(grouped_gemm_kernel<MODE, SPLIT, GATHER>, dim3(grid), dim3(C::kThreads),
-                       C::kSmem, st, pdl, 1, a, a2, b0, b1, x, p);
+                       C::kSmem, st, pdl, 1, a, a2, b0, b1, x, x2, p);
 }
 
 }  // namespace
@@ -677,6 +679,7 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
   split_tail(p, sm_count);
   p.idx = idx; p.gate = nullptr; p.ent_pos = nullptr; p.out = H_hi; p.out_lo = H_lo;
+  p.out_direct = nullptr; p.out_direct_f32 = 0;
   p.csr_blocks = 0;
   if (csr != nullptr) {
     if (!gemm1_sm100_fuses_csr(s, split)) return cudaErrorInvalidValue;
@@ -689,15 +692,20 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
   p.rows_y = s.y_rows;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (tma_gather)
-    return split ? launch<kGemm1, true, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl)
-                 : launch<kGemm1, false, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl);
-  return split ? launch<kGemm1, true, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl)
-               : launch<kGemm1, false, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl);
+    return split ? launch<kGemm1, true, kGatherTma4>(ma, ma, mb0, mb1, xb, xb, p, sm_count, st,
+                                                     s.pdl)
+                 : launch<kGemm1, false, kGatherTma4>(ma, ma, mb0, mb1, xb, xb, p, sm_count, st,
+                                                      s.pdl);
+  return split ? launch<kGemm1, true, kGatherLsu>(ma, ma, mb0, mb1, xb, xb, p, sm_count, st,
+                                                  s.pdl)
+               : launch<kGemm1, false, kGatherLsu>(ma, ma, mb0, mb1, xb, xb, p, sm_count, st,
+                                                   s.pdl);
 }
 
 cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
                                const int32_t* ent_pos, const void* W2, const Shape& s, bool split,
-                               void* Y, unsigned* err, int sm_count, cudaStream_t st) {
+                               void* Y, void* out_direct, bool out_direct_f32, unsigned* err,
+                               int sm_count, cudaStream_t st) {
   CUtensorMap ma, ma2, mb;
   const int64_t rows = (int64_t)s.E * s.Ce;
   if (!rows_map(&ma, H_hi, rows, s.F, kBM) || !weight_map(&mb, W2, s.E, s.F, s.d))
@@ -711,13 +719,19 @@ cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* 
   p.num_tiles = s.E * p.tiles_m * p.tiles_n;
   split_tail(p, sm_count);
   p.idx = nullptr; p.gate = gate; p.ent_pos = ent_pos; p.out = Y; p.out_lo = nullptr;
+  p.out_direct = out_direct; p.out_direct_f32 = out_direct_f32 ? 1 : 0;
   p.csr_blocks = 0;
   p.err = err;
   p.wait_ns = s.wait_ns;
   p.rows_x = s.T;
   p.rows_y = s.y_rows;
-  return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl)
-               : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl);
+  // the H rows by cp.async, the W2 tiles by TMA
+  const __nv_bfloat16* hh = static_cast<const __nv_bfloat16*>(H_hi);
+  const __nv_bfloat16* hl = static_cast<const __nv_bfloat16*>(split ? H_lo : H_hi);
+  return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, hh, hl, p, sm_count, st,
+                                                  s.pdl)
+               : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, hh, hl, p, sm_count, st,
+                                                   s.pdl);
 }
 
 }  // namespace nmoe

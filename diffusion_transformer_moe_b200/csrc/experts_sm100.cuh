@@ -21,10 +21,12 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
                                void* H_hi, void* H_lo, const CsrArgs* csr, unsigned* err,
                                int sm_count, cudaStream_t st);
 
-// Row e*Ce + s of H W2_e, times gate[e, s], goes to Y row ent_pos[e*Ce + s].
+// Row e*Ce + s of H W2_e, times gate[e, s], goes to Y row ent_pos[e*Ce + s]; a
+// negative position -(t + 1) sends it instead to row t of out_direct (fp32 if
+// out_direct_f32, else bf16), rounded once (the token's only entry).
 cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
                                const int32_t* ent_pos, const void* W2, const Shape& s,
-                               bool split, void* Y, unsigned* err, int sm_count,
-                               cudaStream_t st);
+                               bool split, void* Y, void* out_direct, bool out_direct_f32,
+                               unsigned* err, int sm_count, cudaStream_t st);
 
 }  // namespace nmoe

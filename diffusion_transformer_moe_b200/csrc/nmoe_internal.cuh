@@ -122,18 +122,19 @@ cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, f
 // bnd: the table launch_select wrote, or NULL to search idx instead.
 // combine == NMOE_COMBINE_NORMALIZED rewrites gate[] in place to
 // route_scale * gate / (sum of the token's gates). ent_pos (may be NULL) receives, for
-// each entry e*Ce + slot, its index in the token-major order of tok_ent. With `shared`,
-// every token's span starts with one more entry, its shared-expert row (tok_ent value
-// E*Ce + t), so tok_ptr[T] = E*Ce + T.
+// each entry e*Ce + slot, its index in the token-major order of tok_ent, or with
+// `direct` -(t + 1) for the one entry of a token t that a single expert chose. With
+// `shared`, every token's span starts with one more entry, its shared-expert row
+// (tok_ent value E*Ce + t), so tok_ptr[T] = E*Ce + T.
 cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, bool shared,
                        int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
-                       nmoe_combine combine, float route_scale, unsigned* err,
+                       nmoe_combine combine, float route_scale, bool direct, unsigned* err,
                        cudaStream_t st);
 // The same arguments, for a kernel that builds the lists itself (csr_block.cuh).
 struct CsrArgs;
 CsrArgs csr_args(const int32_t* idx, const int32_t* bnd, const Shape& s, bool shared,
                  int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
-                 nmoe_combine combine, float route_scale, unsigned* err);
+                 nmoe_combine combine, float route_scale, bool direct, unsigned* err);
 
 // CUDA-core expert GEMMs. dt is the type of x and the weights; h_f32 / y_f32 select
 // fp32 (else dt) for the H and Y intermediates.
@@ -152,9 +153,12 @@ cudaError_t launch_gemm2_simt(const void* H, const float* gate, const void* W2,
 // Y is fp32 if y_f32 (else bf16), out fp32 if out_f32.
 // With residual (x's dtype: bf16 if res_bf16, else fp32), out[t] = residual[t] +
 // tanh(clamp(gate2[t / S], -2, 2)) * (that sum), gate2 NULL meaning a gate of 1.
+// skip_single: tokens with exactly one row were written by the down projection (their
+// rows of Y were never written): neither read nor stored here.
 cudaError_t launch_combine(const void* Y, const int32_t* tok_ptr, const Shape& s, bool y_f32,
                            bool out_f32, void* out, const void* residual, bool res_bf16,
-                           const float* gate2, unsigned* err, int sm_count, cudaStream_t st);
+                           const float* gate2, bool skip_single, unsigned* err, int sm_count,
+                           cudaStream_t st);
 
 // Expert parallelism (ep.cu): rows[0 .. *count) = the token-major rows of tokens
 // [t_begin, t_end) whose expert is in [e_begin, e_end), ascending, then -1 up to

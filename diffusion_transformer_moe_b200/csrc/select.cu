@@ -384,10 +384,10 @@ cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, f
 
 cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, bool shared,
                        int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
-                       nmoe_combine combine, float route_scale, unsigned* err,
+                       nmoe_combine combine, float route_scale, bool direct, unsigned* err,
                        cudaStream_t st) {
   const CsrArgs a = csr_args(idx, bnd, s, shared, tok_ptr, tok_ent, ent_pos, gate, combine,
-                             route_scale, err);
+                             route_scale, direct, err);
   dim3 grid((unsigned)ceil_div(s.T, kBlockTok));
   return launch_kernel(csr_kernel, grid, dim3(kCsrThreads), csr_smem_bytes(s.E), st, s.pdl, 1,
                        a);
@@ -395,12 +395,12 @@ cudaError_t launch_csr(const int32_t* idx, const int32_t* bnd, const Shape& s, b
 
 CsrArgs csr_args(const int32_t* idx, const int32_t* bnd, const Shape& s, bool shared,
                  int32_t* tok_ptr, int32_t* tok_ent, int32_t* ent_pos, float* gate,
-                 nmoe_combine combine, float route_scale, unsigned* err) {
+                 nmoe_combine combine, float route_scale, bool direct, unsigned* err) {
   CsrArgs a;
   a.idx = idx; a.bnd = bnd; a.T = s.T; a.E = s.E; a.Ce = s.Ce; a.shared = shared ? 1 : 0;
   a.tok_ptr = tok_ptr; a.tok_ent = tok_ent; a.ent_pos = ent_pos; a.gate = gate;
   a.normalize = combine == NMOE_COMBINE_NORMALIZED ? 1 : 0;
-  a.route_scale = route_scale; a.err = err;
+  a.route_scale = route_scale; a.direct = direct ? 1 : 0; a.err = err;
   return a;
 }
 

@@ -130,9 +130,15 @@ def prepare(x, W_r, W1, W3, W2, C_: int, E: int, world: int, rank: int, n_segmen
     L._check(L.lib().nmoe_forward_ex(x.data_ptr(), W_r.data_ptr(), W1.data_ptr(),
                                      W3.data_ptr(), W2.data_ptr(), T, d, E, F, C_, None,
                                      L._stream(stream), C.byref(o)), "nmoe_forward_ex")
-    # what I computed for each owner; what each other rank computed for my tokens
+    # what I computed for each other owner; what each other rank computed for my tokens
+    # (my own rows for my own tokens are already in my Y: nothing is listed for them)
     send, recv = [], []
+    zero = torch.zeros(1, dtype=torch.int32, device=x.device)
     for r in range(world):
+        if r == rank:
+            send.append((None, zero))
+            recv.append((None, zero))
+            continue
         send.append(st.rows(split_range(T, world, r), st.e_range, st.send_splits[r], stream))
         recv.append(st.rows(st.t_range, split_range(E, world, r), st.recv_splits[r], stream))
     send_splits, recv_splits = list(st.send_splits), list(st.recv_splits)

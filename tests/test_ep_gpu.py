@@ -88,6 +88,7 @@ def test_forward_over_a_one_rank_nccl_group():
         ref = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], 64)
         out = ep.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], 64, 4)
         torch.cuda.synchronize()
+        assert nm.get_last_error() == 0
         assert torch.equal(out, ref)
     finally:
         dist.destroy_process_group()
