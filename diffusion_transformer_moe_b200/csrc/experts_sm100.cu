@@ -57,13 +57,11 @@ constexpr int kTmemCols = 2 * kAccCols;
 constexpr uint64_t kDrainNs = 20000000ull;      // 20 ms per drain wait after an abort
 
 enum { kGemm1 = 0, kGemm2 = 1 };
-// How the A tiles are fetched: gemm1's token rows by 16-byte cp.async copies (LSU) or TMA
-// tile::gather4; gemm2's H rows by cp.async (LSU) or plain TMA tiles (kGatherTma4).
-enum { kGatherLsu = 0, kGatherTma4 = 1 };
+enum { kGatherLsu = 0, kGatherTma4 = 1 };       // how gemm1 fetches its token rows
 
 template <int MODE, bool SPLIT, int GATHER>
 struct Cfg {
-  static constexpr bool kLsuA = GATHER == kGatherLsu;
+  static constexpr bool kLsuA = MODE == kGemm1 && GATHER == kGatherLsu;
   static constexpr int kATiles = (MODE == kGemm2 && SPLIT) ? 2 : 1;
   static constexpr int kAStageBytes = kATiles * kABytes;
   static constexpr int kStageBytes = kAStageBytes + kBBytes;
@@ -168,7 +166,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                     const __grid_constant__ CUtensorMap map_a2,
                     const __grid_constant__ CUtensorMap map_b0,
                     const __grid_constant__ CUtensorMap map_b1, const __nv_bfloat16* x,
-                    const __nv_bfloat16* x2, const Params p) {
+                    const Params p) {
   using C = Cfg<MODE, SPLIT, GATHER>;
   constexpr int kStages = C::kStages;
   pdl_launch_dependents();
@@ -201,7 +199,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     abort_flag = 0;
     fence_mbar_init();
     if (!C::kLsuA) prefetch_tensormap(&map_a);
-    if (!C::kLsuA && C::kATiles == 2) prefetch_tensormap(&map_a2);
+    if (C::kATiles == 2) prefetch_tensormap(&map_a2);
     prefetch_tensormap(&map_b0);
     if (MODE == kGemm1) prefetch_tensormap(&map_b1);
   }
@@ -255,9 +253,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                         k0, e);
           }
         } else {
-          if (!C::kLsuA && lane == 0)
+          if (lane == 0)
             tma_load_2d(a_tile(stage, 0), &map_a, &full_bar[stage], k0, e * p.Ce + m0);
-          if (!C::kLsuA && C::kATiles == 2 && lane == 1)
+          if (C::kATiles == 2 && lane == 1)
             tma_load_2d(a_tile(stage, 1), &map_a2, &full_bar[stage], k0, e * p.Ce + m0);
           if (lane < nbox)
             tma_load_3d(b_dst + lane * kBBoxBytes, &map_b0, &full_bar[stage], n0 + 64 * lane,
@@ -278,11 +276,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
     }
     __syncwarp();
   } else if (C::kLsuA && warp >= 2 && warp < 2 + C::kAWarps) {
-    // ---------------- cp.async loads of the A rows ----------------
-    // gemm1: the chosen token rows of x; gemm2: the expert's rows of H (hi, and lo with
-    // SPLIT). These copies go through the load/store units, beside the weight tiles that
-    // the TMA unit brings in, so the two paths fill shared memory together (a kernel
-    // whose every tile comes by TMA is held to the TMA unit's rate).
+    // ---------------- cp.async gather of the token rows (gemm1) ----------------
     // Warp pw owns tile rows [32 pw, 32 pw + 32); per instruction each group of eight
     // lanes copies one row's 128-byte k-slice (eight 16-byte pieces), and the piece c of
     // row r lands at r * 128 + ((c ^ (r % 8)) * 16): the 128-byte swizzle TMA would apply.
@@ -302,40 +296,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
       for (int i = 0; i < 8; ++i) {
         const int r = pw * 32 + i * 4 + sub;
         const int s = m0 + r;
-        // gemm1: the chosen token (idx NULL: row s); gemm2: the expert's row of H. Rows
-        // past the expert's Ce are read from a valid row and never stored.
-        int64_t t;
-        if (MODE == kGemm1)
-          t = checked_row(s < p.Ce ? (p.idx ? p.idx[(int64_t)e * p.Ce + s] : s) : 0, p);
-        else
-          t = (int64_t)e * p.Ce + (s < p.Ce ? s : 0);
-        src[i] = x + t * p.K + c * 8;
+        const int t = checked_row(s < p.Ce ? (p.idx ? p.idx[(int64_t)e * p.Ce + s] : s) : 0, p);
+        src[i] = x + (int64_t)t * p.K + c * 8;
         dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
       }
-      // gemm2 with SPLIT: the lo rows sit at the same offsets of x2
-      const int64_t lo_off = (MODE == kGemm2 && C::kATiles == 2) ? (x2 - x) : 0;
       for (int kb = 0; kb < nk; ++kb) {
         int w = 1;
         if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, p.wait_ns);
         if (__shfl_sync(0xffffffffu, w, 0) == 0) { ok = false; break; }
         uint8_t* dst = a_tile(stage, 0);
-        uint8_t* dst2 = a_tile(stage, 1);
         const int k0 = kb * kBK;
         if (k0 + c * 8 < p.K) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) cp_async16(dst + dst_off[i], src[i] + k0);
-          if (C::kATiles == 2) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) cp_async16(dst2 + dst_off[i], src[i] + lo_off + k0);
-          }
           cp_async_arrive_noinc(&full_bar[stage]);
-        } else {  // beyond the row: zeros, as the TMA path's out-of-bounds fill
+        } else {  // beyond d: zeros, as the TMA path's out-of-bounds fill
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
+          for (int i = 0; i < 8; ++i)
             *reinterpret_cast<uint4*>(dst + dst_off[i]) = make_uint4(0, 0, 0, 0);
-            if (C::kATiles == 2)
-              *reinterpret_cast<uint4*>(dst2 + dst_off[i]) = make_uint4(0, 0, 0, 0);
-          }
           fence_proxy_async_smem();
           mbar_arrive(&full_bar[stage]);
         }
@@ -641,12 +619,12 @@ void split_tail(Params& p, int sm_count) {
 
 template <int MODE, bool SPLIT, int GATHER>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b0,
-                   const CUtensorMap& b1, const __nv_bfloat16* x, const __nv_bfloat16* x2,
-                   const Params& p, int sm_count, cudaStream_t st, bool pdl) {
+                   const CUtensorMap& b1, const __nv_bfloat16* x, const Params& p,
+                   int sm_count, cudaStream_t st, bool pdl) {
   using C = Cfg<MODE, SPLIT, GATHER>;
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   return launch_kernel(grouped_gemm_kernel<MODE, SPLIT, GATHER>, dim3(grid), dim3(C::kThreads),
-                       C::kSmem, st, pdl, 1, a, a2, b0, b1, x, x2, p);
+                       C::kSmem, st, pdl, 1, a, a2, b0, b1, x, p);
 }
 
 }  // namespace
@@ -692,14 +670,10 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
   p.rows_y = s.y_rows;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (tma_gather)
-    return split ? launch<kGemm1, true, kGatherTma4>(ma, ma, mb0, mb1, xb, xb, p, sm_count, st,
-                                                     s.pdl)
-                 : launch<kGemm1, false, kGatherTma4>(ma, ma, mb0, mb1, xb, xb, p, sm_count, st,
-                                                      s.pdl);
-  return split ? launch<kGemm1, true, kGatherLsu>(ma, ma, mb0, mb1, xb, xb, p, sm_count, st,
-                                                  s.pdl)
-               : launch<kGemm1, false, kGatherLsu>(ma, ma, mb0, mb1, xb, xb, p, sm_count, st,
-                                                   s.pdl);
+    return split ? launch<kGemm1, true, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl)
+                 : launch<kGemm1, false, kGatherTma4>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl);
+  return split ? launch<kGemm1, true, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl)
+               : launch<kGemm1, false, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl);
 }
 
 cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
@@ -725,13 +699,8 @@ cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* 
   p.wait_ns = s.wait_ns;
   p.rows_x = s.T;
   p.rows_y = s.y_rows;
-  // the H rows by cp.async, the W2 tiles by TMA
-  const __nv_bfloat16* hh = static_cast<const __nv_bfloat16*>(H_hi);
-  const __nv_bfloat16* hl = static_cast<const __nv_bfloat16*>(split ? H_lo : H_hi);
-  return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, hh, hl, p, sm_count, st,
-                                                  s.pdl)
-               : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, hh, hl, p, sm_count, st,
-                                                   s.pdl);
+  return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl)
+               : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl);
 }
 
 }  // namespace nmoe

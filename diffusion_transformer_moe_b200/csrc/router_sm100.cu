@@ -16,12 +16,10 @@
 // one fp32 division (relative error a few 1e-7).
 //
 // Each 128-token tile is split along d between the two CTAs of a cluster (so T = 8192
-// fills 128 SMs, not 64). In each CTA, four loader warps copy the x tiles into a 6-stage
-// ring with 16-byte cp.async copies while warp 0 brings the W_r tiles in by TMA (a kernel
-// whose every tile comes by TMA is held to the TMA unit's fill rate; the two paths fill
-// shared memory side by side); warp 1 (one thread) issues tcgen05.mma (M = 128, N = E
-// rounded up to 64, K = 16) into a ring of TMEM chunk buffers; 4*G epilogue warps
-// (G = ceil(E/CW)) each own 32 tokens x CW experts. Then each CTA sends its sums for the partner's half
+// fills 128 SMs, not 64). In each CTA, warp 0 streams x and W_r tiles with TMA into a
+// 6-stage ring; warp 1 (one thread) issues tcgen05.mma (M = 128, N = E rounded up to
+// 64, K = 16) into a ring of TMEM chunk buffers; 4*G epilogue warps (G = ceil(E/CW))
+// each own 32 tokens x CW experts. Then each CTA sends its sums for the partner's half
 // of the tokens to the partner's shared memory (distributed shared memory, no global
 // traffic), and all its epilogue warps finish the score function and both score layouts
 // for its 64 tokens. Every wait is bounded.
@@ -47,11 +45,9 @@ constexpr int kBBoxBytes = 64 * kBK * 2;   // 8 KB: 64 experts x 64 k
 constexpr int kMaxE = 128;
 constexpr int kSplit = 2;   // CTAs per token tile (one cluster), each owning half of d
 constexpr int kChunkKB = 2; // k-blocks accumulated per TMEM chunk slice (128-long chunks)
-
 constexpr uint64_t kDrainNs = 20000000ull;  // 20 ms per drain wait after an abort
 
 struct Params {
-  const __nv_bfloat16* x;  // [T, d], loaded by the cp.async warps
   int T, d, E, S;
   int epad;         // N of the MMA: E rounded up to 64
   int nbox;         // epad / 64
@@ -74,14 +70,11 @@ __device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
 
 // Each epilogue thread owns CW experts (16 up to E = 64, else 32) of one token row;
 // G = ceil(E / CW) column groups, so the epilogue has 4 G warps (one per TMEM lane
-// quarter and group). LW loader warps copy the x tiles with cp.async (4 up to E = 64);
-// with LW = 0 the TMA producer brings them in too (the wider epilogue of E > 64 leaves
-// no registers for loader warps).
-template <int G, int CW, int LW>
-__global__ void __launch_bounds__(32 * (2 + LW) + 128 * G, 1)
+// quarter and group).
+template <int G, int CW>
+__global__ void __launch_bounds__(64 + 128 * G, 1)
 router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
                     const __grid_constant__ CUtensorMap map_w, const Params p) {
-  constexpr int kEpiWarp0 = 2 + LW;             // first epilogue warp
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -104,11 +97,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
   const int t0 = (blockIdx.x / kSplit) * kBM;
 
   if (threadIdx.x == 0) {
-    // full: the W_r copy's arrival plus one per loader thread (its x copies landed)
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full_bar[i], 1 + 32 * LW);
-      mbar_init(&empty_bar[i], 1);
-    }
+    for (int i = 0; i < kStages; ++i) { mbar_init(&full_bar[i], 1); mbar_init(&empty_bar[i], 1); }
     for (int i = 0; i < p.nbuf; ++i) { mbar_init(&tfull_bar[i], 1); mbar_init(&tempty_bar[i], 4 * G); }
     mbar_init(&drain_bar, 1);
     abort_flag = 0;
@@ -116,7 +105,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
     prefetch_tensormap(&map_x);
     prefetch_tensormap(&map_w);
   }
-  if (warp == kEpiWarp0) tmem_alloc(&tmem_base_sh, 512);
+  if (warp == 2) tmem_alloc(&tmem_base_sh, 512);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
@@ -130,9 +119,9 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
       uint32_t phase = 0, issued_mask = 0, issued_par = 0;
       for (int kb = 0; kb < nk; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, p.wait_ns)) break;
-        mbar_arrive_expect_tx(&full_bar[stage], LW ? b_bytes : kABytes + b_bytes);
+        mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
         const int k0 = (kb0 + kb) * kBK;
-        if (!LW) tma_load_2d(sA + stage * kABytes, &map_x, &full_bar[stage], k0, t0);
+        tma_load_2d(sA + stage * kABytes, &map_x, &full_bar[stage], k0, t0);
         for (int j = 0; j < p.nbox; ++j)
           tma_load_2d(sB + stage * b_bytes + j * kBBoxBytes, &map_w, &full_bar[stage], 64 * j,
                       k0);
@@ -147,45 +136,6 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
             mbar_wait(&full_bar[s], (issued_par >> s) & 1u, &dummy, kDrainNs);
       }
     }
-  } else if (LW > 0 && warp >= 2 && warp < kEpiWarp0) {
-    // ---------------- cp.async loaders of the x tiles ----------------
-    // Warp lw owns tile rows [32 lw, 32 lw + 32); per instruction each group of eight
-    // lanes copies one row's 128-byte k-slice, piece c of row r landing at r * 128 +
-    // ((c ^ (r % 8)) * 16), the 128-byte swizzle TMA would apply. Rows past T read the
-    // last token (their scores are never stored); k past d is zero-filled.
-    const int lw = warp - 2;
-    const int sub = lane >> 3, c = lane & 7;
-    const __nv_bfloat16* src[8];
-    uint32_t dst_off[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = lw * 32 + i * 4 + sub;
-      const int t = min(t0 + r, p.T - 1);
-      src[i] = p.x + (int64_t)t * p.d + c * 8;
-      dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
-    }
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int kb = 0; kb < nk; ++kb) {
-      int w = 1;
-      if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, p.wait_ns);
-      if (__shfl_sync(0xffffffffu, w, 0) == 0) break;
-      uint8_t* dst = sA + stage * kABytes;
-      const int k0 = (kb0 + kb) * kBK;
-      if (k0 + c * 8 < p.d) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) cp_async16(dst + dst_off[i], src[i] + k0);
-        cp_async_arrive_noinc(&full_bar[stage]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          *reinterpret_cast<uint4*>(dst + dst_off[i]) = make_uint4(0, 0, 0, 0);
-        fence_proxy_async_smem();
-        mbar_arrive(&full_bar[stage]);
-      }
-      if (++stage == kStages) { stage = 0; phase ^= 1; }
-    }
-    cp_async_wait<0>();  // no copy may still be writing when the ring is reused
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -198,7 +148,6 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
         if (first && !mbar_wait(&tempty_bar[buf], buf_phase ^ 1, abort_v, p.wait_ns)) break;
         if (!mbar_wait(&full_bar[stage], phase, abort_v, p.wait_ns)) break;
         tc_fence_after();
-        if (LW) fence_proxy_async_smem();  // cp.async writes -> tensor-core reads
         const uint32_t a_addr = smem_u32(sA + stage * kABytes);
         const uint32_t b_addr = smem_u32(sB + stage * b_bytes);
         const uint32_t d0 = tmem_base + buf * p.epad;
@@ -223,7 +172,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
   } else {
     // ---------------- epilogue: 32 tokens x CW experts per warp ----------------
     const int q = warp & 3;
-    const int g = (warp - kEpiWarp0) >> 2;
+    const int g = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const int e0 = g * CW;
     // Kahan-compensated fp32 sums of the chunk sums: hi accumulates, lo keeps
@@ -303,7 +252,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
     // and the kEpc experts of group et / 64 (2G groups).
     constexpr int kEpc = CW / 2;
     const int nthr = 128 * G;
-    const int et = threadIdx.x - 32 * kEpiWarp0;
+    const int et = threadIdx.x - 64;
     const int tk = et & 63, grp = et >> 6;
     const int eb = grp * kEpc;
     const int t = t0 + rank * 64 + tk;
@@ -408,8 +357,8 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
         if (eb + j < p.E) p.scores_t[(int64_t)(eb + j) * p.T + t] = pr[j];
     }
   }
-  if (warp < kEpiWarp0) {
-    // the producer, loader and MMA warps take part in the two cluster barriers as well
+  if (warp < 2) {
+    // the producer and MMA warps take part in the two cluster barriers as well
     __syncwarp();
     cluster.sync();
     cluster.sync();
@@ -417,7 +366,7 @@ router_sm100_kernel(const __grid_constant__ CUtensorMap map_x,
 
   __syncthreads();
   if (threadIdx.x == 0 && abort_flag) atomicOr(p.err, kErrTimeout);
-  if (warp == kEpiWarp0) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
@@ -461,7 +410,6 @@ cudaError_t launch_router_sm100(const void* x, const void* W_r, const Shape& s,
                                 nmoe_score_fn fn, const float* bias, float* scores,
                                 float* scores_t, unsigned* err, cudaStream_t st) {
   Params p;
-  p.x = static_cast<const __nv_bfloat16*>(x);
   p.T = s.T; p.d = s.d; p.E = s.E; p.S = s.S;
   p.epad = (int)ceil_div(s.E, 64) * 64;
   p.nbox = p.epad / 64;
@@ -484,14 +432,12 @@ cudaError_t launch_router_sm100(const void* x, const void* W_r, const Shape& s,
   // 16 experts per thread up to E = 64 (up to 16 epilogue warps), 32 beyond
   const int CW = s.E <= 64 ? 16 : 32;
   const int G = (int)ceil_div(s.E, CW);
-  auto k = CW == 16 ? (G == 1 ? router_sm100_kernel<1, 16, 4>
-                     : G == 2 ? router_sm100_kernel<2, 16, 4>
-                     : G == 3 ? router_sm100_kernel<3, 16, 4>
-                              : router_sm100_kernel<4, 16, 4>)
-                    : (G == 3 ? router_sm100_kernel<3, 32, 0> : router_sm100_kernel<4, 32, 0>);
-  const int lw = CW == 16 ? 4 : 0;
-  return launch_kernel(k, dim3((unsigned)(ceil_div(s.T, kBM) * kSplit)),
-                       dim3(32 * (2 + lw) + 128 * G), smem,
+  auto k = CW == 16 ? (G == 1 ? router_sm100_kernel<1, 16>
+                     : G == 2 ? router_sm100_kernel<2, 16>
+                     : G == 3 ? router_sm100_kernel<3, 16>
+                              : router_sm100_kernel<4, 16>)
+                    : (G == 3 ? router_sm100_kernel<3, 32> : router_sm100_kernel<4, 32>);
+  return launch_kernel(k, dim3((unsigned)(ceil_div(s.T, kBM) * kSplit)), dim3(64 + 128 * G), smem,
                        st, s.pdl, kSplit, mx, mw, p);
 }
 

@@ -49,6 +49,13 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
+// Bit k of the low byte of b moved to bit 4k (the other bits cleared).
+__device__ __forceinline__ uint32_t spread4(uint32_t b) {
+  b = (b | (b << 12)) & 0x000F000Fu;
+  b = (b | (b << 6)) & 0x03030303u;
+  return (b | (b << 3)) & 0x11111111u;
+}
+
 __device__ __forceinline__ unsigned is_bad(uint32_t key) {
   return key >= 0x7f800000u;  // negative, +inf or NaN
 }
@@ -163,12 +170,14 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
 
   reinterpret_cast<uint4*>(s_hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
   if (tid == 0) s_ncand = 0;
+  __syncthreads();  // the histogram is zero before the row's first digit is counted
   pdl_wait();
 
   const uint32_t* row =
       reinterpret_cast<const uint32_t*>(scores_t + (int64_t)e * Tn + (int64_t)g * S);
   const uint32_t* keys = row;
-  // Non-negative finite scores only: sign bit clear and below +inf.
+  // Non-negative finite scores only: sign bit clear and below +inf. The first digit's
+  // histogram (bits 31..20) is counted as the row is read, with no pass of its own.
   unsigned bad = 0;
   if (cached) {
     int head = 0;
@@ -181,6 +190,10 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
         const uint4 v = r4[i];
         bad |= is_bad(v.x) | is_bad(v.y) | is_bad(v.z) | is_bad(v.w);
         k4[i] = v;
+        atomicAdd(&s_hist[v.x >> 20], 1u);
+        atomicAdd(&s_hist[v.y >> 20], 1u);
+        atomicAdd(&s_hist[v.z >> 20], 1u);
+        atomicAdd(&s_hist[v.w >> 20], 1u);
       }
       head = 4 * n4;
     }
@@ -189,11 +202,16 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
       const uint32_t v = row[i];
       bad |= is_bad(v);
       s_keys[i] = v;
+      atomicAdd(&s_hist[v >> 20], 1u);
     }
     keys = s_keys;
   } else {
 #pragma unroll 4
-    for (int i = tid; i < S; i += kSelThreads) bad |= is_bad(row[i]);
+    for (int i = tid; i < S; i += kSelThreads) {
+      const uint32_t v = row[i];
+      bad |= is_bad(v);
+      atomicAdd(&s_hist[v >> 20], 1u);
+    }
   }
   if (__syncthreads_or((int)bad) && tid == 0) atomicOr(err, kErrDeviceCheck);
 
@@ -208,8 +226,10 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
   for (int pass = 0; pass < 3 && !ranked; ++pass) {
     const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
     const uint32_t dmask = pass == 2 ? 0xffu : 0xfffu;
-    histogram(src, n, pmask, prefix, shift, dmask, s_hist);
-    __syncthreads();
+    if (pass > 0) {  // the first digit was counted while the row was read
+      histogram(src, n, pmask, prefix, shift, dmask, s_hist);
+      __syncthreads();
+    }
     find_digit(s_hist, (unsigned)k, s_wsum, s_res);
     __syncthreads();
     prefix |= s_res[0] << shift;
@@ -221,7 +241,56 @@ select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int 
       // Keys of the threshold's bin, with their positions (their order is irrelevant
       // to the histograms), and, 32 keys to a word, which keys lie in a higher bin:
       // those are above the threshold whatever it is (the equal words start empty).
-      for (int i0 = 0; i0 < S; i0 += kSelThreads) {
+      if (cached) {
+        // four keys per lane: a warp sweeps 128 consecutive keys (four words) per step
+        for (int c0 = 128 * warp; c0 < S; c0 += 128 * kSelWarps) {
+          const int i = c0 + 4 * lane;
+          const uint4 v = *reinterpret_cast<const uint4*>(keys + i);
+          const uint32_t kv[4] = {v.x, v.y, v.z, v.w};
+          unsigned a[4];
+          int nin = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const bool live = i + j < S;
+            a[j] = __ballot_sync(0xffffffffu, live && (kv[j] & pmask) > prefix);
+            nin += live && (kv[j] & pmask) == prefix;
+          }
+          if (lane < 4) {  // word lane: keys c0 + 32 lane .. + 31 = lanes 8 lane .. + 7
+            const int w = (c0 >> 5) + lane;
+            if (w < nw) {
+              uint32_t word = 0;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) word |= spread4((a[j] >> (8 * lane)) & 0xffu) << j;
+              s_gtw[w] = word;
+              s_eqw[w] = 0u;
+            }
+          }
+          // this lane's candidates go to consecutive slots after the warp's earlier lanes'
+          int before = nin;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, before, o);
+            if (lane >= o) before += t;
+          }
+          const int total = __shfl_sync(0xffffffffu, before, 31);
+          before -= nin;
+          if (total > 0) {
+            unsigned base = 0;
+            if (lane == 0) base = atomicAdd(&s_ncand, (unsigned)total);
+            unsigned at = __shfl_sync(0xffffffffu, base, 0) + (unsigned)before;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (i + j < S && (kv[j] & pmask) == prefix) {
+                if (at < (unsigned)kCandMax) {
+                  s_cand[at] = kv[j];
+                  s_cidx[at] = i + j;
+                }
+                ++at;
+              }
+            }
+          }
+        }
+      } else for (int i0 = 0; i0 < S; i0 += kSelThreads) {
         const int i = i0 + tid;
         const uint32_t key = i < S ? keys[i] : 0u;
         const bool in = i < S && (key & pmask) == prefix;
