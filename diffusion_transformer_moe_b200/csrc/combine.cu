@@ -14,25 +14,23 @@
 //   out[t, :] = residual[t, :] + tanh(clamp(gate2[t / S, :], -2, 2)) * sum,
 // in fp32 before the one rounding.
 //
-// Each CTA owns a contiguous token range and a slice of at most kMaxGroups 16-byte
-// column groups; every thread owns one column group. The CTA lists, in shared memory, the
-// rows of Y it has to read, in order (each token's rows are contiguous in Y); every thread
-// then walks the list with eight independent loads in flight, adding into the current
-// token's sum and storing it when the list crosses the token's end: the memory access
-// pattern of a plain copy, with no synchronisation between warps inside a round.
+// Each CTA owns a contiguous token range, whose rows of Y form one contiguous span, and a
+// slice of at most kMaxGroups 16-byte column groups; every thread owns one column group and
+// walks the span row by row with eight independent loads in flight, adding into the
+// current token's sum and storing it when the row index crosses the token's end: the
+// memory access pattern of a plain copy, with no synchronisation between warps.
 //
 // When the down projection has already written the output row of every token that a
-// single expert chose (its sum is that one term, rounded once), those tokens' rows of Y
-// were never written: they are left out of the list, and such a token costs neither a
-// load nor a store here.
+// single expert chose (its sum is that one term, rounded once), such a token's row of Y
+// was never written: the walk still passes over it (keeping the loads a plain stream) but
+// the token's sum is not stored, so it costs no output write here.
 #include "nmoe_internal.cuh"
 
 namespace nmoe {
 namespace {
 
 constexpr int kAhead = 8;                 // rows loaded per round
-constexpr int kMaxTokPerCta = 1024;       // tokens per CTA
-constexpr int kRowChunk = 2048;           // rows listed per pass over the list
+constexpr int kMaxTokPerCta = 4096;
 constexpr int kMaxGroups = 512;           // column groups (threads) per CTA
 
 template <typename T> struct Vec;        // 16 bytes of T, unpacked to fp32
@@ -132,9 +130,7 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
                int skip_single, unsigned* __restrict__ err) {
   constexpr int N = Vec<TY>::N;          // columns per 16-byte group
   pdl_launch_dependents();
-  __shared__ int s_ptr[kMaxTokPerCta + 1];   // Y row of each token's first entry
-  __shared__ int s_cpt[kMaxTokPerCta + 1];   // each token's first position in the list
-  __shared__ int s_rows[kRowChunk];          // the list, one chunk at a time
+  __shared__ int s_ptr[kMaxTokPerCta + 1];
   const int t0 = min(Tn, (int)blockIdx.x * tok_per_cta), t1 = min(Tn, t0 + tok_per_cta);
   pdl_wait();
   for (int i = threadIdx.x; i <= t1 - t0; i += blockDim.x) s_ptr[i] = tok_ptr[t0 + i];
@@ -150,41 +146,17 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
       return;
     }
   }
-  // Positions in the list: token i keeps its s_ptr[i+1] - s_ptr[i] rows, or none when it
-  // has exactly one and the down projection wrote its output.
-  const int n = t1 - t0;
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    int run = 0;
-    for (int base = 0; base <= n; base += 32) {
-      const int i = base + lane;
-      int c = 0;
-      if (i < n) {
-        const int cnt = s_ptr[i + 1] - s_ptr[i];
-        c = (skip_single && cnt == 1) ? 0 : cnt;
-      }
-      int inc = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += v;
-      }
-      if (i <= n) s_cpt[i] = run + inc - c;
-      run += __shfl_sync(0xffffffffu, inc, 31);
-    }
-  }
-  __syncthreads();
-  const int m = s_cpt[n];
   const int grp = blockIdx.y * blockDim.x + threadIdx.x;
-  const bool active = grp < d / N;
+  if (grp >= d / N) return;
+  const int r0 = s_ptr[0], r1 = s_ptr[t1 - t0];
   const int col = grp * N;
   const int64_t stride = d / N;          // 16-byte groups per row
+  [[maybe_unused]] Gated<N> gt{residual, res_bf16 != 0, gate2, d, S, col};
   const uint4* src = reinterpret_cast<const uint4*>(Y) + grp;
   float acc[N];
 #pragma unroll
   for (int i = 0; i < N; ++i) acc[i] = 0.f;
-  [[maybe_unused]] Gated<N> gt{residual, res_bf16 != 0, gate2, d, S, col};
-  // the sum of token t is complete: store it, unless the down projection already did
+  // token t's sum is complete: store it (unless the down projection already did)
   auto finish = [&](int t) {
     const int i = t - t0;
     if (!(skip_single && s_ptr[i + 1] - s_ptr[i] == 1)) {
@@ -195,39 +167,25 @@ combine_kernel(const TY* __restrict__ Y, const int32_t* __restrict__ tok_ptr, in
     for (int k = 0; k < N; ++k) acc[k] = 0.f;
   };
   int t = t0;                            // token whose sum is being built
-  int tend = s_cpt[1];                   // its rows end here in the list
-  for (int c0 = 0; c0 < m; c0 += kRowChunk) {
-    const int c1 = min(m, c0 + kRowChunk);
-    // the chunk's rows: token i's positions [s_cpt[i], s_cpt[i+1]) cut to [c0, c1)
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const int lo = max(s_cpt[i], c0), hi = min(s_cpt[i + 1], c1);
-      for (int j = lo; j < hi; ++j) s_rows[j - c0] = s_ptr[i] + (j - s_cpt[i]);
-    }
-    __syncthreads();
-    if (active) {
-      for (int j = c0; j < c1; j += kAhead) {
-        uint4 v[kAhead];
+  int tend = s_ptr[1];                   // its rows end here
+  for (int r = r0; r < r1; r += kAhead) {
+    uint4 v[kAhead];
 #pragma unroll
-        for (int k = 0; k < kAhead; ++k)
-          v[k] = j + k < c1 ? __ldg(src + (int64_t)s_rows[j + k - c0] * stride)
-                            : make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < kAhead; ++k)
+      v[k] = r + k < r1 ? __ldg(src + (int64_t)(r + k) * stride) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int k = 0; k < kAhead; ++k) {
-          if (j + k < c1) {
-            while (j + k >= tend) {      // token t is complete (or had no rows to read)
-              finish(t);
-              ++t;
-              tend = s_cpt[t - t0 + 1];
-            }
-            Vec<TY>::add(acc, v[k]);
-          }
+    for (int k = 0; k < kAhead; ++k) {
+      if (r + k < r1) {
+        while (r + k >= tend) {          // token t is complete (or had no rows)
+          finish(t);
+          ++t;
+          tend = s_ptr[t - t0 + 1];
         }
+        Vec<TY>::add(acc, v[k]);
       }
     }
-    __syncthreads();                     // the chunk's list is read before the next one
   }
-  if (active)
-    for (; t < t1; ++t) finish(t);       // the last token and any after it without rows
+  for (; t < t1; ++t) finish(t);         // the last token and any empty ones after it
 }
 
 template <typename TY, typename TO>

@@ -212,6 +212,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
+    // Every weight tile is read exactly once per call: its copies are marked evict-first,
+    // so that the weight stream (hundreds of MB) does not push out of L2 the token rows,
+    // H and Y that this kernel and the next one read again.
+    const uint64_t wpol = l2_policy_evict_first();
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // per stage: ever issued / parity of last issue
@@ -249,8 +253,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
           if (lane < nbox) {
             const int per = nbox / 2;
             const CUtensorMap* mb = lane < per ? &map_b0 : &map_b1;
-            tma_load_3d(b_dst + lane * kBBoxBytes, mb, &full_bar[stage], n0 + 64 * (lane % per),
-                        k0, e);
+            tma_load_3d_hint(b_dst + lane * kBBoxBytes, mb, &full_bar[stage],
+                             n0 + 64 * (lane % per), k0, e, wpol);
           }
         } else {
           if (lane == 0)
@@ -258,8 +262,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
           if (C::kATiles == 2 && lane == 1)
             tma_load_2d(a_tile(stage, 1), &map_a2, &full_bar[stage], k0, e * p.Ce + m0);
           if (lane < nbox)
-            tma_load_3d(b_dst + lane * kBBoxBytes, &map_b0, &full_bar[stage], n0 + 64 * lane,
-                        k0, e);
+            tma_load_3d_hint(b_dst + lane * kBBoxBytes, &map_b0, &full_bar[stage],
+                             n0 + 64 * lane, k0, e, wpol);
         }
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);

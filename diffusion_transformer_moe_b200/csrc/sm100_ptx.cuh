@@ -99,6 +99,25 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// L2 eviction-priority policies for the cache-hinted copies below (createpolicy, the
+// whole access range): evict-first for data read once (weight streams), so that it does
+// not push out of L2 the intermediates the next kernel reads again.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* m, uint64_t* bar,
+                                                 int c0, int c1, int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+      "l"(policy)
+      : "memory");
+}
+
 // Four rows (r0..r3) of a 2-D tensor, columns [c0, c0 + box width), in one copy. The
 // tensor map's box is one row high; the four rows land one after another in `dst`.
 __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar,
