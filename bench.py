@@ -181,19 +181,22 @@ STAGE_SOURCE = {"router": "router_sm100.cu", "select": "select.cu", "csr": "sele
 # ---- clocks during the timed region ----------------------------------------------------
 
 class ClockSampler:
-    """Samples SM clocks and clock-event reasons every millisecond through NVML (read
-    only), so that even a timed region of a few milliseconds holds several samples."""
+    """Samples SM clocks and clock-event reasons through NVML (read only) from a thread
+    that starts before the warm-up, every half millisecond, each sample stamped with the
+    host time; the record keeps the samples taken inside the timed region (mark()
+    brackets it), so that even a region of a few milliseconds holds several."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
-        self.samples = []
+        self.samples = []        # (host time, SM MHz, reason mask)
+        self.window = None
         self.mx = None
-        self.reasons = set()
         self.err = None
         self._stop = threading.Event()
+        self._switch = None
 
     def start(self):
         try:
@@ -210,19 +213,20 @@ class ClockSampler:
         except Exception as e:  # no NVML: report that instead of clocks
             self.err = f"nvml unavailable: {type(e).__name__}"
             return
+        # let the sampling thread run between the launching thread's calls
+        self._switch = sys.getswitchinterval()
+        sys.setswitchinterval(1e-4)
         self.t = threading.Thread(target=self._run, daemon=True)
         self.t.start()
 
     def _sample(self):
         nv = self.nv
-        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
         try:
             mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
         except AttributeError:
             mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
-        for name, bit in self.REASONS.items():
-            if mask & bit:
-                self.reasons.add(name)
+        self.samples.append((time.perf_counter(), mhz, mask))
 
     def _run(self):
         while not self._stop.is_set():
@@ -231,17 +235,34 @@ class ClockSampler:
             except Exception as e:
                 self.err = f"nvml sample failed: {type(e).__name__}"
                 return
-            self._stop.wait(0.001)
+            self._stop.wait(0.0005)
+
+    def mark(self, which):
+        """mark("begin") / mark("end") around the timed region."""
+        t = time.perf_counter()
+        self.window = (t, t) if which == "begin" else (self.window[0], t)
 
     def stop(self):
         if self.err and not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err]}
         self._stop.set()
         self.t.join(timeout=2)
-        if not self.samples:
+        if self._switch is not None:
+            sys.setswitchinterval(self._switch)
+        inside = self.samples
+        if self.window is not None:
+            lo, hi = self.window
+            inside = [x for x in self.samples if lo <= x[0] <= hi]
+            if not inside:  # none landed inside: the ones nearest each end
+                inside = sorted(self.samples, key=lambda x: min(abs(x[0] - lo),
+                                                                 abs(x[0] - hi)))[:2]
+        if not inside:
             self._sample()
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.mx,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+            inside = self.samples[-1:]
+        reasons = sorted(name for name, bit in self.REASONS.items()
+                         if any(m & bit for _, _, m in inside))
+        return {"sm_mhz": statistics.median(m for _, m, _ in inside), "sm_max_mhz": self.mx,
+                "reasons": reasons, "samples": len(inside)}
 
 
 # ---- the CPU oracle (reference arm and cpu_baseline) --------------------------------------
@@ -399,7 +420,7 @@ class Flush:
             self.clean.amax()
 
 
-def _timed_steps(step, K, flush, stream, barrier, per_step_events=True):
+def _timed_steps(step, K, flush, stream, barrier, clocks=None):
     """Exactly K steps between a barrier + synchronize on both sides; the L2 flush runs
     before each step, outside its CUDA events (recorded on the launching stream).
     Returns the summed milliseconds of the K steps."""
@@ -408,12 +429,16 @@ def _timed_steps(step, K, flush, stream, barrier, per_step_events=True):
           for _ in range(K)]
     barrier()
     torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.mark("begin")
     for i in range(K):
         flush()
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.mark("end")
     barrier()
     return sum(s_.elapsed_time(e_) for s_, e_ in ev)
 
@@ -444,6 +469,8 @@ def measure(args, w, seed, dev, dist, K, W, inter, shared_f=0, extras=True):
         if dist is not None:
             dist.barrier()
 
+    clocks = ClockSampler(dev.index)
+    clocks.start()
     for _ in range(W):
         flush()
         step()
@@ -453,9 +480,7 @@ def measure(args, w, seed, dev, dist, K, W, inter, shared_f=0, extras=True):
 
     # the timed region: K whole-layer steps, launched back to back as a user would,
     # with the SM clocks sampled throughout
-    clocks = ClockSampler(dev.index)
-    clocks.start()
-    ms = _timed_steps(step, K, flush, stream, barrier)
+    ms = _timed_steps(step, K, flush, stream, barrier, clocks)
     clk = clocks.stop()
     # per-stage times: K more steps with CUDA events between the stages (the events keep
     # the stages from overlapping their launches, so this pass is not the headline)

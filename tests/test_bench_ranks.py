@@ -120,3 +120,31 @@ def test_both_arms_carry_the_same_config():
     c = bench._workload_config(w)
     assert set(c) == {"workload", "T", "d", "E", "F", "C", "segments", "l2"}
     assert c == bench._workload_config(w, "write+read")
+
+
+def test_clock_sampler_reports_only_the_timed_region(monkeypatch):
+    # a fake NVML whose clock and reasons change when the timed region begins and ends:
+    # the record must hold only the samples taken in between
+    import time
+    import types
+    phase = {"v": 0}
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0, nvmlInit=lambda: None, nvmlDeviceGetHandleByIndex=lambda i: i,
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: (600, 1900, 700)[phase["v"]],
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: (0x40, 0x4, 0x8)[phase["v"]])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    cs = bench.ClockSampler(0)
+    cs.start()
+    time.sleep(0.02)
+    phase["v"] = 1
+    time.sleep(0.005)  # a sample under way when the phase changed has finished
+    cs.mark("begin")
+    time.sleep(0.02)
+    cs.mark("end")
+    phase["v"] = 2
+    time.sleep(0.02)
+    rec = cs.stop()
+    assert rec["samples"] >= 3
+    assert rec["sm_mhz"] == 1900 and rec["sm_max_mhz"] == 1965
+    assert rec["reasons"] == ["sw_power_cap"]
