@@ -62,6 +62,10 @@ def _args():
                          "N(0, 1), so plain bf16 intermediates meet every tolerance (the "
                          "full-row parity test checks it) and the down GEMM runs one MMA "
                          "per k-step instead of the split pair's two")
+    ap.add_argument("--min-timed-s", type=float, default=1.0,
+                    help="repeat the timed region (each repeat exactly --steps steps between "
+                         "a barrier + synchronize) until the repeats cover at least this "
+                         "many seconds of step time, so the clock record spans a long load")
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="only run this many layer calls of the workload, untimed, and exit "
                          "(a short, fixed launch sequence for ncu captures)")
@@ -127,6 +131,13 @@ def stage_bytes(w, shared_f=0):
         b["gemm2_scale"] += 2 * Fs * d + 2 * T * Fs + 2 * T * d
         b["combine"] += 2 * T * d + 2 * T * d
     return b
+
+
+def gather_bytes(w):
+    """The standalone gather (each expert's chosen rows of x copied into one contiguous
+    block): E*Ce bf16 rows read and written. The layer does not run it; its gate/up GEMM
+    reads the same rows into its A tiles (those bytes are in gemm1_swiglu above)."""
+    return 2 * 2 * w.E * w.Ce * w.d
 
 
 def stage_design_bytes(w, intermediate="split", shared_f=0):
@@ -420,7 +431,7 @@ class Flush:
             self.clean.amax()
 
 
-def _timed_steps(step, K, flush, stream, barrier, clocks=None):
+def _timed_steps(step, K, flush, stream, barrier, clocks=None, mark=("begin", "end")):
     """Exactly K steps between a barrier + synchronize on both sides; the L2 flush runs
     before each step, outside its CUDA events (recorded on the launching stream).
     Returns the summed milliseconds of the K steps."""
@@ -429,18 +440,35 @@ def _timed_steps(step, K, flush, stream, barrier, clocks=None):
           for _ in range(K)]
     barrier()
     torch.cuda.synchronize()
-    if clocks is not None:
-        clocks.mark("begin")
+    if clocks is not None and mark[0]:
+        clocks.mark(mark[0])
     for i in range(K):
         flush()
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
-    if clocks is not None:
-        clocks.mark("end")
+    if clocks is not None and mark[1]:
+        clocks.mark(mark[1])
     barrier()
     return sum(s_.elapsed_time(e_) for s_, e_ in ev)
+
+
+def _repeated_regions(run_region, clocks, min_s, dist, dev):
+    """The timed region, repeated: run_region(marks) times one region of exactly K steps
+    (marking the clock window's begin / end as told) and returns its milliseconds. The
+    first region fixes how many repeats cover min_s seconds of step time (the largest
+    count over the ranks, so that every rank runs the same collective sequence); the clock
+    record spans all of them. Returns the per-region milliseconds."""
+    import math
+    first = run_region(("begin", None))
+    want = max(1, math.ceil(min_s * 1e3 / max(first, 1e-6))) if min_s > 0 else 1
+    reps = int(max_over_ranks([float(want)], dist, dev)[0])
+    regions = [first]
+    for _ in range(1, reps):
+        regions.append(run_region((None, None)))
+    clocks.mark("end")
+    return regions
 
 
 def measure(args, w, seed, dev, dist, K, W, inter, shared_f=0, extras=True):
@@ -479,15 +507,18 @@ def measure(args, w, seed, dev, dist, K, W, inter, shared_f=0, extras=True):
         raise RuntimeError("device-side check failed during warm-up")
 
     # the timed region: K whole-layer steps, launched back to back as a user would,
-    # with the SM clocks sampled throughout
-    ms = _timed_steps(step, K, flush, stream, barrier, clocks)
+    # repeated until the repeats cover --min-timed-s, with the SM clocks sampled throughout
+    regions = _repeated_regions(
+        lambda mk: _timed_steps(step, K, flush, stream, barrier, clocks, mark=mk), clocks,
+        args.min_timed_s, dist, dev)
+    ms = sum(regions) / len(regions)   # mean milliseconds of one K-step region
     clk = clocks.stop()
     # per-stage times: K more steps with CUDA events between the stages (the events keep
     # the stages from overlapping their launches, so this pass is not the headline)
     traced_ms = _timed_steps(lambda: step(trace), K, flush, stream, barrier)
     stage_ms, ncalls = trace.read()
     trace.close()
-    r = dict(ms=ms, traced_ms=traced_ms, clocks=clk,
+    r = dict(ms=ms, regions=len(regions), region_ms=regions, traced_ms=traced_ms, clocks=clk,
              stage_ms={k: v / max(ncalls, 1) for k, v in stage_ms.items()},
              launches=nm.kernels_per_call(w.T, w.d, w.E, w.F, w.C, intermediate=inter,
                                           n_segments=w.segments, shared_f=shared_f or None))
@@ -507,6 +538,14 @@ def measure(args, w, seed, dev, dist, K, W, inter, shared_f=0, extras=True):
         r["graph_ms"] = _timed_steps(graph.replay, K, flush, stream, barrier)
         del graph
         r.update(_e2e(args, w, a, d, block, ws, inter, K, W, dev, barrier))
+        # the standalone gather of the chosen rows (not part of the layer's step)
+        _, scores_t = nm.router(x, W_r, n_segments=w.segments)
+        idx = nm.select(scores_t, w.C, n_segments=w.segments, csr=False)[0]
+        packed = torch.empty(idx.numel(), w.d, dtype=x.dtype, device=dev)
+        nm.gather_rows(x, idx, out=packed)
+        r["gather_ms"] = _timed_steps(lambda: nm.gather_rows(x, idx, out=packed), K, flush,
+                                      stream, barrier) / K
+        del packed
     if nm.get_last_error() != 0:
         raise RuntimeError("device-side check failed during the timed steps")
     return r
@@ -579,6 +618,17 @@ def _stage_report(w, stage_ms, peaks, inter, shared_f):
     return out
 
 
+def _gather_report(w, ms, peaks):
+    """The standalone gather's HBM figure (timed alone, K launches, L2 flushed before
+    each)."""
+    b = gather_bytes(w)
+    return {"us": ms * 1e3, "GB/s": b / (ms / 1e3) / 1e9,
+            "hbm_frac": b / (ms / 1e3) / 1e9 / peaks["hbm"], "bytes_per_launch": b,
+            "how": "nmoe_rows_gather of the layer's own idx [E, Ce] from x into one block "
+                   "per expert, timed alone; the layer fuses this copy into the gate/up "
+                   "GEMM's A-tile loads, so it is not part of the step"}
+
+
 def _roofline(w, stage_ms, peaks, inter, shared_f):
     """The dominant kernel's roofline: the larger of its algorithmic byte time and its
     FLOP time at the measured peaks (the sustained tensor figure: the kernel runs inside
@@ -642,8 +692,9 @@ def run_ours(args, w, rank, world, local_rank, dist):
         wt = I.WORKLOADS[args.tensor_workload]
         tb = measure(args, wt, rank, dev, dist, K, W, args.tensor_intermediate, 0,
                      extras=False)
-    keys = ["ms", "traced_ms", "graph_ms", "e2e_ms"] + (["tb_ms"] if tb else [])
-    vals = [m["ms"], m["traced_ms"], m["graph_ms"], m["e2e_ms"]] + ([tb["ms"]] if tb else [])
+    keys = ["ms", "traced_ms", "graph_ms", "e2e_ms", "gather_ms"] + (["tb_ms"] if tb else [])
+    vals = ([m["ms"], m["traced_ms"], m["graph_ms"], m["e2e_ms"], m["gather_ms"]]
+            + ([tb["ms"]] if tb else []))
     mx = dict(zip(keys, max_over_ranks(vals, dist, dev)))
     if rank != 0:
         return
@@ -655,6 +706,11 @@ def run_ours(args, w, rank, world, local_rank, dist):
         "metric": METRIC, "value": replica_throughput(w.T, world, K, mx["ms"]),
         "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": mx["ms"] / K, "higher_is_better": True, "scaling": "weak",
+        "timed_regions": {"count": m["regions"], "steps_each": K,
+                          "ms_per_step_each": [round(x / K, 5) for x in m["region_ms"]],
+                          "how": "the K-step timed region repeated until the repeats cover "
+                                 f"{args.min_timed_s:g} s of step time; value and ms_per_step "
+                                 "are their mean (the slowest rank's)"},
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": _workload_config(w, args.l2_flush),
         "parallelism": f"replicas x{world} (one independent layer per GPU, no exchange)",
@@ -667,6 +723,7 @@ def run_ours(args, w, rank, world, local_rank, dist):
         "tensor_frac_of_layer": flops / per_step_s / 1e12 / peaks["tensor_sustained"],
         "roofline": _roofline(w, m["stage_ms"], peaks, inter, args.shared_f),
         "stages": _stage_report(w, m["stage_ms"], peaks, inter, args.shared_f),
+        "gather": _gather_report(w, mx["gather_ms"], peaks),
         "traced_ms_per_step": mx["traced_ms"] / K,
         "graph_replay": {"ms_per_step": mx["graph_ms"] / K,
                          "value": replica_throughput(w.T, world, K, mx["graph_ms"]),
@@ -689,6 +746,7 @@ def run_ours(args, w, rank, world, local_rank, dist):
         line["tensor_bound"] = {
             "config": _workload_config(wt, args.l2_flush), "intermediates": ti,
             "steps": K, "warmup": W, "ms_per_step": mx["tb_ms"] / K,
+            "timed_regions": tb["regions"],
             "value": replica_throughput(wt.T, world, K, mx["tb_ms"]), "unit": "tokens/s",
             "tflops": tflops / t_s / 1e12,
             "tensor_frac_of_layer": tflops / t_s / 1e12 / peaks["tensor_sustained"],

@@ -8,6 +8,6 @@ synthetic workload generators. The shared library ``libnmoe.so`` is built in pla
 
 from . import inputs  # noqa: F401
 from ._lib import (  # noqa: F401
-    EXPORTS, LIB_PATH, NmoeError, Trace, build_info, forward, get_last_error,
+    EXPORTS, LIB_PATH, NmoeError, Trace, build_info, forward, gather_rows, get_last_error,
     kernels_per_call, lib, router, select, workspace_size,
 )

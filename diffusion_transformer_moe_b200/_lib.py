@@ -246,6 +246,23 @@ def select(scores_t, C_: int, n_segments=1, csr=True, stream=None):
     return idx, gate, tok_ptr, tok_ent
 
 
+def gather_rows(src, rows, out=None, stream=None):
+    """out[i] = src[rows[i]] (a zero row where rows[i] < 0): rows of a 2-D device tensor
+    whose row is a multiple of 16 bytes; rows is device int32 (any shape, read flat).
+    With src = x and rows = idx, out holds each expert's chosen rows as one block."""
+    _dev(src, "src"); _dev(rows, "rows")
+    if src.dim() != 2 or not src.is_contiguous() or rows.dtype != torch.int32 \
+            or not rows.is_contiguous():
+        raise ValueError("src must be a contiguous 2-D tensor and rows contiguous int32")
+    n = rows.numel()
+    if out is None:
+        out = torch.empty(n, src.shape[1], dtype=src.dtype, device=src.device)
+    _check(lib().nmoe_rows_gather(src.data_ptr(), rows.data_ptr(), n,
+                                  src.shape[1] * src.element_size(), out.data_ptr(),
+                                  _stream(stream)), "nmoe_rows_gather")
+    return out
+
+
 def forward(x, W_r, W1, W3, W2, C_: int, out=None, stream=None, **opts):
     """The whole layer. ``opts`` are the nmoe_options fields (score_fn, combine,
     route_scale, n_segments, router_bias, workspace, scores_out, idx_out, trace,

@@ -498,7 +498,8 @@ nmoe_status nmoe_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent, int64_t
 namespace {
 nmoe_status rows_copy(const void* src, const int32_t* rows, int64_t n, int64_t row_bytes,
                       void* dst, bool gather, nmoe_stream_t stream) {
-  if (n < 0 || row_bytes < 16 || row_bytes % 16 != 0) return NMOE_ERR_INVALID_ARG;
+  if (n < 0 || row_bytes < 16 || row_bytes % 16 != 0 || row_bytes / 16 > INT32_MAX)
+    return NMOE_ERR_INVALID_ARG;
   if (n > 0 && (!src || !rows || !dst || !aligned16(src) || !aligned16(dst)))
     return NMOE_ERR_INVALID_ARG;
   DevState* ds = nullptr;

@@ -237,7 +237,16 @@ NMOE_API nmoe_status nmoe_ep_rows(const int32_t* tok_ptr, const int32_t* tok_ent
 
 /* dst[i, :] = src[rows[i], :] (gather; a zero row where rows[i] < 0) / dst[rows[i], :] =
  * src[i, :] (scatter; nothing where rows[i] < 0) for i < n: rows of row_bytes bytes (a
- * positive multiple of 16), 16-byte aligned device arrays; rows device int32. */
+ * positive multiple of 16), 16-byte aligned device arrays; rows device int32. Ownership
+ * stays with the caller; rows[i] must index a row of src (gather) or dst (scatter); any
+ * other rows[i] >= 0 is an error the library cannot detect.
+ *
+ * With src = x and rows = the chosen tokens idx [E, Ce] (flattened), the gather is the
+ * grouped-matmul path's "permute the tokens into contiguous per-expert blocks" step
+ * (NucleusMoE-Image walkthrough, section 6): dst holds each expert's Ce rows as one
+ * block. The layer itself never runs it (the gate/up GEMM reads the chosen rows of x
+ * straight into its A tiles); it stands alone for expert parallelism and to measure
+ * that copy's bandwidth. */
 NMOE_API nmoe_status nmoe_rows_gather(const void* src, const int32_t* rows, int64_t n,
                                       int64_t row_bytes, void* dst, nmoe_stream_t stream);
 NMOE_API nmoe_status nmoe_rows_scatter(const void* src, const int32_t* rows, int64_t n,

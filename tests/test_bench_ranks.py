@@ -24,9 +24,25 @@ dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
 # rank-dependent timings: the job is as slow as its slowest rank, per quantity
 mine = [10.0 + 2.0 * rank, 30.0 - rank, 5.0]
 got = bench.max_over_ranks(mine, dist, "cpu")
+# repeated timed regions: rank 0's regions take 100 ms, rank 1's 400 ms; both must run
+# the larger count (10 regions for 1 s), so their collectives stay paired
+class Clk:
+    marks = []
+    def mark(self, m):
+        self.marks.append(m)
+clk = Clk()
+calls = []
+def region(mk):
+    calls.append(mk)
+    if mk[0]:
+        clk.mark(mk[0])
+    dist.barrier()
+    return 100.0 if rank == 0 else 400.0
+regions = bench._repeated_regions(region, clk, 1.0, dist, "cpu")
 dist.barrier()
 dist.destroy_process_group()
-print(json.dumps({"rank": rank, "got": got}))
+print(json.dumps({"rank": rank, "got": got, "regions": regions, "calls": calls,
+                  "marks": clk.marks}))
 """
 
 
@@ -57,6 +73,27 @@ def test_two_gloo_ranks_take_the_max_of_every_timing():
         outs.append(json.loads(o.strip().splitlines()[-1]))
     for r in outs:
         assert r["got"] == [12.0, 30.0, 5.0]
+        assert len(r["regions"]) == 10
+        assert r["calls"][0] == ["begin", None]
+        assert all(c == [None, None] for c in r["calls"][1:])
+        assert r["marks"] == ["begin", "end"]
+
+
+def test_one_rank_repeats_regions_until_the_minimum_time():
+    class Clk:
+        def __init__(self):
+            self.marks = []
+
+        def mark(self, m):
+            self.marks.append(m)
+
+    clk = Clk()
+    times = iter([300.0, 310.0, 290.0, 305.0, 999.0])
+    regions = bench._repeated_regions(lambda mk: next(times), clk, 1.0, None, "cpu")
+    assert regions == [300.0, 310.0, 290.0, 305.0]     # ceil(1000 / 300) = 4
+    assert clk.marks == ["end"]                         # the region marks its own begin
+    assert bench._repeated_regions(lambda mk: 5000.0, clk, 1.0, None, "cpu") == [5000.0]
+    assert bench._repeated_regions(lambda mk: 1.0, clk, 0.0, None, "cpu") == [1.0]
 
 
 def test_replica_throughput_counts_every_rank_over_the_slowest_time():
