@@ -72,10 +72,10 @@ struct Cfg {
   static constexpr int kEpiWarp0 = 2 + kAWarps;
   static constexpr int kThreads = 32 * (2 + kAWarps + kEpiWarps);
   static constexpr int kFullCount = 1 + 32 * kAWarps;    // TMA arrive + one per gather thread
-  // staging block per epilogue warp: gemm2 with fp32 Y, 32 rows x 32 fp32; gemm1, 32
-  // rows x 32 bf16 of H (and as much again for H lo)
+  // staging block per epilogue warp: gemm2, 32 rows x 128 bytes of Y (32 fp32 with SPLIT,
+  // else 64 bf16); gemm1, 32 rows x 32 bf16 of H (and as much again for H lo)
   static constexpr int kEpiStage =
-      MODE == kGemm2 ? (SPLIT ? 32 * 32 * 4 : 0) : (SPLIT ? 2 * 32 * 64 : 32 * 64);
+      MODE == kGemm2 ? 32 * 128 : (SPLIT ? 2 * 32 * 64 : 32 * 64);
   static constexpr size_t kSmem = kRingBytes + kEpiWarps * kEpiStage + 1024;
   static_assert(kSmem <= 232448, "dynamic shared memory beyond the 227 KB a CTA may use");
 };
@@ -467,8 +467,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
         // staging block of this warp: 16-byte chunk c of row r at r * 128 + (c ^ (r % 8)) * 16
         float* sb = reinterpret_cast<float*>(epi_smem +
                                              (warp - C::kEpiWarp0) * C::kEpiStage);
+        // columns per round: 32 fp32 (SPLIT) or 64 bf16, 128 bytes of the row either way
+        constexpr int kStep = SPLIT ? 32 : 64;
 #pragma unroll 1
-        for (int j0 = c_lo; j0 < c_lo + c_n; j0 += 32) {
+        for (int j0 = c_lo; j0 < c_lo + c_n; j0 += kStep) {
           uint32_t y[32];
           tmem_ld32(taddr + j0, y);
           tmem_ld_wait();
@@ -508,46 +510,62 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
             }
             __syncwarp();  // the block is read before the next chunk overwrites it
           } else {
-            uint32_t h[16];
+            // 64 columns: this round's 32 and the next 32, as bf16 (one rounding each)
+            uint32_t h[32];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               h[i] = pack_bf16x2(gw * __uint_as_float(y[2 * i]),
                                  gw * __uint_as_float(y[2 * i + 1]));
-            if (valid && !direct) {
-              __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.out) + orow;
+            tmem_ld32(taddr + j0 + 32, y);
+            tmem_ld_wait();
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const int c = n0 + j0 + 8 * v;
-                if (c < p.N)
-                  *reinterpret_cast<uint4*>(yr + c) =
-                      make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+            for (int i = 0; i < 16; ++i)
+              h[16 + i] = pack_bf16x2(gw * __uint_as_float(y[2 * i]),
+                                      gw * __uint_as_float(y[2 * i + 1]));
+            // Each thread holds one row's 128 bytes; through the staging block a store
+            // covers 4 rows with 128 contiguous bytes each (instead of 32 rows x 16 bytes).
+            uint8_t* sh = reinterpret_cast<uint8_t*>(sb);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(sh + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
+            __syncwarp();
+            const int c = lane & 7;
+            const int col = n0 + j0 + 8 * c;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = 4 * i + (lane >> 3);
+              const int64_t ro = __shfl_sync(0xffffffffu, orow, r);
+              const int rv = __shfl_sync(0xffffffffu, (int)valid, r);
+              const int rd = __shfl_sync(0xffffffffu, (int)direct, r);
+              const uint4 v = *reinterpret_cast<const uint4*>(sh + r * 128 + ((c ^ (r & 7)) << 4));
+              if (!rv || col >= p.N) continue;
+              if (!rd) {
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ro + col) = v;
+                continue;
               }
-            } else if (valid) {
               // the combine's sum of one bf16 term: 0 + float(bf16(y)), rounded once
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+              float f[8];
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const int c = n0 + j0 + 8 * v;
-                if (c >= p.N) continue;
-                float f[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float2 t = __bfloat1622float2(
-                      *reinterpret_cast<const __nv_bfloat162*>(&h[4 * v + i]));
-                  f[2 * i] = t.x + 0.f;
-                  f[2 * i + 1] = t.y + 0.f;
-                }
-                if (p.out_direct_f32) {
-                  float* o = static_cast<float*>(p.out_direct) + orow + c;
-                  *reinterpret_cast<float4*>(o) = make_float4(f[0], f[1], f[2], f[3]);
-                  *reinterpret_cast<float4*>(o + 4) = make_float4(f[4], f[5], f[6], f[7]);
-                } else {
-                  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out_direct) + orow +
-                                            c) =
-                      make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-                }
+              for (int k = 0; k < 4; ++k) {
+                const float2 t =
+                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+                f[2 * k] = t.x + 0.f;
+                f[2 * k + 1] = t.y + 0.f;
+              }
+              if (p.out_direct_f32) {
+                float* o = static_cast<float*>(p.out_direct) + ro + col;
+                *reinterpret_cast<float4*>(o) = make_float4(f[0], f[1], f[2], f[3]);
+                *reinterpret_cast<float4*>(o + 4) = make_float4(f[4], f[5], f[6], f[7]);
+              } else {
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out_direct) + ro +
+                                          col) =
+                    make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                               pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
               }
             }
+            __syncwarp();  // the block is read before the next round overwrites it
           }
         }
       }
