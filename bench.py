@@ -79,10 +79,15 @@ def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
+        # the SM clock the sustained figure was taken at, where the file records one
+        mhz = next((v for k, v in d.items() if isinstance(v, (int, float))
+                    and "sustained" in k and "mhz" in k.lower()), None)
         return dict(hbm=d["hbm_gbs"], tensor=d["bf16_tflops"],
                     tensor_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
-                    source="measured")
-    return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, source="fallback")
+                    sustained_mhz=mhz, source="measured")
+    # fallback: the sustained bf16 figure was taken at about 1.3 GHz under the power cap
+    return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, sustained_mhz=1300.0,
+                source="fallback")
 
 
 L2_NOTE = {
@@ -591,7 +596,34 @@ def _e2e(args, w, a, d, block, ws, inter, K, W, dev, barrier):
     t1.record(streams[0])
     torch.cuda.synchronize()
     barrier()
-    return dict(e2e_ms=t0.elapsed_time(t1), e2e_streams=n_streams,
+    e2e_ms = t0.elapsed_time(t1)
+    # the same steps' copies alone (x in, out back, the same streams and buffers): the
+    # end-to-end step's PCIe ceiling
+    xd = [torch.empty_like(d["x"]) for _ in range(n_streams)]
+    od = [torch.empty(outs[0].shape, dtype=outs[0].dtype, device=dev) for _ in range(n_streams)]
+
+    def copy_step(i):
+        j = i % n_streams
+        with torch.cuda.stream(streams[j]):
+            xd[j].copy_(x_host, non_blocking=True)
+            outs[j].copy_(od[j], non_blocking=True)
+
+    for i in range(n_streams):
+        copy_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    t0.record(streams[0])
+    for s_ in streams[1:]:
+        s_.wait_event(t0)
+    for i in range(K):
+        copy_step(i)
+    for s_ in streams[1:]:
+        streams[0].wait_stream(s_)
+    t1.record(streams[0])
+    torch.cuda.synchronize()
+    barrier()
+    return dict(e2e_ms=e2e_ms, copy_ms=t0.elapsed_time(t1), e2e_streams=n_streams,
                 h2d=x_host.numel() * x_host.element_size(),
                 d2h=outs[0].numel() * outs[0].element_size())
 
@@ -692,8 +724,9 @@ def run_ours(args, w, rank, world, local_rank, dist):
         wt = I.WORKLOADS[args.tensor_workload]
         tb = measure(args, wt, rank, dev, dist, K, W, args.tensor_intermediate, 0,
                      extras=False)
-    keys = ["ms", "traced_ms", "graph_ms", "e2e_ms", "gather_ms"] + (["tb_ms"] if tb else [])
-    vals = ([m["ms"], m["traced_ms"], m["graph_ms"], m["e2e_ms"], m["gather_ms"]]
+    keys = (["ms", "traced_ms", "graph_ms", "e2e_ms", "copy_ms", "gather_ms"]
+            + (["tb_ms"] if tb else []))
+    vals = ([m["ms"], m["traced_ms"], m["graph_ms"], m["e2e_ms"], m["copy_ms"], m["gather_ms"]]
             + ([tb["ms"]] if tb else []))
     mx = dict(zip(keys, max_over_ranks(vals, dist, dev)))
     if rank != 0:
@@ -734,7 +767,10 @@ def run_ours(args, w, rank, world, local_rank, dist):
                 "ms_per_step": mx["e2e_ms"] / K,
                 "how": "nmoe_forward_ex with host_io (x copied in, out copied back to pinned "
                        "host memory inside each call), steps rotating over "
-                       f"{m['e2e_streams']} streams"},
+                       f"{m['e2e_streams']} streams",
+                "copies_only_ms_per_step": mx["copy_ms"] / K,
+                "frac_of_copies_only": mx["copy_ms"] / mx["e2e_ms"],
+                "pcie_GBps_per_direction": m["h2d"] * K / (mx["copy_ms"] / 1e3) / 1e9},
         "clocks": m["clocks"],
     }
     if tb is not None:
@@ -757,6 +793,16 @@ def run_ours(args, w, rank, world, local_rank, dist):
             "stages": st, "gpu_launches": K * tb["launches"],
             "clocks": tb["clocks"],
         }
+        mhz, ref = tb["clocks"].get("sm_mhz"), peaks.get("sustained_mhz")
+        if mhz and ref:
+            # tensor throughput scales with the SM clock: the sustained peak at the median
+            # clock this run held under the power cap
+            pk = peaks["tensor_sustained"] * mhz / ref
+            line["tensor_bound"]["clock_normalized"] = {
+                "sm_mhz": mhz, "peak_reference_mhz": ref, "peak_at_sm_mhz": pk,
+                "tensor_frac_of_layer": tflops / t_s / 1e12 / pk,
+                "gemms": {k: st[k]["TFLOP/s"] / pk for k in ("gemm1_swiglu", "gemm2_scale")},
+            }
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
