@@ -584,6 +584,253 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
   }
 }
 
+// ---- the down projection on CTA pairs (bf16 intermediates, long expert blocks) ----------
+//
+// With bf16 H and Y and at least 256 rows per expert, gemm2 runs on pairs of CTAs (a 2-CTA
+// cluster): one tcgen05.mma.cta_group::2 per k-step covers 256 rows of one expert (128
+// from each CTA's shared memory) x N = 256 columns of d, and each CTA stages only half of
+// the W2 tile (128 columns). Per CTA and k-block the ring takes 16 KB of H and 16 KB of W2
+// instead of 16 KB + 32 KB for the same MMA work, so six stages fit. Each CTA's TMEM
+// receives its own 128 rows for all 256 columns, and its epilogue is the one-CTA kernel's.
+//
+// Barriers: the ring's full barriers live in the leader (rank 0): both CTAs' copies
+// complete on them (cta_group::2) and the leader's producer alone arrives, announcing both
+// CTAs' bytes (the other CTA's copies may land first: the phase cannot complete while that
+// arrival is missing). The empty and accumulator-full barriers live in each CTA (the
+// leader's MMA thread commits to both); the accumulator-empty barriers in the leader (all
+// sixteen epilogue warps of the pair arrive). Every wait is bounded.
+constexpr int kPairStages = 6;
+constexpr int kPairABytes = kABytes;                             // 128 rows x 64 K
+constexpr int kPairBBytes = 2 * kBBoxBytes;                      // 128 columns x 64 K
+constexpr int kPairStageBytes = kPairABytes + kPairBBytes;       // 32 KB
+constexpr int kPairEpiWarps = 8;
+constexpr int kPairThreads = 32 * (2 + kPairEpiWarps);
+constexpr int kPairEpiStage = 32 * 128;
+constexpr size_t kPairSmem =
+    (size_t)kPairStages * kPairStageBytes + kPairEpiWarps * kPairEpiStage + 1024;
+static_assert(kPairSmem <= 232448, "dynamic shared memory beyond the 227 KB a CTA may use");
+
+__global__ void __launch_bounds__(kPairThreads, 1)
+pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
+                  const __grid_constant__ CUtensorMap map_w, const Params p) {
+  pdl_launch_dependents();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[kPairStages], empty_bar[kPairStages];
+  __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: the leader, which issues the MMAs
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int nk = (p.K + kBK - 1) / kBK;
+  auto a_tile = [&](int st) { return smem + st * kPairStageBytes; };
+  auto b_tile = [&](int st) { return smem + st * kPairStageBytes + kPairABytes; };
+  uint8_t* const epi_smem = smem + (size_t)kPairStages * kPairStageBytes;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPairStages; ++i) {
+      mbar_init(&full_bar[i], 1);  // the leader's producer, with both CTAs' bytes
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull_bar[i], 1);
+      mbar_init(&tempty_bar[i], 2 * kPairEpiWarps);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&map_h);
+    prefetch_tensormap(&map_w);
+  }
+  if (warp == 1) tmem_alloc_pair(&tmem_base_sh, kTmemCols);
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers are initialised and the TMEM is allocated
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+  volatile int* abort_v = &abort_flag;
+  pdl_wait();  // the previous kernel's outputs (H, gate, ent_pos) are complete
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    const uint64_t wpol = l2_policy_evict_first();
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int item = pair; item < p.num_items; item += npairs) {
+      const Tile tl = tile_of(item, p, 256);
+      const int nbox = tl.half ? 1 : 2;  // 64-column boxes of this CTA's half of the W2 tile
+      const uint32_t bytes = (uint32_t)(kPairABytes + nbox * kBBoxBytes);
+      // tile_of counts row blocks of kBM; a pair item spans two of them
+      const int hrow = tl.e * p.Ce + 2 * tl.m0 + (int)rank * kBM;
+      const int col0 = tl.n0 + (int)rank * nbox * 64;
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1, abort_v, p.wait_ns);
+        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+        if (!ok) break;
+        const uint32_t fb = mapa_shared(&full_bar[stage], 0);
+        if (lane == 0 && rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * bytes);
+        __syncwarp();
+        const int k0 = kb * kBK;
+        if (lane == 0) tma_load_2d_pair(a_tile(stage), &map_h, fb, k0, hrow);
+        if (lane >= 1 && lane <= nbox)
+          tma_load_3d_pair(b_tile(stage) + (lane - 1) * kBBoxBytes, &map_w, fb,
+                           col0 + 64 * (lane - 1), k0, tl.e, wpol);
+        if (++stage == kPairStages) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (the leader's one thread) ----------------
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc_full = idesc_bf16(256, 256, 1);  // B (W2) MN-major
+      constexpr uint32_t idesc_half = idesc_bf16(256, 128, 1);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int item = pair; item < p.num_items && ok; item += npairs) {
+        const uint32_t idesc = tile_of(item, p, 256).half ? idesc_half : idesc_full;
+        if (!(ok = mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_v, p.wait_ns))) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!(ok = mbar_wait(&full_bar[stage], phase, abort_v, p.wait_ns))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(smem_u32(a_tile(stage)) + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(smem_u32(b_tile(stage)) + kk * 2048, kBBoxBytes, 1024);
+            mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          mma_commit_pair(mapa_shared(&empty_bar[stage], 0));
+          mma_commit_pair(mapa_shared(&empty_bar[stage], 1));
+          if (++stage == kPairStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit_pair(mapa_shared(&tfull_bar[acc], 0));
+        mma_commit_pair(mapa_shared(&tfull_bar[acc], 1));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      // every MMA issued above has completed once drain_bar flips
+      mma_commit_pair(mapa_shared(&drain_bar, 0));
+      int dummy = 0;
+      mbar_wait(&drain_bar, 0, &dummy, kDrainNs);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: eight warps per CTA, two per TMEM lane quarter ----------
+    // This CTA's 128 rows of the item, every column; the one-CTA kernel's bf16 path.
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    uint8_t* sh = epi_smem + (warp - 2) * kPairEpiStage;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int item = pair; item < p.num_items; item += npairs) {
+      const Tile tl = tile_of(item, p, 256);
+      const int acc_n = tl.half ? 128 : 256;
+      const int c_n = acc_n / 2;
+      const int c_lo = half * c_n;
+      int w = 1;
+      if (lane == 0) w = mbar_wait(&tfull_bar[acc], acc_phase, abort_v, p.wait_ns);
+      if (__shfl_sync(0xffffffffu, w, 0) == 0) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * kAccCols;
+      const int s = 2 * tl.m0 + (int)rank * kBM + row;   // item rows: 2 * m0 + [0, 256)
+      bool valid = s < p.Ce;
+      const int64_t ent = (int64_t)tl.e * p.Ce + (valid ? s : 0);
+      int64_t pos = p.ent_pos[ent];
+      if (kDebugChecks && valid &&
+          (pos >= p.rows_y ||
+           (pos < 0 && (p.out_direct == nullptr || -pos - 1 >= (int64_t)p.rows_x)))) {
+        atomicOr(p.err, kErrDeviceCheck);
+        valid = false;
+        pos = 0;
+      }
+      const bool direct = pos < 0;   // the token's only entry
+      const int64_t orow = (direct ? -pos - 1 : pos) * p.N;
+      const float gw = valid ? (p.gate ? p.gate[ent] : 1.f) : 0.f;
+#pragma unroll 1
+      for (int j0 = c_lo; j0 < c_lo + c_n; j0 += 64) {
+        uint32_t y[32], h[32];
+        tmem_ld32(taddr + j0, y);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          h[i] = pack_bf16x2(gw * __uint_as_float(y[2 * i]), gw * __uint_as_float(y[2 * i + 1]));
+        tmem_ld32(taddr + j0 + 32, y);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          h[16 + i] =
+              pack_bf16x2(gw * __uint_as_float(y[2 * i]), gw * __uint_as_float(y[2 * i + 1]));
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(sh + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+              make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
+        __syncwarp();
+        const int c = lane & 7;
+        const int col = tl.n0 + j0 + 8 * c;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 4 * i + (lane >> 3);
+          const int64_t ro = __shfl_sync(0xffffffffu, orow, r);
+          const int rv = __shfl_sync(0xffffffffu, (int)valid, r);
+          const int rd = __shfl_sync(0xffffffffu, (int)direct, r);
+          const uint4 v = *reinterpret_cast<const uint4*>(sh + r * 128 + ((c ^ (r & 7)) << 4));
+          if (!rv || col >= p.N) continue;
+          if (!rd) {
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ro + col) = v;
+            continue;
+          }
+          // the combine's sum of one bf16 term: 0 + float(bf16(y)), rounded once
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          float f[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[k]));
+            f[2 * k] = t.x + 0.f;
+            f[2 * k + 1] = t.y + 0.f;
+          }
+          if (p.out_direct_f32) {
+            float* o = static_cast<float*>(p.out_direct) + ro + col;
+            *reinterpret_cast<float4*>(o) = make_float4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<float4*>(o + 4) = make_float4(f[4], f[5], f[6], f[7]);
+          } else {
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out_direct) + ro + col) =
+                make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                           pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+          }
+        }
+        __syncwarp();  // the block is read before the next round overwrites it
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(&tempty_bar[acc], 0));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  __syncthreads();
+  if (*abort_v) {
+    // a wait ran out: give the copies this CTA issued (which complete on the leader's
+    // barriers, out of this CTA's sight) time to land before the pair's final barrier
+    const uint64_t t0 = globaltimer_ns();
+    while ((int64_t)(globaltimer_ns() - t0) < 1000000) {
+    }
+  }
+  cluster_sync_all();  // the other CTA no longer touches this CTA's barriers or TMEM
+  if (threadIdx.x == 0 && abort_flag) atomicOr(p.err, kErrTimeout);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 // ---- host side ----------------------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -698,10 +945,64 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
                : launch<kGemm1, false, kGatherLsu>(ma, ma, mb0, mb1, xb, p, sm_count, st, s.pdl);
 }
 
-cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
-                               const int32_t* ent_pos, const void* W2, const Shape& s, bool split,
-                               void* Y, void* out_direct, bool out_direct_f32, unsigned* err,
-                               int sm_count, cudaStream_t st) {
+namespace {
+
+// Pairs of SMs that can hold one pair CTA each at the same time (a pair's two CTAs sit on
+// one TPC): what the occupancy calculator reports for 2-CTA clusters of the pair kernel.
+int pair_slots(int sm_count) {
+  static int slots = -1;
+  if (slots < 0) {
+    int n = 0;
+    if (set_smem_limit(reinterpret_cast<const void*>(pair_gemm2_kernel), kPairSmem) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(sm_count & ~1));
+      cfg.blockDim = dim3(kPairThreads);
+      cfg.dynamicSmemBytes = kPairSmem;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, pair_gemm2_kernel, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    slots = n;
+  }
+  return slots;
+}
+
+cudaError_t launch_gemm2_pair(const void* H, const float* gate, const int32_t* ent_pos,
+                              const void* W2, const Shape& s, void* Y, void* out_direct,
+                              bool out_direct_f32, unsigned* err, int npairs, cudaStream_t st) {
+  CUtensorMap mh, mw;
+  const int64_t rows = (int64_t)s.E * s.Ce;
+  if (!rows_map(&mh, H, rows, s.F, kBM) || !weight_map(&mw, W2, s.E, s.F, s.d))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.Ce = s.Ce; p.K = s.F; p.N = s.d;
+  p.tiles_m = (int)ceil_div(s.Ce, 2 * kBM);
+  p.tiles_n = (int)ceil_div(s.d, 256);
+  p.num_tiles = s.E * p.tiles_m * p.tiles_n;
+  split_tail(p, npairs);
+  p.idx = nullptr; p.gate = gate; p.ent_pos = ent_pos; p.out = Y; p.out_lo = nullptr;
+  p.out_direct = out_direct; p.out_direct_f32 = out_direct_f32 ? 1 : 0;
+  p.csr_blocks = 0;
+  p.err = err;
+  p.wait_ns = s.wait_ns;
+  p.rows_x = s.T;
+  p.rows_y = s.y_rows;
+  const int pairs = p.num_items < npairs ? p.num_items : npairs;
+  return launch_kernel(pair_gemm2_kernel, dim3((unsigned)(2 * pairs)), dim3(kPairThreads),
+                       kPairSmem, st, s.pdl, 2, mh, mw, p);
+}
+
+cudaError_t launch_gemm2_one_cta(const void* H_hi, const void* H_lo, const float* gate,
+                                 const int32_t* ent_pos, const void* W2, const Shape& s,
+                                 bool split, void* Y, void* out_direct, bool out_direct_f32,
+                                 unsigned* err, int sm_count, cudaStream_t st) {
   CUtensorMap ma, ma2, mb;
   const int64_t rows = (int64_t)s.E * s.Ce;
   if (!rows_map(&ma, H_hi, rows, s.F, kBM) || !weight_map(&mb, W2, s.E, s.F, s.d))
@@ -723,6 +1024,23 @@ cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* 
   p.rows_y = s.y_rows;
   return split ? launch<kGemm2, true, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl)
                : launch<kGemm2, false, kGatherLsu>(ma, ma2, mb, mb, nullptr, p, sm_count, st, s.pdl);
+}
+
+}  // namespace
+
+bool gemm2_sm100_uses_pairs(const Shape& s, bool split, int sm_count) {
+  return !split && s.Ce >= 2 * kBM && s.d % 64 == 0 && pair_slots(sm_count) > 0;
+}
+
+cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
+                               const int32_t* ent_pos, const void* W2, const Shape& s, bool split,
+                               void* Y, void* out_direct, bool out_direct_f32, unsigned* err,
+                               int sm_count, cudaStream_t st) {
+  if (gemm2_sm100_uses_pairs(s, split, sm_count))
+    return launch_gemm2_pair(H_hi, gate, ent_pos, W2, s, Y, out_direct, out_direct_f32, err,
+                             pair_slots(sm_count), st);
+  return launch_gemm2_one_cta(H_hi, H_lo, gate, ent_pos, W2, s, split, Y, out_direct,
+                              out_direct_f32, err, sm_count, st);
 }
 
 }  // namespace nmoe
