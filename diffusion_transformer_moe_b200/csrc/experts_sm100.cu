@@ -584,14 +584,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
   }
 }
 
-// ---- the down projection on CTA pairs (bf16 intermediates, long expert blocks) ----------
+// ---- the down projection on CTA pairs (long expert blocks) -------------------------------
 //
-// With bf16 H and Y and at least 256 rows per expert, gemm2 runs on pairs of CTAs (a 2-CTA
-// cluster): one tcgen05.mma.cta_group::2 per k-step covers 256 rows of one expert (128
-// from each CTA's shared memory) x N = 256 columns of d, and each CTA stages only half of
-// the W2 tile (128 columns). Per CTA and k-block the ring takes 16 KB of H and 16 KB of W2
-// instead of 16 KB + 32 KB for the same MMA work, so six stages fit. Each CTA's TMEM
-// receives its own 128 rows for all 256 columns, and its epilogue is the one-CTA kernel's.
+// With at least 256 rows per expert, gemm2 runs on pairs of CTAs (a 2-CTA cluster): one
+// tcgen05.mma.cta_group::2 per k-step (two with SPLIT: H hi, then H lo, into one
+// accumulator) covers 256 rows of one expert (128 from each CTA's shared memory) x N = 256
+// columns of d, and each CTA stages only half of the W2 tile (128 columns). Per CTA and
+// k-block the ring takes 16 KB of H (32 KB with SPLIT) and 16 KB of W2 instead of 16 (32) +
+// 32 KB for the same MMA work: six stages fit (four with SPLIT). Each CTA's TMEM receives
+// its own 128 rows for all 256 columns, and its epilogue is the one-CTA kernel's.
 //
 // Barriers: the ring's full barriers live in the leader (rank 0): both CTAs' copies
 // complete on them (cta_group::2) and the leader's producer alone arrives, announcing both
@@ -599,20 +600,29 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
 // arrival is missing). The empty and accumulator-full barriers live in each CTA (the
 // leader's MMA thread commits to both); the accumulator-empty barriers in the leader (all
 // sixteen epilogue warps of the pair arrive). Every wait is bounded.
-constexpr int kPairStages = 6;
-constexpr int kPairABytes = kABytes;                             // 128 rows x 64 K
 constexpr int kPairBBytes = 2 * kBBoxBytes;                      // 128 columns x 64 K
-constexpr int kPairStageBytes = kPairABytes + kPairBBytes;       // 32 KB
 constexpr int kPairEpiWarps = 8;
 constexpr int kPairThreads = 32 * (2 + kPairEpiWarps);
 constexpr int kPairEpiStage = 32 * 128;
-constexpr size_t kPairSmem =
-    (size_t)kPairStages * kPairStageBytes + kPairEpiWarps * kPairEpiStage + 1024;
-static_assert(kPairSmem <= 232448, "dynamic shared memory beyond the 227 KB a CTA may use");
 
+template <bool SPLIT>
+struct PairCfg {
+  static constexpr int kATiles = SPLIT ? 2 : 1;                  // H hi (and H lo)
+  static constexpr int kAStageBytes = kATiles * kABytes;         // 128 rows x 64 K each
+  static constexpr int kStageBytes = kAStageBytes + kPairBBytes;
+  static constexpr int kStages = SPLIT ? 4 : 6;
+  static constexpr size_t kSmem =
+      (size_t)kStages * kStageBytes + kPairEpiWarps * kPairEpiStage + 1024;
+  static_assert(kSmem <= 232448, "dynamic shared memory beyond the 227 KB a CTA may use");
+};
+
+template <bool SPLIT>
 __global__ void __launch_bounds__(kPairThreads, 1)
 pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
+                  const __grid_constant__ CUtensorMap map_hlo,
                   const __grid_constant__ CUtensorMap map_w, const Params p) {
+  using PC = PairCfg<SPLIT>;
+  constexpr int kPairStages = PC::kStages;
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -626,9 +636,9 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
   const uint32_t rank = cluster_ctarank();  // 0: the leader, which issues the MMAs
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nk = (p.K + kBK - 1) / kBK;
-  auto a_tile = [&](int st) { return smem + st * kPairStageBytes; };
-  auto b_tile = [&](int st) { return smem + st * kPairStageBytes + kPairABytes; };
-  uint8_t* const epi_smem = smem + (size_t)kPairStages * kPairStageBytes;
+  auto a_tile = [&](int st, int h) { return smem + st * PC::kStageBytes + h * kABytes; };
+  auto b_tile = [&](int st) { return smem + st * PC::kStageBytes + PC::kAStageBytes; };
+  uint8_t* const epi_smem = smem + (size_t)kPairStages * PC::kStageBytes;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPairStages; ++i) {
@@ -643,6 +653,7 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
     abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&map_h);
+    if (SPLIT) prefetch_tensormap(&map_hlo);
     prefetch_tensormap(&map_w);
   }
   if (warp == 1) tmem_alloc_pair(&tmem_base_sh, kTmemCols);
@@ -661,7 +672,7 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
     for (int item = pair; item < p.num_items; item += npairs) {
       const Tile tl = tile_of(item, p, 256);
       const int nbox = tl.half ? 1 : 2;  // 64-column boxes of this CTA's half of the W2 tile
-      const uint32_t bytes = (uint32_t)(kPairABytes + nbox * kBBoxBytes);
+      const uint32_t bytes = (uint32_t)(PC::kAStageBytes + nbox * kBBoxBytes);
       // tile_of counts row blocks of kBM; a pair item spans two of them
       const int hrow = tl.e * p.Ce + 2 * tl.m0 + (int)rank * kBM;
       const int col0 = tl.n0 + (int)rank * nbox * 64;
@@ -675,7 +686,8 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
         if (lane == 0 && rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * bytes);
         __syncwarp();
         const int k0 = kb * kBK;
-        if (lane == 0) tma_load_2d_pair(a_tile(stage), &map_h, fb, k0, hrow);
+        if (lane == 0) tma_load_2d_pair(a_tile(stage, 0), &map_h, fb, k0, hrow);
+        if (SPLIT && lane == 3) tma_load_2d_pair(a_tile(stage, 1), &map_hlo, fb, k0, hrow);
         if (lane >= 1 && lane <= nbox)
           tma_load_3d_pair(b_tile(stage) + (lane - 1) * kBBoxBytes, &map_w, fb,
                            col0 + 64 * (lane - 1), k0, tl.e, wpol);
@@ -702,9 +714,12 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(smem_u32(a_tile(stage)) + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(smem_u32(b_tile(stage)) + kk * 2048, kBBoxBytes, 1024);
-            mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+#pragma unroll
+            for (int h = 0; h < PC::kATiles; ++h) {
+              const uint64_t ad = sdesc_sw128(smem_u32(a_tile(stage, h)) + kk * 32, 16, 1024);
+              mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk | h) != 0);
+            }
           }
           mma_commit_pair(mapa_shared(&empty_bar[stage], 0));
           mma_commit_pair(mapa_shared(&empty_bar[stage], 1));
@@ -723,7 +738,7 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
     __syncwarp();
   } else {
     // ---------------- epilogue: eight warps per CTA, two per TMEM lane quarter ----------
-    // This CTA's 128 rows of the item, every column; the one-CTA kernel's bf16 path.
+    // This CTA's 128 rows of the item, every column; the one-CTA kernel's paths.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
@@ -754,11 +769,47 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
       const bool direct = pos < 0;   // the token's only entry
       const int64_t orow = (direct ? -pos - 1 : pos) * p.N;
       const float gw = valid ? (p.gate ? p.gate[ent] : 1.f) : 0.f;
+      constexpr int kStep = SPLIT ? 32 : 64;  // columns per round: 128 bytes of the row
 #pragma unroll 1
-      for (int j0 = c_lo; j0 < c_lo + c_n; j0 += 64) {
+      for (int j0 = c_lo; j0 < c_lo + c_n; j0 += kStep) {
         uint32_t y[32], h[32];
         tmem_ld32(taddr + j0, y);
         tmem_ld_wait();
+        if (SPLIT) {
+          // fp32 Y: 32 columns per round through the staging block, 4 rows x 128 bytes per
+          // store
+          float* sb = reinterpret_cast<float*>(sh);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(sb + lane * 32 + ((c ^ (lane & 7)) << 2)) = make_float4(
+                gw * __uint_as_float(y[4 * c]), gw * __uint_as_float(y[4 * c + 1]),
+                gw * __uint_as_float(y[4 * c + 2]), gw * __uint_as_float(y[4 * c + 3]));
+          __syncwarp();
+          const int c = lane & 7;
+          const int col = tl.n0 + j0 + 4 * c;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            const int64_t ro = __shfl_sync(0xffffffffu, orow, r);
+            const int rv = __shfl_sync(0xffffffffu, (int)valid, r);
+            const int rd = __shfl_sync(0xffffffffu, (int)direct, r);
+            float4 v = *reinterpret_cast<const float4*>(sb + r * 32 + ((c ^ (r & 7)) << 2));
+            if (!rv || col >= p.N) continue;
+            if (!rd) {
+              *reinterpret_cast<float4*>(static_cast<float*>(p.out) + ro + col) = v;
+              continue;
+            }
+            // the combine's sum of one term: 0 + y (a -0 becomes +0), rounded once
+            v = make_float4(v.x + 0.f, v.y + 0.f, v.z + 0.f, v.w + 0.f);
+            if (p.out_direct_f32)
+              *reinterpret_cast<float4*>(static_cast<float*>(p.out_direct) + ro + col) = v;
+            else
+              *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out_direct) + ro + col) =
+                  make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+          }
+          __syncwarp();  // the block is read before the next round overwrites it
+          continue;
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           h[i] = pack_bf16x2(gw * __uint_as_float(y[2 * i]), gw * __uint_as_float(y[2 * i + 1]));
@@ -949,16 +1000,17 @@ namespace {
 
 // Pairs of SMs that can hold one pair CTA each at the same time (a pair's two CTAs sit on
 // one TPC): what the occupancy calculator reports for 2-CTA clusters of the pair kernel.
+template <bool SPLIT>
 int pair_slots(int sm_count) {
   static int slots = -1;
   if (slots < 0) {
     int n = 0;
-    if (set_smem_limit(reinterpret_cast<const void*>(pair_gemm2_kernel), kPairSmem) ==
-        cudaSuccess) {
+    if (set_smem_limit(reinterpret_cast<const void*>(pair_gemm2_kernel<SPLIT>),
+                       PairCfg<SPLIT>::kSmem) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3((unsigned)(sm_count & ~1));
       cfg.blockDim = dim3(kPairThreads);
-      cfg.dynamicSmemBytes = kPairSmem;
+      cfg.dynamicSmemBytes = PairCfg<SPLIT>::kSmem;
       cudaLaunchAttribute attr;
       attr.id = cudaLaunchAttributeClusterDimension;
       attr.val.clusterDim.x = 2;
@@ -966,7 +1018,8 @@ int pair_slots(int sm_count) {
       attr.val.clusterDim.z = 1;
       cfg.attrs = &attr;
       cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&n, pair_gemm2_kernel, &cfg) != cudaSuccess) n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, pair_gemm2_kernel<SPLIT>, &cfg) != cudaSuccess)
+        n = 0;
     }
     cudaGetLastError();
     slots = n;
@@ -974,13 +1027,20 @@ int pair_slots(int sm_count) {
   return slots;
 }
 
-cudaError_t launch_gemm2_pair(const void* H, const float* gate, const int32_t* ent_pos,
-                              const void* W2, const Shape& s, void* Y, void* out_direct,
-                              bool out_direct_f32, unsigned* err, int npairs, cudaStream_t st) {
-  CUtensorMap mh, mw;
+int pair_slots(bool split, int sm_count) {
+  return split ? pair_slots<true>(sm_count) : pair_slots<false>(sm_count);
+}
+
+cudaError_t launch_gemm2_pair(const void* H, const void* H_lo, bool split, const float* gate,
+                              const int32_t* ent_pos, const void* W2, const Shape& s, void* Y,
+                              void* out_direct, bool out_direct_f32, unsigned* err, int npairs,
+                              cudaStream_t st) {
+  CUtensorMap mh, mhl, mw;
   const int64_t rows = (int64_t)s.E * s.Ce;
   if (!rows_map(&mh, H, rows, s.F, kBM) || !weight_map(&mw, W2, s.E, s.F, s.d))
     return cudaErrorInvalidValue;
+  if (split && !rows_map(&mhl, H_lo, rows, s.F, kBM)) return cudaErrorInvalidValue;
+  if (!split) mhl = mh;
   Params p;
   p.Ce = s.Ce; p.K = s.F; p.N = s.d;
   p.tiles_m = (int)ceil_div(s.Ce, 2 * kBM);
@@ -995,8 +1055,11 @@ cudaError_t launch_gemm2_pair(const void* H, const float* gate, const int32_t* e
   p.rows_x = s.T;
   p.rows_y = s.y_rows;
   const int pairs = p.num_items < npairs ? p.num_items : npairs;
-  return launch_kernel(pair_gemm2_kernel, dim3((unsigned)(2 * pairs)), dim3(kPairThreads),
-                       kPairSmem, st, s.pdl, 2, mh, mw, p);
+  if (split)
+    return launch_kernel(pair_gemm2_kernel<true>, dim3((unsigned)(2 * pairs)),
+                         dim3(kPairThreads), PairCfg<true>::kSmem, st, s.pdl, 2, mh, mhl, mw, p);
+  return launch_kernel(pair_gemm2_kernel<false>, dim3((unsigned)(2 * pairs)),
+                       dim3(kPairThreads), PairCfg<false>::kSmem, st, s.pdl, 2, mh, mhl, mw, p);
 }
 
 cudaError_t launch_gemm2_one_cta(const void* H_hi, const void* H_lo, const float* gate,
@@ -1029,7 +1092,7 @@ cudaError_t launch_gemm2_one_cta(const void* H_hi, const void* H_lo, const float
 }  // namespace
 
 bool gemm2_sm100_uses_pairs(const Shape& s, bool split, int sm_count) {
-  return !split && s.Ce >= 2 * kBM && s.d % 64 == 0 && pair_slots(sm_count) > 0;
+  return s.Ce >= 2 * kBM && s.d % 64 == 0 && pair_slots(split, sm_count) > 0;
 }
 
 cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* gate,
@@ -1037,8 +1100,8 @@ cudaError_t launch_gemm2_sm100(const void* H_hi, const void* H_lo, const float* 
                                void* Y, void* out_direct, bool out_direct_f32, unsigned* err,
                                int sm_count, cudaStream_t st) {
   if (gemm2_sm100_uses_pairs(s, split, sm_count))
-    return launch_gemm2_pair(H_hi, gate, ent_pos, W2, s, Y, out_direct, out_direct_f32, err,
-                             pair_slots(sm_count), st);
+    return launch_gemm2_pair(H_hi, H_lo, split, gate, ent_pos, W2, s, Y, out_direct,
+                             out_direct_f32, err, pair_slots(split, sm_count), st);
   return launch_gemm2_one_cta(H_hi, H_lo, gate, ent_pos, W2, s, split, Y, out_direct,
                               out_direct_f32, err, sm_count, st);
 }

@@ -21,8 +21,8 @@ cudaError_t launch_gemm1_sm100(const void* x, const int32_t* idx, const void* W1
                                void* H_hi, void* H_lo, const CsrArgs* csr, unsigned* err,
                                int sm_count, cudaStream_t st);
 
-// True when launch_gemm2_sm100 runs this shape on CTA pairs (bf16 intermediates, at least
-// 256 rows per expert, d a multiple of 64, and 2-CTA clusters of the pair kernel fit).
+// True when launch_gemm2_sm100 runs this shape on CTA pairs (at least 256 rows per expert,
+// d a multiple of 64, and 2-CTA clusters of the pair kernel fit).
 bool gemm2_sm100_uses_pairs(const Shape& s, bool split, int sm_count);
 
 // Row e*Ce + s of H W2_e, times gate[e, s], goes to Y row ent_pos[e*Ce + s]; a

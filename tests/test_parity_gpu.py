@@ -133,19 +133,21 @@ def test_output_and_intermediate_options_match_oracle(opts):
     _full_parity(a, 37, "bf16f32" if opts.get("out_f32") else "bf16", opts)
 
 
-# The down projection on CTA pairs (bf16 intermediates, at least 256 rows per expert):
-# pair items of 256 rows x 256 columns, a ragged last row block (Ce not a multiple of
-# 256), a ragged last column block (d not a multiple of 256), and a last wave run as
-# half-width items; bf16 and fp32 outputs (the single-entry rows go to either directly).
+# The down projection on CTA pairs (at least 256 rows per expert; split or bf16
+# intermediates): pair items of 256 rows x 256 columns, a ragged last row block (Ce not a
+# multiple of 256), a ragged last column block (d not a multiple of 256), and a last wave
+# run as half-width items; bf16 and fp32 outputs (the single-entry rows go to either
+# directly).
+@pytest.mark.parametrize("inter", ["split", "bf16"])
 @pytest.mark.parametrize("T,d,E,F,C_,out_f32", [
     (1024, 320, 6, 192, 384, False),     # Ce = 384: the second pair item's rows run out
     (2048, 512, 4, 256, 640, True),      # fp32 output
     (600, 256, 3, 136, 256, False),      # one row block per expert; ragged K
     (2048, 512, 20, 128, 384, False),    # 80 items: 74 whole (N = 256), 12 halves
 ])
-def test_pair_down_projection_matches_oracle(T, d, E, F, C_, out_f32):
+def test_pair_down_projection_matches_oracle(T, d, E, F, C_, out_f32, inter):
     a = I.make_small(T, d, E, F, "bf16", seed=T + d)
-    opts = dict(intermediate="bf16", out_f32=out_f32)
+    opts = dict(intermediate=inter, out_f32=out_f32)
     _full_parity(a, C_, "bf16f32" if out_f32 else "bf16", opts)
 
 
