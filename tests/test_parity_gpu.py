@@ -144,6 +144,9 @@ def test_output_and_intermediate_options_match_oracle(opts):
     (2048, 512, 4, 256, 640, True),      # fp32 output
     (600, 256, 3, 136, 256, False),      # one row block per expert; ragged K
     (2048, 512, 20, 128, 384, False),    # 80 items: 74 whole (N = 256), 12 halves
+    (2048, 256, 4, 192, 1100, False),    # Ce >= 1024: the gate/up GEMM takes two row
+                                         # blocks per item too; its last item's second
+                                         # block runs past Ce
 ])
 def test_pair_down_projection_matches_oracle(T, d, E, F, C_, out_f32, inter):
     a = I.make_small(T, d, E, F, "bf16", seed=T + d)
