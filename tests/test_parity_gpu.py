@@ -571,3 +571,45 @@ def test_bf16_intermediates_full_workload(name):
     assert rel <= BF16_REL
     if not w.lognormal_scale:
         assert mx <= BF16_ABS
+
+
+# -- the layer inside a CUDA graph -------------------------------------------------------------
+
+@pytest.mark.parametrize("inter", ["split", "bf16"])
+@pytest.mark.parametrize("T,d,E,F,C_", [
+    (8192, 2048, 64, 1024, 128),     # the 1024 px layer: one-CTA GEMMs, ring combine
+    (2048, 256, 4, 192, 1100),       # large experts: pair down GEMM, two row blocks per
+                                     # gate/up item, register combine
+])
+def test_captured_graph_replays_the_direct_call(T, d, E, F, C_, inter):
+    """After one direct call (the library's one-time setup, which a stream capture may not
+    contain), the layer captured into a CUDA graph — programmatic dependent launches and
+    2-CTA clusters included — replays to the direct call's output bit for bit."""
+    a = I.make_small(T, d, E, F, "bf16", seed=T + E)
+    dev = {k: v.cuda() for k, v in a.items()}
+    ws = torch.empty(nm.workspace_size(T, d, E, F, C_, intermediate=inter), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+
+    def call():
+        nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], C_, out=out,
+                   workspace=ws, intermediate=inter)
+
+    call()
+    torch.cuda.synchronize()
+    want = out.clone()
+    out.zero_()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            call()
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, want)
+    assert nm.get_last_error() == 0
+    del g
