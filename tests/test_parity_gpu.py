@@ -248,6 +248,29 @@ def test_repeated_calls_with_and_without_stage_events_stay_clean():
             assert torch.equal(out, ref)
 
 
+@pytest.mark.parametrize("inter", ["split", "bf16"])
+def test_repeated_large_expert_calls_stay_clean(inter):
+    # the pair down GEMM and the two-row-block gate/up GEMM (Ce = 1100), back to back
+    # (programmatic dependent launch) and with events between the stages: no bounded wait
+    # may run out, and every call gives the same output
+    T, d, E, F, C_ = 2048, 256, 4, 192, 1100
+    a = I.make_small(T, d, E, F, "bf16", seed=5)
+    dev = {k: v.cuda() for k, v in a.items()}
+    ws = torch.empty(nm.workspace_size(T, d, E, F, C_, intermediate=inter), dtype=torch.uint8,
+                     device="cuda")
+    ref = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], C_, workspace=ws,
+                     intermediate=inter)
+    torch.cuda.synchronize()
+    for traced in (False, True):
+        for _ in range(12):
+            tr = nm.Trace(1) if traced else None
+            out = nm.forward(dev["x"], dev["W_r"], dev["W1"], dev["W3"], dev["W2"], C_,
+                             workspace=ws, intermediate=inter, trace=tr)
+            torch.cuda.synchronize()
+            assert nm.get_last_error() == 0
+            assert torch.equal(out, ref)
+
+
 def test_tensor_core_path_launches_five_kernels():
     # router, select, gate/up GEMM (which also builds the token lists), down GEMM, combine
     assert nm.kernels_per_call(8192, 2048, 64, 1024, 128) == 5
