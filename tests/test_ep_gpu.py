@@ -54,6 +54,8 @@ def _emulated_ep(dev, C_, E, world, n_segments=1, exact=False):
     ("bf16", 1024, 256, 8, 256, 128, 1),     # tensor-core path
     ("bf16", 768, 136, 6, 200, 100, 2),      # ragged sizes, selection per segment
     ("f32", 256, 128, 6, 96, 40, 1),         # CUDA-core path
+    ("bf16", 2048, 256, 8, 192, 384, 1),     # the pair down GEMM on each rank's experts
+    ("bf16", 2048, 256, 4, 192, 1100, 1),    # and two row blocks per gate/up item
 ])
 def test_expert_parallel_equals_one_gpu(world, dtype, T, d, E, F, C_, nseg, exact):
     a = I.make_small(T, d, E, F, dtype, seed=T + E)
