@@ -38,6 +38,10 @@
 // and returns.
 #include <cudaTypedefs.h>
 
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include "csr_block.cuh"
 #include "experts_sm100.cuh"
 #include "sm100_ptx.cuh"
@@ -928,16 +932,7 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
 // ---- host side ----------------------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
-  return fn;
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
 }
 
 // bf16 tensor map with 128-byte swizzle. dims/box are innermost first; strides are the
@@ -1054,29 +1049,39 @@ namespace {
 // one TPC): what the occupancy calculator reports for 2-CTA clusters of the pair kernel.
 template <bool SPLIT>
 int pair_slots(int sm_count) {
-  static int slots = -1;
-  if (slots < 0) {
-    int n = 0;
-    if (set_smem_limit(reinterpret_cast<const void*>(pair_gemm2_kernel<SPLIT>),
-                       PairCfg<SPLIT>::kSmem) == cudaSuccess) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)(sm_count & ~1));
-      cfg.blockDim = dim3(kPairThreads);
-      cfg.dynamicSmemBytes = PairCfg<SPLIT>::kSmem;
-      cudaLaunchAttribute attr;
-      attr.id = cudaLaunchAttributeClusterDimension;
-      attr.val.clusterDim.x = 2;
-      attr.val.clusterDim.y = 1;
-      attr.val.clusterDim.z = 1;
-      cfg.attrs = &attr;
-      cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&n, pair_gemm2_kernel<SPLIT>, &cfg) != cudaSuccess)
-        n = 0;
-    }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
     cudaGetLastError();
-    slots = n;
+    return 0;
   }
-  return slots;
+  static std::mutex mu;
+  static std::vector<std::pair<int, int>> cache;  // (device, slots)
+  std::lock_guard<std::mutex> lk(mu);
+  for (const auto& c : cache)
+    if (c.first == dev) return c.second;
+  int n = 0;
+  if (set_smem_limit(reinterpret_cast<const void*>(pair_gemm2_kernel<SPLIT>),
+                     PairCfg<SPLIT>::kSmem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sm_count & ~1));
+    cfg.blockDim = dim3(kPairThreads);
+    cfg.dynamicSmemBytes = PairCfg<SPLIT>::kSmem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, pair_gemm2_kernel<SPLIT>, &cfg) != cudaSuccess) {
+      cudaGetLastError();  // no pair slots: the one-CTA kernel runs instead
+      n = 0;
+    }
+  } else {
+    cudaGetLastError();
+  }
+  cache.emplace_back(dev, n);
+  return n;
 }
 
 int pair_slots(bool split, int sm_count) {

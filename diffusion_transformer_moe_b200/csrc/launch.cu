@@ -1,4 +1,6 @@
 // Host-side launch helpers shared by the kernels of libnmoe.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 #include <vector>
 
@@ -32,6 +34,23 @@ cudaError_t set_smem_limit(const void* kernel, size_t bytes) {
     }
   g_smem.push_back({kernel, dev, bytes});
   return cudaSuccess;
+}
+
+void* tensor_map_encoder() {
+  // looked up once; a function-local static is initialised exactly once, even when
+  // several host threads make their first call at the same time
+  static void* const fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();  // the failed query is not the caller's error
+      f = nullptr;
+    }
+    return f;
+  }();
+  return fn;
 }
 
 }  // namespace nmoe

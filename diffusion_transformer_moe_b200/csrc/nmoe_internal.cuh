@@ -50,6 +50,10 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // shared memory goes through here, not only those asking for more than 48 KB.
 cudaError_t set_smem_limit(const void* kernel, size_t bytes);
 
+// The driver's cuTensorMapEncodeTiled (cast to its PFN type by the caller), or NULL when the
+// driver does not provide it; looked up once per process, safe from several host threads.
+void* tensor_map_encoder();
+
 // Launch with programmatic stream serialization (pdl) and an optional 1-D cluster.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
