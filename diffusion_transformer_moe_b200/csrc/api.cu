@@ -343,6 +343,9 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
            : nmoe::launch_gemm2_simt(H, gate + eoff, W2, ent_pos + eoff, sl, o.dtype, split,
                                      y_f32, Y, st);
   mark(5);
+  // the tensor-core down GEMM signals the combine only after its own wait (see
+  // nmoe_internal.cuh), so the combine may read the token lists before its wait
+  s.after_gemm2 = s.pdl && tc && run_experts;
   if (e == cudaSuccess && !o.skip_combine)
     e = nmoe::launch_combine(Y, tok_ptr, s, y_f32, out_f32, outd, o.residual, !f32, o.gate2,
                              direct, ds->err, ds->sm_count, st);

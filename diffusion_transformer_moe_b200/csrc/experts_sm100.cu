@@ -179,7 +179,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                     const Params p) {
   using C = Cfg<MODE, SPLIT, GATHER, MT>;
   constexpr int kStages = C::kStages;
-  pdl_launch_dependents();
+  if (MODE != kGemm2) pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -219,6 +219,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
   const uint32_t tmem_base = tmem_base_sh;
   volatile int* abort_v = &abort_flag;
   pdl_wait();  // the previous kernel's outputs (idx, x or H, gate) are complete
+  // the down GEMM lets the next kernel start only now: everything before it is complete
+  if (MODE == kGemm2) pdl_launch_dependents();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -670,7 +672,6 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
                   const __grid_constant__ CUtensorMap map_w, const Params p) {
   using PC = PairCfg<SPLIT>;
   constexpr int kPairStages = PC::kStages;
-  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -710,6 +711,7 @@ pair_gemm2_kernel(const __grid_constant__ CUtensorMap map_h,
   const uint32_t tmem_base = tmem_base_sh;
   volatile int* abort_v = &abort_flag;
   pdl_wait();  // the previous kernel's outputs (H, gate, ent_pos) are complete
+  pdl_launch_dependents();  // after the wait, as in the one-CTA down GEMM
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------

@@ -38,7 +38,11 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 // Programmatic dependent launch. Every kernel of the layer lets the next kernel on the
 // stream start its prologue early (launch_dependents, issued by every thread at entry)
-// and waits for the previous grid's memory (wait) before its first global access.
+// and waits for the previous grid's memory (wait) before its first global access. The
+// tensor-core down GEMM is the exception: it issues launch_dependents only after its own
+// wait, so the kernel after it starts only once every earlier kernel of the call (and
+// whatever ran before the call) has completed, and may read their outputs before its own
+// wait (the combine reads its token lists there).
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -101,6 +105,9 @@ struct Shape {
   bool pdl;      // launch with programmatic dependent launch
   uint64_t wait_ns;  // budget of each bounded device-side wait (nmoe_options)
   int64_t y_rows;    // rows of the layer's Y (all experts' entries, plus the shared rows)
+  // The previous launch on the stream is the tensor-core down GEMM with programmatic
+  // dependent launch (it signals its dependents only after its own wait).
+  bool after_gemm2 = false;
 };
 
 // Budget of a device-side wait when the caller sets none: far beyond any wait of a
