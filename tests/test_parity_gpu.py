@@ -179,6 +179,13 @@ def test_segments_not_aligned_to_token_blocks(dtype):
     _full_parity(a, 20, dtype, dict(n_segments=3))
 
 
+def test_long_segments_not_aligned_to_token_blocks():
+    # 3 segments of 4100 tokens: the selection's block boundary table, which the gate/up
+    # GEMM's token lists read, across segment edges that fall inside 32-token blocks
+    a = I.make_small(12300, 64, 6, 64, "bf16", seed=29)
+    _full_parity(a, 40, "bf16", dict(n_segments=3))
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_router_bias_matches_oracle(dtype):
     a = I.make_small(192, 64, 6, 64, dtype, seed=22)
@@ -382,6 +389,38 @@ def test_select_edge_sizes(T, E, C_, nseg):
     ptr, ent = O.token_lists(want, T)
     assert np.array_equal(tok_ptr.cpu().numpy(), ptr)
     assert np.array_equal(tok_ent.cpu().numpy(), ent)
+
+
+@pytest.mark.parametrize("S,E,C_,nseg,tie", [
+    (8192, 4, 5300, 1, 0.0),     # the threshold's bin holds a few hundred keys or fewer
+    (8192, 3, 128, 1, 0.0),      # ~700 keys in the bin: two more digits over the list
+    (10007, 5, 77, 1, 0.0),      # odd row length
+    (4100, 6, 1, 3, 0.0),        # capacity 1; segments that do not start on a 32-token block
+    (4096, 2, 4096, 2, 0.0),     # every key chosen
+    (12000, 4, 6000, 1, 0.5),    # half the keys tie at the threshold: too many to list
+    (9000, 3, 4500, 1, 0.05),    # ties inside a listed bin
+])
+def test_select_long_rows_match_oracle(S, E, C_, nseg, tie):
+    """Long rows staged in shared memory, down every path of the radix select (ranked
+    candidates, two more digits over the candidate list, a bin too large to list, every
+    key chosen), against the oracle, bit-exact, token lists included."""
+    g = torch.Generator().manual_seed(S + C_)
+    T = S * nseg
+    p = torch.rand(T, E, generator=g)
+    if tie > 0:
+        p[torch.rand(T, E, generator=g) < tie] = 0.5
+    scores_t = p.t().contiguous().cuda()
+    idx, gate, tok_ptr, tok_ent = nm.select(scores_t, C_, n_segments=nseg)
+    torch.cuda.synchronize()
+    want = O.select(p.numpy(), C_, nseg)
+    assert np.array_equal(idx.cpu().numpy(), want)
+    ptr, ent = O.token_lists(want, T)
+    assert np.array_equal(tok_ptr.cpu().numpy(), ptr)
+    assert np.array_equal(tok_ent.cpu().numpy(), ent)
+    np.testing.assert_array_equal(
+        gate.cpu().numpy(),
+        np.stack([p.numpy()[want[e], e] for e in range(E)]))
+    assert nm.get_last_error() == 0
 
 
 _FRESH_SELECT = """
