@@ -293,7 +293,8 @@ nmoe_status forward_impl(const void* x, const void* W_r, const void* W1, const v
                                    scores_t, st);
   }
   mark(1);
-  if (e == cudaSuccess) e = nmoe::launch_select(scores_t, s, idx, gate, bnd, ds->err, st);
+  if (e == cudaSuccess)
+    e = nmoe::launch_select(scores_t, s, idx, gate, bnd, ds->err, ds->sm_count, st);
   mark(2);
   // the expert GEMMs cover experts [e_lo, e_hi): their slice of idx, gate and ent_pos
   Shape sl = s;
@@ -440,7 +441,7 @@ nmoe_status nmoe_select(const float* scores_t, int64_t T, int64_t E, int64_t C,
   const Shape s = make_shape(T, 8, E, 8, C, n_segments);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // no scratch here: the CSR build searches idx instead of reading a boundary table
-  cudaError_t e = nmoe::launch_select(scores_t, s, idx, gate, nullptr, ds->err, st);
+  cudaError_t e = nmoe::launch_select(scores_t, s, idx, gate, nullptr, ds->err, ds->sm_count, st);
   if (e == cudaSuccess && tok_ptr)
     e = nmoe::launch_csr(idx, nullptr, s, false, tok_ptr, tok_ent, nullptr, gate,
                          NMOE_COMBINE_RAW, 1.f, false, ds->err, st);

@@ -128,7 +128,7 @@ constexpr int kSelectMaxRow = 1 << 19;
 // comes before the block; select_bound_entries(s) int32 entries.
 size_t select_bound_entries(const Shape& s);
 cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, float* gate,
-                          int32_t* bnd, unsigned* err, cudaStream_t st);
+                          int32_t* bnd, unsigned* err, int sm_count, cudaStream_t st);
 
 // bnd: the table launch_select wrote, or NULL to search idx instead.
 // combine == NMOE_COMBINE_NORMALIZED rewrites gate[] in place to

@@ -146,10 +146,12 @@ __device__ __forceinline__ void find_digit(const unsigned* hist, unsigned k, uns
   }
 }
 
-// Two CTAs per SM (32 registers a thread, no spills): more rows than SMs (the model
-// default shape's 128 experts x 2 segments) run in one wave, not two (its selection
-// 22.6 -> 19.2 us traced, interleaved A/B; no change where rows <= SMs).
-__global__ void __launch_bounds__(kSelThreads, 2)
+// MIN_CTAS = 2 (32 registers a thread, no spills) fits two CTAs on an SM, for calls with
+// more rows than SMs (the model default shape's 128 experts x 2 segments run in one wave,
+// not two: its selection 22.6 -> 19.2 us traced, interleaved A/B); with fewer rows the
+// one-CTA build (more registers) runs.
+template <int MIN_CTAS>
+__global__ void __launch_bounds__(kSelThreads, MIN_CTAS)
 select_kernel(const float* __restrict__ scores_t, int64_t Tn, int S, int C, int Ce, int E,
               int cached, int32_t* __restrict__ idx, float* __restrict__ gate,
               int32_t* __restrict__ bnd, unsigned* __restrict__ err) {
@@ -443,14 +445,16 @@ size_t select_bound_entries(const Shape& s) {
 }
 
 cudaError_t launch_select(const float* scores_t, const Shape& s, int32_t* idx, float* gate,
-                          int32_t* bnd, unsigned* err, cudaStream_t st) {
+                          int32_t* bnd, unsigned* err, int sm_count, cudaStream_t st) {
   if (s.S > kSelectMaxRow) return cudaErrorInvalidValue;
   const int cached = s.S <= kSelMaxCached;
   const size_t nw4 = (size_t)((ceil_div(s.S, 32) + 3) & ~3);
   const size_t smem = sizeof(uint32_t) * ((cached ? (size_t)((s.S + 3) & ~3) : 0) + 2 * nw4 +
                                           (size_t)kCandMax);
   dim3 grid((unsigned)s.E, (unsigned)s.n_seg);
-  return launch_kernel(select_kernel, grid, dim3(kSelThreads), smem, st, s.pdl, 1, scores_t,
+  const bool two = (int64_t)s.E * s.n_seg > sm_count;
+  return launch_kernel(two ? select_kernel<2> : select_kernel<1>, grid, dim3(kSelThreads), smem,
+                       st, s.pdl, 1, scores_t,
                        (int64_t)s.T, s.S, s.C, s.Ce, s.E, cached, idx, gate, bnd, err);
 }
 
