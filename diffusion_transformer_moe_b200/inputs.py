@@ -88,6 +88,11 @@ WORKLOADS = {
         # width 1344, capacity factor 8) on a 1024 px CFG pair, selection per image
         Workload("model_default_1024px_cfg", T=8192, d=2048, E=128, F=1344,
                  capacity_factor=8, dtype="bf16", segments=2),
+        # the batch-4 layer's expert GEMM shapes (2048 rows per expert, d = 3072, F = 1536)
+        # with 16 experts instead of 64: the same kernels in ~1 GB of device memory, the
+        # size for a full ncu capture of the tensor-bound GEMMs
+        Workload("batch4_16experts", T=8192, d=3072, E=16, F=1536, capacity_factor=4,
+                 dtype="bf16"),
     )
 }
 
