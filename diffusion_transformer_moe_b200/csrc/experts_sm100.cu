@@ -36,6 +36,16 @@
 // is MN-major; both use the 128-byte swizzle. Every wait is bounded; a wait that runs
 // out sets the device error word and the kernel drains its copies and MMAs, frees TMEM
 // and returns.
+//
+// Larger experts take two variants:
+// * 1024 or more rows per expert: each gate/up work item covers two 128-row blocks that
+//   share every weight tile (MT = 2). Both accumulators then belong to one item, so they
+//   are not double-buffered across items.
+// * 256 or more rows per expert: the down projection runs on 2-CTA clusters
+//   (pair_gemm2_kernel). One tcgen05.mma.cta_group::2 covers M = 256 rows, and each CTA
+//   stages its own 128 H rows and half of the W2 tile.
+// Both down GEMMs issue griddepcontrol.launch_dependents only after their own wait, so the
+// combine after them may read the token lists early.
 #include <cudaTypedefs.h>
 
 #include <mutex>
